@@ -1,0 +1,169 @@
+/*
+ * muon.h — C ABI of libmuon, a B200 (sm_100a) implementation of the Muon
+ * optimizer step for matrix parameters.
+ *
+ * Method: "Muon is Scalable for LLM Training" (Moonlight technical report,
+ * Liu et al. 2025), Section 2:
+ *   - Sec. 2.1, Eq. 1 and the paragraph after it: momentum M_t = mu M_{t-1} + G_t
+ *     with M_0 = 0, and the Nesterov-style input Y = mu M_t + G_t;
+ *   - Sec. 2.1, Eq. 2: Newton-Schulz on X_0 = Y / ||Y||_F with the quintic
+ *     iteration X_k = a X + b (X X^T) X + c (X X^T)^2 X;
+ *   - Sec. 2.2, Eq. 3 and Eq. 4 (= Sec. 3.1, Eq. 7): the decoupled, shape-scaled
+ *     update W_t = W_{t-1} - eta (rms_scale sqrt(max(A,B)) O_t + lambda W_{t-1});
+ *   - Sec. 2.3, Algorithm 1, last line: the logged update RMS sqrt(mean(u^2)).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are dense, row-major, contiguous, and live in device memory
+ *     of the device that is current when the plan is created.  "Host" arrays
+ *     (descriptor lists, coefficient triples) are read before the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; no entry point synchronizes
+ *     the host except muon_get_status and muon_profile_read, which say so.
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     error return means nothing was launched and no tensor was modified.
+ *   - A plan is not thread-safe: calls on one plan must be serialized by the
+ *     caller and enqueued on streams that are ordered with each other.
+ */
+#ifndef MUON_H_
+#define MUON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad enum, non-finite hyper-parameter */
+  MUON_ERR_SHAPE_MISMATCH = 2, /* descriptor count or shapes differ from the plan */
+  MUON_ERR_UNSUPPORTED = 3,    /* request the plan was not built for (e.g. fp32 path without MUON_INIT_FP32_NS) */
+  MUON_ERR_NO_MEMORY = 4,      /* device or pinned-host allocation failed in muon_init */
+  MUON_ERR_CUDA = 5,           /* a CUDA call or launch failed */
+  MUON_ERR_NONFINITE = 6,      /* (muon_get_status) a Frobenius norm was NaN or Inf */
+  MUON_ERR_TIMEOUT = 7,        /* (muon_get_status) a device-side wait gave up; results of that call are invalid */
+  MUON_ERR_ALIAS = 8           /* W, G, M (or X_in, O_out) buffers overlap */
+} muon_status_t;
+
+typedef enum { MUON_DT_BF16 = 0, MUON_DT_FP32 = 1 } muon_dtype_t;
+
+/* Arithmetic of the Newton-Schulz products.
+ *   MUON_NS_BF16: bf16 operands, fp32 accumulation on the tensor cores (tcgen05),
+ *                 iterate X carried between iterations as a bf16 hi/lo pair
+ *                 (about 16 significant bits).  The production path.
+ *   MUON_NS_FP32: fp32 operands and fp32 products on the CUDA cores; a
+ *                 validation path, needs MUON_INIT_FP32_NS at plan creation. */
+typedef enum { MUON_NS_BF16 = 0, MUON_NS_FP32 = 1 } muon_ns_precision_t;
+
+/* muon_init flags */
+#define MUON_INIT_ZERO_MOMENTUM 0x1u /* zero every M on `stream` (M_0 = 0, Sec. 2.1) */
+#define MUON_INIT_FP32_NS       0x2u /* also reserve the workspace of the fp32 path */
+
+/* One matrix parameter.  Shape [rows, cols]; for muon_init only the shape is
+ * kept (pointers may be NULL unless MUON_INIT_ZERO_MOMENTUM is given), for
+ * muon_step every pointer is used and may differ from call to call. */
+typedef struct {
+  float*      W;        /* fp32 [rows, cols], updated in place                     */
+  const void* G;        /* gradient [rows, cols], dtype g_dtype, read only          */
+  float*      M;        /* fp32 momentum [rows, cols], updated in place            */
+  int64_t     rows;     /* A in Lemma 1; 1 <= rows <= 65536                         */
+  int64_t     cols;     /* B in Lemma 1; 1 <= cols <= 65536                         */
+  int32_t     g_dtype;  /* muon_dtype_t                                              */
+  int32_t     reserved; /* must be 0                                                 */
+} muon_param_t;
+
+/* Per-call hyper-parameters (all finite). */
+typedef struct {
+  float   lr;            /* eta_t, the learning rate of this step (schedule is the caller's) */
+  float   weight_decay;  /* lambda (Eq. 3)                                                     */
+  float   momentum;      /* mu (Eq. 1)                                                         */
+  int32_t ns_steps;      /* N, 0..32 (N = 0 gives O = Y / ||Y||_F)                              */
+  float   a, b, c;       /* quintic coefficients of Eq. 2                                      */
+  float   rms_scale;     /* the 0.2 of Eq. 4                                                   */
+  int32_t nesterov;      /* 1: Newton-Schulz input mu M_t + G_t; 0: M_t (plain Eq. 1)          */
+  int32_t ns_precision;  /* muon_ns_precision_t                                                */
+} muon_hparams_t;
+
+typedef struct muon_plan_s* muon_plan_t;
+
+/* Fill `hp` with the pages' values: lr 4.2e-4 (Sec. 3.3 peak), weight_decay 0.1
+ * (Sec. 3.3), momentum 0.95, ns_steps 5 (Sec. 2.2), (a, b, c) =
+ * (3.4445, -4.7750, 2.0315) (Sec. 2.1), rms_scale 0.2 (Eq. 4), nesterov 1,
+ * ns_precision MUON_NS_BF16.  Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
+MUON_API muon_status_t muon_hparams_default(muon_hparams_t* hp);
+
+/* Build a plan for `n` matrices with the shapes in params[0..n).  The plan
+ * owns its device workspace (see muon_workspace_bytes), tile and chunk
+ * schedules and TMA descriptors; shapes and count are fixed for its lifetime.
+ * With MUON_INIT_ZERO_MOMENTUM the M buffers are zeroed on `stream`.
+ * The current CUDA device must be an sm_100 part.
+ * Errors: INVALID_ARG (out/params NULL, n < 1, shape out of range, reserved != 0,
+ * M NULL with ZERO_MOMENTUM), UNSUPPORTED (device is not sm_100), NO_MEMORY, CUDA.
+ * On error *out is set to NULL and nothing is allocated. */
+MUON_API muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags,
+                        void* stream);
+
+/* One Muon step over all n matrices of the plan (n and every shape must equal
+ * the plan's):  M <- mu M + G;  Y = mu M + G (or M);  O = Newton-Schulz(Y) with
+ * N = hp->ns_steps in the wide orientation (a matrix with rows > cols is
+ * treated as its transpose; no data is transposed);  W <- W - lr (rms_scale
+ * sqrt(max(rows, cols)) O + weight_decay W).  A matrix whose Y is exactly 0
+ * gets O = 0 (pure weight decay).  If update_rms is not NULL it receives, on
+ * the device, n floats sqrt(mean(O^2)) in descriptor order.
+ * W, G, M of all descriptors must be pairwise disjoint.
+ * Errors: INVALID_ARG, SHAPE_MISMATCH, ALIAS, UNSUPPORTED, CUDA.  Non-finite
+ * norms and device-side timeouts are reported later by muon_get_status. */
+MUON_API muon_status_t muon_step(muon_plan_t plan, const muon_param_t* params, int32_t n, const muon_hparams_t* hp,
+                        float* update_rms, void* stream);
+
+/* Newton-Schulz only (no momentum, no weight update) for all n matrices of
+ * the plan: O_out[i] = Newton-Schulz(X_in[i]) with ns_steps iterations of
+ * Eq. 2 and coefficients abc[0..2].  X_in[i] has the plan's i-th shape and
+ * dtype in_dtype; O_out[i] is fp32 of the same shape.  X_in and O_out are
+ * host arrays of n device pointers; no input may overlap an output.
+ * Errors: INVALID_ARG, ALIAS, UNSUPPORTED, CUDA. */
+MUON_API muon_status_t muon_orthogonalize(muon_plan_t plan, const void* const* X_in, float* const* O_out, int32_t n,
+                                 int32_t in_dtype, int32_t ns_steps, const float abc[3], int32_t ns_precision,
+                                 void* stream);
+
+/* Device bytes owned by the plan (workspace, schedules, descriptors). 0 for NULL. */
+MUON_API size_t muon_workspace_bytes(muon_plan_t plan);
+
+/* Synchronizes the plan's last stream, returns the sticky device status of all
+ * calls since the previous muon_get_status (MUON_OK, MUON_ERR_TIMEOUT or
+ * MUON_ERR_NONFINITE; TIMEOUT wins) and clears it.  CUDA errors: MUON_ERR_CUDA. */
+MUON_API muon_status_t muon_get_status(muon_plan_t plan);
+
+/* Release everything the plan owns.  Synchronizes the plan's last stream
+ * first.  NULL is a no-op. */
+MUON_API void muon_destroy(muon_plan_t plan);
+
+/* Static English text for a status code (never NULL). */
+MUON_API const char* muon_status_string(muon_status_t s);
+
+/* Phase timing, for measurement.  When enabled, every step/orthogonalize call
+ * records CUDA events on its stream at each phase boundary.  Phases:
+ * 0 momentum/normalise, 1 Gram (X X^T), 2 polynomial (b A + c A^2),
+ * 3 X update (a X + B X, includes the fused weight update of the last
+ * iteration), 4 stand-alone update and RMS finalisation. */
+#define MUON_NUM_PHASES 5
+MUON_API muon_status_t muon_profile_enable(muon_plan_t plan, int32_t enable);
+
+/* Synchronizes, then adds the elapsed milliseconds of every recorded call
+ * since the last read into phase_ms[MUON_NUM_PHASES] and the launch counts
+ * into launches[MUON_NUM_PHASES] (both zeroed by the caller), writes the
+ * number of calls into *calls, and resets the record. */
+MUON_API muon_status_t muon_profile_read(muon_plan_t plan, double* phase_ms, int64_t* launches, int32_t* calls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_H_ */

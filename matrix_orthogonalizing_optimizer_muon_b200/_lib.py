@@ -1,0 +1,153 @@
+"""ctypes binding of libmuon's C ABI (include/muon.h).
+
+Argument marshalling only: every step of the optimizer runs in the library's
+CUDA kernels.  The functions keep the C names; ``load()`` raises if the
+shared library has not been built, so nothing can silently fall back to
+another implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so")
+
+MUON_OK = 0
+MUON_ERR_INVALID_ARG = 1
+MUON_ERR_SHAPE_MISMATCH = 2
+MUON_ERR_UNSUPPORTED = 3
+MUON_ERR_NO_MEMORY = 4
+MUON_ERR_CUDA = 5
+MUON_ERR_NONFINITE = 6
+MUON_ERR_TIMEOUT = 7
+MUON_ERR_ALIAS = 8
+
+MUON_DT_BF16 = 0
+MUON_DT_FP32 = 1
+MUON_NS_BF16 = 0
+MUON_NS_FP32 = 1
+MUON_INIT_ZERO_MOMENTUM = 0x1
+MUON_INIT_FP32_NS = 0x2
+MUON_NUM_PHASES = 5
+PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
+
+EXPORTED = ("muon_hparams_default", "muon_init", "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
+            "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read")
+
+
+class muon_param_t(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("G", ctypes.c_void_p), ("M", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("g_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class muon_hparams_t(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("weight_decay", ctypes.c_float), ("momentum", ctypes.c_float),
+                ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float), ("b", ctypes.c_float),
+                ("c", ctypes.c_float), ("rms_scale", ctypes.c_float), ("nesterov", ctypes.c_int32),
+                ("ns_precision", ctypes.c_int32)]
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libmuon.so (once).  Raises if it was not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libmuon.so not found at {LIB_PATH}; build it with "
+                           "`python -m matrix_orthogonalizing_optimizer_muon_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    lib.muon_hparams_default.argtypes = [ctypes.POINTER(muon_hparams_t)]
+    lib.muon_hparams_default.restype = ctypes.c_int
+    lib.muon_init.argtypes = [ctypes.POINTER(P), ctypes.POINTER(muon_param_t), ctypes.c_int32, ctypes.c_uint32, P]
+    lib.muon_init.restype = ctypes.c_int
+    lib.muon_step.argtypes = [P, ctypes.POINTER(muon_param_t), ctypes.c_int32, ctypes.POINTER(muon_hparams_t), P, P]
+    lib.muon_step.restype = ctypes.c_int
+    lib.muon_orthogonalize.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.POINTER(ctypes.c_float), ctypes.c_int32, P]
+    lib.muon_orthogonalize.restype = ctypes.c_int
+    lib.muon_workspace_bytes.argtypes = [P]
+    lib.muon_workspace_bytes.restype = ctypes.c_size_t
+    lib.muon_get_status.argtypes = [P]
+    lib.muon_get_status.restype = ctypes.c_int
+    lib.muon_destroy.argtypes = [P]
+    lib.muon_destroy.restype = None
+    lib.muon_status_string.argtypes = [ctypes.c_int]
+    lib.muon_status_string.restype = ctypes.c_char_p
+    lib.muon_profile_enable.argtypes = [P, ctypes.c_int32]
+    lib.muon_profile_enable.restype = ctypes.c_int
+    lib.muon_profile_read.argtypes = [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                                      ctypes.POINTER(ctypes.c_int32)]
+    lib.muon_profile_read.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().muon_status_string(int(status)).decode()
+
+
+def check(status: int, where: str) -> None:
+    if status != MUON_OK:
+        raise MuonError(status, where)
+
+
+# ------------------------------------------------------------------ same-name wrappers
+
+def muon_hparams_default() -> muon_hparams_t:
+    hp = muon_hparams_t()
+    check(load().muon_hparams_default(ctypes.byref(hp)), "muon_hparams_default")
+    return hp
+
+
+def muon_init(params, n: int, flags: int, stream: int) -> ctypes.c_void_p:
+    plan = ctypes.c_void_p()
+    check(load().muon_init(ctypes.byref(plan), params, int(n), int(flags), ctypes.c_void_p(stream)), "muon_init")
+    return plan
+
+
+def muon_step(plan, params, n: int, hp: muon_hparams_t, update_rms_ptr: int | None, stream: int) -> None:
+    check(load().muon_step(plan, params, int(n), ctypes.byref(hp), ctypes.c_void_p(update_rms_ptr or 0),
+                           ctypes.c_void_p(stream)), "muon_step")
+
+
+def muon_orthogonalize(plan, x_ptrs, o_ptrs, n: int, in_dtype: int, ns_steps: int, abc, precision: int,
+                       stream: int) -> None:
+    abc_arr = (ctypes.c_float * 3)(*[float(v) for v in abc])
+    check(load().muon_orthogonalize(plan, x_ptrs, o_ptrs, int(n), int(in_dtype), int(ns_steps), abc_arr,
+                                    int(precision), ctypes.c_void_p(stream)), "muon_orthogonalize")
+
+
+def muon_workspace_bytes(plan) -> int:
+    return int(load().muon_workspace_bytes(plan))
+
+
+def muon_get_status(plan) -> int:
+    return int(load().muon_get_status(plan))
+
+
+def muon_destroy(plan) -> None:
+    load().muon_destroy(plan)
+
+
+def muon_profile_enable(plan, enable: bool) -> None:
+    check(load().muon_profile_enable(plan, 1 if enable else 0), "muon_profile_enable")
+
+
+def muon_profile_read(plan):
+    ms = (ctypes.c_double * MUON_NUM_PHASES)()
+    cnt = (ctypes.c_int64 * MUON_NUM_PHASES)()
+    calls = ctypes.c_int32()
+    check(load().muon_profile_read(plan, ms, cnt, ctypes.byref(calls)), "muon_profile_read")
+    return list(ms), list(cnt), int(calls.value)

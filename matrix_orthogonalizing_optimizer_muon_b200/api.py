@@ -1,0 +1,149 @@
+"""Python front-end of libmuon over torch tensors.
+
+PyTorch provides device memory and streams only; ``MuonPlan`` passes raw
+pointers, shapes and the current CUDA stream to the C ABI.
+
+    plan = MuonPlan([W.shape for W in weights], zero_momentum_of=[M...])
+    plan.step(list(zip(weights, grads, moms)), lr=4.2e-4, weight_decay=0.1)
+
+Matrices only: the hybrid split of "Muon is Scalable for LLM Training"
+(Sec. 2.2) sends 1-D parameters, embeddings and the LM head to AdamW, which is
+the caller's business.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib as L
+
+DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _check_tensor(t: torch.Tensor, dtype, name: str, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+_GDT = {torch.bfloat16: L.MUON_DT_BF16, torch.float32: L.MUON_DT_FP32}
+
+
+class MuonPlan:
+    """A libmuon plan for a fixed list of matrix shapes on the current device."""
+
+    def __init__(self, shapes, *, momenta=None, fp32_ns: bool = False, stream=None):
+        shapes = [tuple(int(v) for v in s) for s in shapes]
+        if any(len(s) != 2 for s in shapes):
+            raise ValueError("Muon plans take 2-D shapes only")
+        self.shapes = shapes
+        self.n = len(shapes)
+        arr = (L.muon_param_t * self.n)()
+        flags = L.MUON_INIT_FP32_NS if fp32_ns else 0
+        if momenta is not None:
+            flags |= L.MUON_INIT_ZERO_MOMENTUM
+            for i, M in enumerate(momenta):
+                _check_tensor(M, torch.float32, f"M[{i}]", shapes[i])
+                arr[i].M = M.data_ptr()
+        for i, (r, c) in enumerate(shapes):
+            arr[i].rows, arr[i].cols = r, c
+        self._plan = L.muon_init(arr, self.n, flags, _stream_handle(stream))
+        self._params = (L.muon_param_t * self.n)()
+        self._key = None
+        self._x = (ctypes.c_void_p * self.n)()
+        self._o = (ctypes.c_void_p * self.n)()
+
+    # ------------------------------------------------------------ the step
+    def bind(self, params):
+        """Fill the descriptor array from [(W, G, M), ...]; reused by step()
+        while the same tensors are passed again."""
+        if len(params) != self.n:
+            raise ValueError(f"expected {self.n} (W, G, M) triples, got {len(params)}")
+        key = tuple((W.data_ptr(), G.data_ptr(), M.data_ptr(), G.dtype) for W, G, M in params)
+        if key == self._key:
+            return
+        for i, (W, G, M) in enumerate(params):
+            shp = self.shapes[i]
+            _check_tensor(W, torch.float32, f"W[{i}]", shp)
+            _check_tensor(G, (torch.bfloat16, torch.float32), f"G[{i}]", shp)
+            _check_tensor(M, torch.float32, f"M[{i}]", shp)
+            d = self._params[i]
+            d.W, d.G, d.M = W.data_ptr(), G.data_ptr(), M.data_ptr()
+            d.rows, d.cols = shp
+            d.g_dtype = _GDT[G.dtype]
+            d.reserved = 0
+        self._key = key
+
+    def step(self, params=None, *, lr: float, weight_decay: float, momentum: float = 0.95, ns_steps: int = 5,
+             coeffs=DEFAULT_COEFFS, rms_scale: float = 0.2, nesterov: bool = True, precision: str = "bf16",
+             update_rms: torch.Tensor | None = None, stream=None) -> None:
+        """One Muon step over every matrix (in place on W and M)."""
+        if params is not None:
+            self.bind(params)
+        elif self._key is None:
+            raise ValueError("no parameters bound")
+        hp = L.muon_hparams_t(lr, weight_decay, momentum, int(ns_steps), coeffs[0], coeffs[1], coeffs[2],
+                              rms_scale, 1 if nesterov else 0,
+                              L.MUON_NS_FP32 if precision == "fp32" else L.MUON_NS_BF16)
+        rms_ptr = None
+        if update_rms is not None:
+            _check_tensor(update_rms, torch.float32, "update_rms", (self.n,))
+            rms_ptr = update_rms.data_ptr()
+        L.muon_step(self._plan, self._params, self.n, hp, rms_ptr, _stream_handle(stream))
+
+    def orthogonalize(self, xs, outs, *, ns_steps: int = 5, coeffs=DEFAULT_COEFFS, precision: str = "bf16",
+                      stream=None) -> None:
+        """outs[i] = Newton-Schulz(xs[i]) (fp32 outputs) for every matrix."""
+        if len(xs) != self.n or len(outs) != self.n:
+            raise ValueError("one input and one output per planned matrix")
+        dt = None
+        for i, (x, o) in enumerate(zip(xs, outs)):
+            _check_tensor(x, (torch.bfloat16, torch.float32), f"X[{i}]", self.shapes[i])
+            _check_tensor(o, torch.float32, f"O[{i}]", self.shapes[i])
+            if dt is None:
+                dt = x.dtype
+            elif x.dtype != dt:
+                raise TypeError("all inputs of one call share a dtype")
+            self._x[i] = x.data_ptr()
+            self._o[i] = o.data_ptr()
+        L.muon_orthogonalize(self._plan, self._x, self._o, self.n, _GDT[dt], ns_steps, coeffs,
+                             L.MUON_NS_FP32 if precision == "fp32" else L.MUON_NS_BF16, _stream_handle(stream))
+
+    # ------------------------------------------------------------ bookkeeping
+    @property
+    def workspace_bytes(self) -> int:
+        return L.muon_workspace_bytes(self._plan)
+
+    def status(self) -> int:
+        """Synchronizing read-and-clear of the device status (an int status code)."""
+        return L.muon_get_status(self._plan)
+
+    def profile(self, enable: bool = True) -> None:
+        L.muon_profile_enable(self._plan, enable)
+
+    def profile_read(self):
+        ms, cnt, calls = L.muon_profile_read(self._plan)
+        return {"ms": dict(zip(L.PHASE_NAMES, ms)), "launches": dict(zip(L.PHASE_NAMES, cnt)), "calls": calls}
+
+    def close(self) -> None:
+        if getattr(self, "_plan", None):
+            L.muon_destroy(self._plan)
+            self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

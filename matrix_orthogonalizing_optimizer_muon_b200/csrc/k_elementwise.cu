@@ -1,0 +1,242 @@
+// Elementwise kernels of the Muon step.  All of them are HBM-bound: they are
+// written as chunked streams with 16-byte vector accesses where the caller's
+// pointers allow it, and every reduction is done in a fixed order so that a
+// step is bitwise reproducible.
+//
+// k1: momentum + Nesterov input + Frobenius norm + bf16 hi/lo split
+//     ("Muon is Scalable for LLM Training", Sec. 2.1, Eq. 1, the Nesterov
+//     paragraph, and X_0 = M / ||M||_F).  One CTA per chunk of rows.  The norm
+//     is accumulated in fp64 per chunk; the last CTA of each matrix (arrival
+//     counter) reduces the chunk partials in chunk order and writes
+//     s = 1 / ||Y||_F (0 for an all-zero Y, NaN plus a status bit if the sum
+//     is not finite).
+// apply_update: W <- W - lr (rms_scale sqrt(n) O + wd W) with O = s X, used
+//     when there are no Newton-Schulz iterations (N = 0); the N > 0 path fuses
+//     this update into the last GEMM epilogue (Sec. 2.2, Eq. 4).
+// rms_finalize: sqrt(mean(O^2)) per matrix from per-tile partial sums
+//     (Sec. 2.3, Algorithm 1, returned value).
+#include "muon_internal.cuh"
+
+namespace muon {
+namespace {
+
+__device__ __forceinline__ void load8(const void* base, size_t idx, int dtype, float* v) {
+  if (dtype == 0) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ float load1(const void* base, size_t idx, int dtype) {
+  if (dtype == 0) return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[idx]);
+  return static_cast<const float*>(base)[idx];
+}
+
+// Split y into hi = bf16(y), lo = bf16(y - hi).
+__device__ __forceinline__ void split_store8(__nv_bfloat16* hi, __nv_bfloat16* lo, const float* y) {
+  __align__(16) __nv_bfloat16 h[8];
+  __align__(16) __nv_bfloat16 l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = __float2bfloat16_rn(y[i]);
+    l[i] = __float2bfloat16_rn(y[i] - __bfloat162float(h[i]));
+  }
+  *reinterpret_cast<uint4*>(hi) = *reinterpret_cast<const uint4*>(h);
+  *reinterpret_cast<uint4*>(lo) = *reinterpret_cast<const uint4*>(l);
+}
+
+// Deterministic block sum (fixed shuffle tree, then warps in order).
+template <typename T>
+__device__ T block_sum(T v, T* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  T t = T(0);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+  }
+  return t;  // valid in thread 0
+}
+
+__global__ void __launch_bounds__(kEwThreads) k1_kernel(const ChunkDesc* __restrict__ chunks,
+                                                        const MatInfo* __restrict__ mats,
+                                                        const MatPtrs* __restrict__ ptrs, Workspace ws,
+                                                        StepScalars sc, int mode, int fp32_path) {
+  __shared__ double red[kEwThreads / 32];
+  __shared__ int am_last;
+  const ChunkDesc ch = chunks[blockIdx.x];
+  const int p = ch.x;
+  const MatInfo mi = mats[p];
+  const MatPtrs pt = ptrs[p];
+  const int C = mi.cols, r0 = ch.y, nr = ch.z;
+  const float mu = sc.mu;
+  double acc = 0.0;
+
+  if (pt.vec_ok) {
+    const int cv = C >> 3;
+    const int units = nr * cv;
+    for (int u = threadIdx.x; u < units; u += blockDim.x) {
+      const int rr = u / cv;
+      const int c8 = (u - rr * cv) << 3;
+      const int r = r0 + rr;
+      const size_t gi = (size_t)r * C + c8;
+      const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c8;
+      float y[8];
+      load8(pt.G, gi, pt.g_dtype, y);
+      if (mode == kK1Momentum) {
+        float4* mp = reinterpret_cast<float4*>(pt.M + gi);
+        float4 m0 = mp[0], m1 = mp[1];
+        float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float g = y[i];
+          m[i] = fmaf(mu, m[i], g);                      // M_t = mu M_{t-1} + G_t
+          y[i] = sc.nesterov ? fmaf(mu, m[i], g) : m[i];  // Y = mu M_t + G_t
+        }
+        mp[0] = make_float4(m[0], m[1], m[2], m[3]);
+        mp[1] = make_float4(m[4], m[5], m[6], m[7]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fma((double)y[i], (double)y[i], acc);
+      if (fp32_path) {
+        float4* xp = reinterpret_cast<float4*>(ws.x32[0] + wi);
+        xp[0] = make_float4(y[0], y[1], y[2], y[3]);
+        xp[1] = make_float4(y[4], y[5], y[6], y[7]);
+      } else {
+        split_store8(ws.hi[0] + wi, ws.lo + wi, y);
+      }
+    }
+  } else {
+    const int64_t total = (int64_t)nr * C;
+    for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+      const int rr = (int)(e / C);
+      const int c = (int)(e - (int64_t)rr * C);
+      const int r = r0 + rr;
+      const size_t gi = (size_t)r * C + c;
+      const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c;
+      const float g = load1(pt.G, gi, pt.g_dtype);
+      float y = g;
+      if (mode == kK1Momentum) {
+        const float m = fmaf(mu, pt.M[gi], g);
+        pt.M[gi] = m;
+        y = sc.nesterov ? fmaf(mu, m, g) : m;
+      }
+      acc = fma((double)y, (double)y, acc);
+      if (fp32_path) {
+        ws.x32[0][wi] = y;
+      } else {
+        const __nv_bfloat16 h = __float2bfloat16_rn(y);
+        ws.hi[0][wi] = h;
+        ws.lo[wi] = __float2bfloat16_rn(y - __bfloat162float(h));
+      }
+    }
+  }
+
+  const double part = block_sum(acc, red);
+  if (threadIdx.x == 0) {
+    ws.norm_part[ch.w] = part;
+    __threadfence();
+    const unsigned prev = atomicAdd(ws.norm_count + p, 1u);
+    am_last = (prev == (unsigned)(mi.nchunks - 1));
+  }
+  __syncthreads();
+  if (!am_last) return;
+  __threadfence();
+  double t = 0.0;
+  for (int i = threadIdx.x; i < mi.nchunks; i += blockDim.x) t += __ldcg(ws.norm_part + mi.chunk_base + i);
+  const double f2 = block_sum(t, red);
+  if (threadIdx.x == 0) {
+    float s;
+    if (!isfinite(f2)) {
+      s = __int_as_float(0x7fc00000);
+      atomicOr(ws.status, kStatusNonFinite);
+    } else {
+      s = f2 > 0.0 ? (float)(1.0 / sqrt(f2)) : 0.0f;
+    }
+    ws.s[p] = s;
+    ws.norm_count[p] = 0u;
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) apply_update_kernel(const ChunkDesc* __restrict__ chunks,
+                                                                  const MatInfo* __restrict__ mats,
+                                                                  const MatPtrs* __restrict__ ptrs, Workspace ws,
+                                                                  StepScalars sc, int final_mode, int fp32_path) {
+  __shared__ float red[kEwThreads / 32];
+  const ChunkDesc ch = chunks[blockIdx.x];
+  const int p = ch.x;
+  const MatInfo mi = mats[p];
+  const MatPtrs pt = ptrs[p];
+  const int C = mi.cols, r0 = ch.y, nr = ch.z;
+  const float s = ws.s[p];
+  const float scale = sc.rms_scale * sqrtf((float)mi.n);
+  float acc = 0.0f;
+  const int64_t total = (int64_t)nr * C;
+  for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+    const int rr = (int)(e / C);
+    const int c = (int)(e - (int64_t)rr * C);
+    const int r = r0 + rr;
+    const size_t gi = (size_t)r * C + c;
+    const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c;
+    const float x = fp32_path ? ws.x32[0][wi] : __bfloat162float(ws.hi[0][wi]) + __bfloat162float(ws.lo[wi]);
+    const float o = s * x;
+    acc = fmaf(o, o, acc);
+    if (final_mode == kFinalWeight) {
+      const float w = pt.W[gi];
+      pt.W[gi] = w - sc.lr * fmaf(scale, o, sc.wd * w);
+    } else {
+      pt.W[gi] = o;
+    }
+  }
+  const float part = block_sum(acc, red);
+  if (threadIdx.x == 0) ws.rms_part[ch.w] = part;
+}
+
+__global__ void __launch_bounds__(kEwThreads) rms_finalize_kernel(const MatInfo* __restrict__ mats,
+                                                                  const float* __restrict__ part, int which,
+                                                                  float* __restrict__ out) {
+  __shared__ double red[kEwThreads / 32];
+  const MatInfo mi = mats[blockIdx.x];
+  const int base = which == 1 ? mi.rms_tile_base : which == 2 ? mi.rms32_base : mi.chunk_base;
+  const int count = which == 1 ? mi.rms_tile_count : which == 2 ? mi.rms32_count : mi.nchunks;
+  double t = 0.0;
+  for (int i = threadIdx.x; i < count; i += blockDim.x) t += (double)part[base + i];
+  const double sum = block_sum(t, red);
+  if (threadIdx.x == 0) out[blockIdx.x] = (float)sqrt(sum / ((double)mi.rows * (double)mi.cols));
+}
+
+}  // namespace
+
+cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
+                      Workspace ws, StepScalars sc, int mode, int fp32_path, cudaStream_t st) {
+  k1_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, mode, fp32_path);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
+                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, cudaStream_t st) {
+  apply_update_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, final_mode, fp32_path);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which, float* out,
+                                cudaStream_t st) {
+  rms_finalize_kernel<<<nmat, kEwThreads, 0, st>>>(mats, part, which, out);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,625 @@
+// Host side of libmuon: the C ABI declared in include/muon.h.
+//
+// muon_init turns the list of parameter shapes into a plan: one device
+// allocation that holds the Newton-Schulz workspace, the per-matrix
+// descriptors, the tile schedules of every GEMM phase, the chunk schedule of
+// the elementwise kernels and one TMA descriptor per operand buffer.  A step
+// is then a fixed sequence of launches on the caller's stream:
+//   k1 (momentum, Nesterov input, Frobenius norm, bf16 split)
+//   N x [Gram, polynomial, X update]   (tensor cores; the last X update
+//                                       applies the weight update)
+//   optional update-RMS finalisation.
+// No host synchronisation happens in muon_step; per-call device pointers are
+// uploaded only when they differ from the previous call's.
+#include "muon.h"
+#include "muon_internal.cuh"
+
+#include <cuda.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+using namespace muon;
+
+namespace {
+
+constexpr int kMaxDim = 65536;
+constexpr int kMaxNsSteps = 32;
+constexpr int kEventPool = 4096;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, cols] array with row pitch `ld`
+// elements; 64 x 64 boxes with 128-byte swizzle, zero fill outside.
+bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBox), static_cast<cuuint32_t>(kBox)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct ProfRec {
+  int first_event;
+  int nlaunch;
+  int phases[3 * kMaxNsSteps + 4];
+};
+
+}  // namespace
+
+struct muon_plan_s {
+  int device = 0;
+  int sm_count = 0;
+  int n = 0;
+  uint32_t flags = 0;
+  bool fp32_ws = false;
+  std::vector<MatInfo> mats;
+  // device memory
+  uint8_t* dmem = nullptr;
+  size_t dbytes = 0;
+  Workspace ws{};
+  MatInfo* mats_d = nullptr;
+  MatPtrs* ptrs_d = nullptr;
+  TileDesc* sym_d = nullptr;
+  TileDesc* full_d = nullptr;
+  TileDesc* sym32_d = nullptr;
+  TileDesc* full32_d = nullptr;
+  int n_sym = 0, n_full = 0, n_sym32 = 0, n_full32 = 0;
+  ChunkDesc* chunks_d = nullptr;
+  int nchunks = 0;
+  void* tmaps_d = nullptr;
+  // per-call pointer table cache
+  std::vector<MatPtrs> ptr_cache;
+  bool ptr_cache_valid = false;
+  MatPtrs* ptr_pinned = nullptr;
+  cudaEvent_t ptr_event = nullptr;
+  bool ptr_event_pending = false;
+  cudaStream_t last_stream = nullptr;
+  // profiling
+  bool prof = false;
+  std::vector<cudaEvent_t> events;
+  int ev_next = 0;
+  std::vector<ProfRec> recs;
+  double prof_ms[MUON_NUM_PHASES] = {};
+  int64_t prof_launches[MUON_NUM_PHASES] = {};
+  int prof_calls = 0;
+};
+
+namespace {
+
+muon_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA; }
+
+bool finite(float v) { return std::isfinite(v); }
+
+struct Interval {
+  uintptr_t lo, hi;
+};
+
+bool any_overlap(std::vector<Interval>& v) {
+  std::sort(v.begin(), v.end(), [](const Interval& a, const Interval& b) { return a.lo < b.lo; });
+  for (size_t i = 1; i < v.size(); ++i)
+    if (v[i].lo < v[i - 1].hi) return true;
+  return false;
+}
+
+// Upload the per-call pointer table if it differs from the last one.
+muon_status_t upload_ptrs(muon_plan_s* pl, const std::vector<MatPtrs>& t, cudaStream_t st) {
+  if (pl->ptr_cache_valid && std::memcmp(t.data(), pl->ptr_cache.data(), t.size() * sizeof(MatPtrs)) == 0)
+    return MUON_OK;
+  if (pl->ptr_event_pending) {
+    if (cudaEventSynchronize(pl->ptr_event) != cudaSuccess) return MUON_ERR_CUDA;
+    pl->ptr_event_pending = false;
+  }
+  std::memcpy(pl->ptr_pinned, t.data(), t.size() * sizeof(MatPtrs));
+  if (cudaMemcpyAsync(pl->ptrs_d, pl->ptr_pinned, t.size() * sizeof(MatPtrs), cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (cudaEventRecord(pl->ptr_event, st) != cudaSuccess) return MUON_ERR_CUDA;
+  pl->ptr_event_pending = true;
+  pl->ptr_cache = t;
+  pl->ptr_cache_valid = true;
+  return MUON_OK;
+}
+
+// ------------------------------------------------------------ profiling
+void prof_flush(muon_plan_s* pl) {
+  for (const ProfRec& r : pl->recs) {
+    cudaEventSynchronize(pl->events[r.first_event + r.nlaunch]);
+    for (int k = 0; k < r.nlaunch; ++k) {
+      float ms = 0.0f;
+      cudaEventElapsedTime(&ms, pl->events[r.first_event + k], pl->events[r.first_event + k + 1]);
+      pl->prof_ms[r.phases[k]] += ms;
+      pl->prof_launches[r.phases[k]] += 1;
+    }
+    pl->prof_calls += 1;
+  }
+  pl->recs.clear();
+  pl->ev_next = 0;
+}
+
+struct Recorder {
+  muon_plan_s* pl;
+  cudaStream_t st;
+  ProfRec rec{};
+  bool on = false;
+  Recorder(muon_plan_s* p, cudaStream_t s, int max_launches) : pl(p), st(s) {
+    if (!pl->prof) return;
+    if (pl->ev_next + max_launches + 1 > static_cast<int>(pl->events.size())) prof_flush(pl);
+    rec.first_event = pl->ev_next;
+    rec.nlaunch = 0;
+    cudaEventRecord(pl->events[pl->ev_next++], st);
+    on = true;
+  }
+  void mark(int phase) {
+    if (!on) return;
+    rec.phases[rec.nlaunch++] = phase;
+    cudaEventRecord(pl->events[pl->ev_next++], st);
+  }
+  ~Recorder() {
+    if (on) pl->recs.push_back(rec);
+  }
+};
+
+// ------------------------------------------------------------ the launch sequence
+muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int precision, int final_mode,
+                     int k1_mode, float* update_rms, cudaStream_t st) {
+  Recorder rec(pl, st, 3 * ns_steps + 3);
+  const int fp32 = precision == MUON_NS_FP32 ? 1 : 0;
+  cudaError_t e = launch_k1(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, k1_mode, fp32, st);
+  if (e != cudaSuccess) return MUON_ERR_CUDA;
+  rec.mark(0);
+  int cur = 0;
+  for (int it = 0; it < ns_steps; ++it) {
+    const bool last = (it == ns_steps - 1);
+    for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
+      const int fm = (ph == kPhaseUpdate && last) ? final_mode : kFinalNone;
+      if (fp32) {
+        Gemm32Args a{};
+        a.tiles = (ph == kPhaseUpdate) ? pl->full32_d : pl->sym32_d;
+        a.ntiles = (ph == kPhaseUpdate) ? pl->n_full32 : pl->n_sym32;
+        a.phase = ph;
+        a.iter = it;
+        a.cur = cur;
+        a.final_mode = fm;
+        a.mats = pl->mats_d;
+        a.ptrs = pl->ptrs_d;
+        a.ws = pl->ws;
+        a.sc = sc;
+        e = launch_gemm_f32(a, st);
+      } else {
+        GemmArgs a{};
+        a.tiles = (ph == kPhaseUpdate) ? pl->full_d : pl->sym_d;
+        a.ntiles = (ph == kPhaseUpdate) ? pl->n_full : pl->n_sym;
+        a.phase = ph;
+        a.iter = it;
+        a.cur = cur;
+        a.final_mode = fm;
+        a.mats = pl->mats_d;
+        a.ptrs = pl->ptrs_d;
+        a.tmaps = pl->tmaps_d;
+        a.ws = pl->ws;
+        a.sc = sc;
+        e = launch_gemm_tc(a, std::min(pl->sm_count, a.ntiles), st);
+      }
+      if (e != cudaSuccess) return MUON_ERR_CUDA;
+      rec.mark(1 + ph);
+    }
+    if (!last) cur ^= 1;
+  }
+  int which = fp32 ? 2 : 1;
+  if (ns_steps == 0) {
+    e = launch_apply_update(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, final_mode, fp32, st);
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    rec.mark(4);
+    which = 0;
+  }
+  if (update_rms != nullptr) {
+    e = launch_rms_finalize(pl->mats_d, pl->n, pl->ws.rms_part, which, update_rms, st);
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    rec.mark(4);
+  }
+  pl->last_stream = st;
+  return MUON_OK;
+}
+
+void free_plan(muon_plan_s* pl) {
+  if (pl == nullptr) return;
+  if (pl->dmem) cudaFree(pl->dmem);
+  if (pl->ptr_pinned) cudaFreeHost(pl->ptr_pinned);
+  if (pl->ptr_event) cudaEventDestroy(pl->ptr_event);
+  for (cudaEvent_t ev : pl->events) cudaEventDestroy(ev);
+  delete pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* muon_status_string(muon_status_t s) {
+  switch (s) {
+    case MUON_OK: return "ok";
+    case MUON_ERR_INVALID_ARG: return "invalid argument";
+    case MUON_ERR_SHAPE_MISMATCH: return "descriptor count or shape differs from the plan";
+    case MUON_ERR_UNSUPPORTED: return "unsupported request for this plan or device";
+    case MUON_ERR_NO_MEMORY: return "out of memory";
+    case MUON_ERR_CUDA: return "CUDA error";
+    case MUON_ERR_NONFINITE: return "non-finite Frobenius norm";
+    case MUON_ERR_TIMEOUT: return "device-side wait timed out";
+    case MUON_ERR_ALIAS: return "buffers overlap";
+  }
+  return "unknown status";
+}
+
+muon_status_t muon_hparams_default(muon_hparams_t* hp) {
+  if (hp == nullptr) return MUON_ERR_INVALID_ARG;
+  hp->lr = 4.2e-4f;
+  hp->weight_decay = 0.1f;
+  hp->momentum = 0.95f;
+  hp->ns_steps = 5;
+  hp->a = 3.4445f;
+  hp->b = -4.7750f;
+  hp->c = 2.0315f;
+  hp->rms_scale = 0.2f;
+  hp->nesterov = 1;
+  hp->ns_precision = MUON_NS_BF16;
+  return MUON_OK;
+}
+
+muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags, void* stream) {
+  if (out == nullptr) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (params == nullptr || n < 1 || n > (1 << 20)) return MUON_ERR_INVALID_ARG;
+  if (flags & ~(MUON_INIT_ZERO_MOMENTUM | MUON_INIT_FP32_NS)) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const muon_param_t& p = params[i];
+    if (p.rows < 1 || p.cols < 1 || p.rows > kMaxDim || p.cols > kMaxDim || p.reserved != 0)
+      return MUON_ERR_INVALID_ARG;
+    if ((flags & MUON_INIT_ZERO_MOMENTUM) && p.M == nullptr) return MUON_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MUON_ERR_UNSUPPORTED;
+  if (get_encode_fn() == nullptr) return MUON_ERR_CUDA;
+
+  muon_plan_s* pl = new (std::nothrow) muon_plan_s();
+  if (pl == nullptr) return MUON_ERR_NO_MEMORY;
+  pl->device = dev;
+  pl->sm_count = prop.multiProcessorCount;
+  pl->n = n;
+  pl->flags = flags;
+  pl->fp32_ws = (flags & MUON_INIT_FP32_NS) != 0;
+  pl->mats.resize(n);
+
+  // ---- per-matrix layout and schedules
+  std::vector<TileDesc> sym, full, sym32, full32;
+  std::vector<ChunkDesc> chunks;
+  size_t total_x = 0, total_a = 0;
+  int rms_tc = 0, rms32 = 0;
+  // LPT order of matrices for the GEMM schedules (largest Newton-Schulz work first)
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  auto work = [&](int i) {
+    const double m = static_cast<double>(std::min(params[i].rows, params[i].cols));
+    const double nn = static_cast<double>(std::max(params[i].rows, params[i].cols));
+    return m * m * nn + m * m * m;
+  };
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return work(x) > work(y); });
+  for (int i = 0; i < n; ++i) {
+    MatInfo& mi = pl->mats[i];
+    const int R = static_cast<int>(params[i].rows), C = static_cast<int>(params[i].cols);
+    mi.rows = R;
+    mi.cols = C;
+    mi.m = std::min(R, C);
+    mi.n = std::max(R, C);
+    mi.tall = R > C ? 1 : 0;
+    mi.ld = static_cast<int>(round_up(C, 8));
+    mi.lda = static_cast<int>(round_up(mi.m, 8));
+    mi.off_x = static_cast<int64_t>(total_x);
+    total_x += round_up(static_cast<size_t>(R) * mi.ld, 128);
+    mi.off_a = static_cast<int64_t>(total_a);
+    total_a += round_up(static_cast<size_t>(mi.m) * mi.lda, 128);
+    const int rows_per_chunk = std::max(1, kChunkElems / C);
+    mi.chunk_base = static_cast<int>(chunks.size());
+    for (int r = 0; r < R; r += rows_per_chunk)
+      chunks.push_back(make_int4(i, r, std::min(rows_per_chunk, R - r), static_cast<int>(chunks.size())));
+    mi.nchunks = static_cast<int>(chunks.size()) - mi.chunk_base;
+    mi.rms_tile_base = rms_tc;
+    mi.rms_tile_count = ((R + kBM - 1) / kBM) * ((C + kBN - 1) / kBN) * kEpiWarps;
+    rms_tc += mi.rms_tile_count;
+    mi.rms32_base = rms32;
+    mi.rms32_count = ((R + kT32 - 1) / kT32) * ((C + kT32 - 1) / kT32);
+    rms32 += mi.rms32_count;
+  }
+  for (int i : order) {
+    const MatInfo& mi = pl->mats[i];
+    for (int r0 = 0; r0 < mi.m; r0 += kBM)
+      for (int c0 = 0; c0 < mi.m && c0 <= r0 + kBM - 1; c0 += kBN) {
+        const int need = std::min({kBN, mi.m - c0, r0 + kBM - c0});
+        sym.push_back(make_int4(i, r0, c0, need));
+      }
+    for (int r0 = 0; r0 < mi.rows; r0 += kBM)
+      for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
+    if (pl->fp32_ws) {
+      for (int r0 = 0; r0 < mi.m; r0 += kT32)
+        for (int c0 = 0; c0 < mi.m; c0 += kT32) sym32.push_back(make_int4(i, r0, c0, 0));
+      for (int r0 = 0; r0 < mi.rows; r0 += kT32)
+        for (int c0 = 0; c0 < mi.cols; c0 += kT32) full32.push_back(make_int4(i, r0, c0, 0));
+    }
+  }
+  pl->n_sym = static_cast<int>(sym.size());
+  pl->n_full = static_cast<int>(full.size());
+  pl->n_sym32 = static_cast<int>(sym32.size());
+  pl->n_full32 = static_cast<int>(full32.size());
+  pl->nchunks = static_cast<int>(chunks.size());
+
+  // ---- carve one device allocation
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_hi0 = take(total_x * 2), o_hi1 = take(total_x * 2), o_lo = take(total_x * 2);
+  const size_t o_A = take(total_a * 2), o_B = take(total_a * 2);
+  size_t o_x0 = 0, o_x1 = 0, o_a32 = 0, o_b32 = 0;
+  if (pl->fp32_ws) {
+    o_x0 = take(total_x * 4);
+    o_x1 = take(total_x * 4);
+    o_a32 = take(total_a * 4);
+    o_b32 = take(total_a * 4);
+  }
+  const size_t n_rms = std::max({static_cast<size_t>(pl->nchunks), static_cast<size_t>(rms_tc),
+                                 static_cast<size_t>(rms32)});
+  const size_t o_s = take(n * sizeof(float));
+  const size_t o_np = take(pl->nchunks * sizeof(double));
+  const size_t o_nc = take(n * sizeof(unsigned));
+  const size_t o_rms = take(n_rms * sizeof(float));
+  const size_t o_status = take(sizeof(unsigned));
+  const size_t o_mats = take(n * sizeof(MatInfo));
+  const size_t o_ptrs = take(n * sizeof(MatPtrs));
+  const size_t o_sym = take(std::max<size_t>(1, sym.size()) * sizeof(TileDesc));
+  const size_t o_full = take(std::max<size_t>(1, full.size()) * sizeof(TileDesc));
+  const size_t o_sym32 = take(std::max<size_t>(1, sym32.size()) * sizeof(TileDesc));
+  const size_t o_full32 = take(std::max<size_t>(1, full32.size()) * sizeof(TileDesc));
+  const size_t o_chunks = take(chunks.size() * sizeof(ChunkDesc));
+  const size_t o_tmaps = take(static_cast<size_t>(n) * 4 * sizeof(CUtensorMap));
+  pl->dbytes = off;
+  if (cudaMalloc(&pl->dmem, pl->dbytes) != cudaSuccess) {
+    cudaGetLastError();
+    free_plan(pl);
+    return MUON_ERR_NO_MEMORY;
+  }
+  uint8_t* b = pl->dmem;
+  Workspace& ws = pl->ws;
+  ws.hi[0] = reinterpret_cast<__nv_bfloat16*>(b + o_hi0);
+  ws.hi[1] = reinterpret_cast<__nv_bfloat16*>(b + o_hi1);
+  ws.lo = reinterpret_cast<__nv_bfloat16*>(b + o_lo);
+  ws.A = reinterpret_cast<__nv_bfloat16*>(b + o_A);
+  ws.B = reinterpret_cast<__nv_bfloat16*>(b + o_B);
+  if (pl->fp32_ws) {
+    ws.x32[0] = reinterpret_cast<float*>(b + o_x0);
+    ws.x32[1] = reinterpret_cast<float*>(b + o_x1);
+    ws.a32 = reinterpret_cast<float*>(b + o_a32);
+    ws.b32 = reinterpret_cast<float*>(b + o_b32);
+  }
+  ws.s = reinterpret_cast<float*>(b + o_s);
+  ws.norm_part = reinterpret_cast<double*>(b + o_np);
+  ws.norm_count = reinterpret_cast<unsigned*>(b + o_nc);
+  ws.rms_part = reinterpret_cast<float*>(b + o_rms);
+  ws.status = reinterpret_cast<unsigned*>(b + o_status);
+  pl->mats_d = reinterpret_cast<MatInfo*>(b + o_mats);
+  pl->ptrs_d = reinterpret_cast<MatPtrs*>(b + o_ptrs);
+  pl->sym_d = reinterpret_cast<TileDesc*>(b + o_sym);
+  pl->full_d = reinterpret_cast<TileDesc*>(b + o_full);
+  pl->sym32_d = reinterpret_cast<TileDesc*>(b + o_sym32);
+  pl->full32_d = reinterpret_cast<TileDesc*>(b + o_full32);
+  pl->chunks_d = reinterpret_cast<ChunkDesc*>(b + o_chunks);
+  pl->tmaps_d = b + o_tmaps;
+
+  // ---- TMA descriptors: hi0, hi1, A, B per matrix
+  std::vector<CUtensorMap> tmaps(static_cast<size_t>(n) * 4);
+  for (int i = 0; i < n; ++i) {
+    const MatInfo& mi = pl->mats[i];
+    bool ok = encode_bf16_2d(&tmaps[4 * i + 0], ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld) &&
+              encode_bf16_2d(&tmaps[4 * i + 1], ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld) &&
+              encode_bf16_2d(&tmaps[4 * i + 2], ws.A + mi.off_a, mi.m, mi.m, mi.lda) &&
+              encode_bf16_2d(&tmaps[4 * i + 3], ws.B + mi.off_a, mi.m, mi.m, mi.lda);
+    if (!ok) {
+      free_plan(pl);
+      return MUON_ERR_CUDA;
+    }
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bool ok = cudaMemcpy(pl->mats_d, pl->mats.data(), n * sizeof(MatInfo), cudaMemcpyHostToDevice) == cudaSuccess;
+  ok = ok && (sym.empty() || cudaMemcpy(pl->sym_d, sym.data(), sym.size() * sizeof(TileDesc),
+                                        cudaMemcpyHostToDevice) == cudaSuccess);
+  ok = ok && (full.empty() || cudaMemcpy(pl->full_d, full.data(), full.size() * sizeof(TileDesc),
+                                         cudaMemcpyHostToDevice) == cudaSuccess);
+  ok = ok && (sym32.empty() || cudaMemcpy(pl->sym32_d, sym32.data(), sym32.size() * sizeof(TileDesc),
+                                          cudaMemcpyHostToDevice) == cudaSuccess);
+  ok = ok && (full32.empty() || cudaMemcpy(pl->full32_d, full32.data(), full32.size() * sizeof(TileDesc),
+                                           cudaMemcpyHostToDevice) == cudaSuccess);
+  ok = ok && cudaMemcpy(pl->chunks_d, chunks.data(), chunks.size() * sizeof(ChunkDesc), cudaMemcpyHostToDevice) ==
+                 cudaSuccess;
+  ok = ok && cudaMemcpy(pl->tmaps_d, tmaps.data(), tmaps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) ==
+                 cudaSuccess;
+  ok = ok && cudaMemset(ws.norm_count, 0, n * sizeof(unsigned)) == cudaSuccess;
+  ok = ok && cudaMemset(ws.status, 0, sizeof(unsigned)) == cudaSuccess;
+  ok = ok && cudaMemset(ws.s, 0, n * sizeof(float)) == cudaSuccess;
+  ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&pl->ptr_pinned), n * sizeof(MatPtrs), cudaHostAllocDefault) ==
+                 cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&pl->ptr_event, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_plan(pl);
+    return MUON_ERR_CUDA;
+  }
+  if (flags & MUON_INIT_ZERO_MOMENTUM) {
+    for (int i = 0; i < n; ++i) {
+      if (cudaMemsetAsync(params[i].M, 0, static_cast<size_t>(params[i].rows) * params[i].cols * sizeof(float), st) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        free_plan(pl);
+        return MUON_ERR_CUDA;
+      }
+    }
+  }
+  pl->last_stream = st;
+  *out = pl;
+  return MUON_OK;
+}
+
+muon_status_t muon_step(muon_plan_t pl, const muon_param_t* params, int32_t n, const muon_hparams_t* hp,
+                        float* update_rms, void* stream) {
+  if (pl == nullptr || params == nullptr || hp == nullptr) return MUON_ERR_INVALID_ARG;
+  if (n != pl->n) return MUON_ERR_SHAPE_MISMATCH;
+  if (!finite(hp->lr) || !finite(hp->weight_decay) || !finite(hp->momentum) || !finite(hp->a) || !finite(hp->b) ||
+      !finite(hp->c) || !finite(hp->rms_scale))
+    return MUON_ERR_INVALID_ARG;
+  if (hp->ns_steps < 0 || hp->ns_steps > kMaxNsSteps) return MUON_ERR_INVALID_ARG;
+  if (hp->nesterov != 0 && hp->nesterov != 1) return MUON_ERR_INVALID_ARG;
+  if (hp->ns_precision != MUON_NS_BF16 && hp->ns_precision != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
+  if (hp->ns_precision == MUON_NS_FP32 && !pl->fp32_ws) return MUON_ERR_UNSUPPORTED;
+  std::vector<MatPtrs> t(n);
+  std::vector<Interval> iv;
+  iv.reserve(3 * static_cast<size_t>(n) + 1);
+  for (int i = 0; i < n; ++i) {
+    const muon_param_t& p = params[i];
+    const MatInfo& mi = pl->mats[i];
+    if (p.rows != mi.rows || p.cols != mi.cols) return MUON_ERR_SHAPE_MISMATCH;
+    if (p.W == nullptr || p.G == nullptr || p.M == nullptr || p.reserved != 0) return MUON_ERR_INVALID_ARG;
+    if (p.g_dtype != MUON_DT_BF16 && p.g_dtype != MUON_DT_FP32) return MUON_ERR_INVALID_ARG;
+    const size_t e = static_cast<size_t>(mi.rows) * mi.cols;
+    const uintptr_t w = reinterpret_cast<uintptr_t>(p.W), g = reinterpret_cast<uintptr_t>(p.G),
+                    m = reinterpret_cast<uintptr_t>(p.M);
+    iv.push_back({w, w + e * 4});
+    iv.push_back({g, g + e * (p.g_dtype == MUON_DT_BF16 ? 2 : 4)});
+    iv.push_back({m, m + e * 4});
+    t[i].W = p.W;
+    t[i].G = p.G;
+    t[i].M = p.M;
+    t[i].g_dtype = p.g_dtype;
+    t[i].vec_ok = ((w | g | m) % 16 == 0 && mi.cols % 8 == 0) ? 1 : 0;
+  }
+  if (update_rms != nullptr) {
+    const uintptr_t r = reinterpret_cast<uintptr_t>(update_rms);
+    iv.push_back({r, r + static_cast<size_t>(n) * 4});
+  }
+  if (any_overlap(iv)) return MUON_ERR_ALIAS;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int cur_dev = -1;
+  if (cudaGetDevice(&cur_dev) != cudaSuccess || cur_dev != pl->device) return MUON_ERR_INVALID_ARG;
+  muon_status_t s = upload_ptrs(pl, t, st);
+  if (s != MUON_OK) return s;
+  StepScalars sc{hp->lr, hp->weight_decay, hp->momentum, hp->a, hp->b, hp->c, hp->rms_scale, hp->nesterov};
+  return run_ns(pl, sc, hp->ns_steps, hp->ns_precision, kFinalWeight, kK1Momentum, update_rms, st);
+}
+
+muon_status_t muon_orthogonalize(muon_plan_t pl, const void* const* X_in, float* const* O_out, int32_t n,
+                                 int32_t in_dtype, int32_t ns_steps, const float abc[3], int32_t ns_precision,
+                                 void* stream) {
+  if (pl == nullptr || X_in == nullptr || O_out == nullptr || abc == nullptr) return MUON_ERR_INVALID_ARG;
+  if (n != pl->n) return MUON_ERR_SHAPE_MISMATCH;
+  if (in_dtype != MUON_DT_BF16 && in_dtype != MUON_DT_FP32) return MUON_ERR_INVALID_ARG;
+  if (ns_steps < 0 || ns_steps > kMaxNsSteps) return MUON_ERR_INVALID_ARG;
+  if (!finite(abc[0]) || !finite(abc[1]) || !finite(abc[2])) return MUON_ERR_INVALID_ARG;
+  if (ns_precision != MUON_NS_BF16 && ns_precision != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
+  if (ns_precision == MUON_NS_FP32 && !pl->fp32_ws) return MUON_ERR_UNSUPPORTED;
+  std::vector<MatPtrs> t(n);
+  std::vector<Interval> iv;
+  iv.reserve(2 * static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    const MatInfo& mi = pl->mats[i];
+    if (X_in[i] == nullptr || O_out[i] == nullptr) return MUON_ERR_INVALID_ARG;
+    const size_t e = static_cast<size_t>(mi.rows) * mi.cols;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(X_in[i]), o = reinterpret_cast<uintptr_t>(O_out[i]);
+    iv.push_back({x, x + e * (in_dtype == MUON_DT_BF16 ? 2 : 4)});
+    iv.push_back({o, o + e * 4});
+    t[i].W = O_out[i];
+    t[i].G = X_in[i];
+    t[i].M = nullptr;
+    t[i].g_dtype = in_dtype;
+    t[i].vec_ok = ((x | o) % 16 == 0 && mi.cols % 8 == 0) ? 1 : 0;
+  }
+  if (any_overlap(iv)) return MUON_ERR_ALIAS;
+  int cur_dev = -1;
+  if (cudaGetDevice(&cur_dev) != cudaSuccess || cur_dev != pl->device) return MUON_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  muon_status_t s = upload_ptrs(pl, t, st);
+  if (s != MUON_OK) return s;
+  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0};
+  return run_ns(pl, sc, ns_steps, ns_precision, kFinalOut, kK1Copy, nullptr, st);
+}
+
+size_t muon_workspace_bytes(muon_plan_t pl) { return pl == nullptr ? 0 : pl->dbytes; }
+
+muon_status_t muon_get_status(muon_plan_t pl) {
+  if (pl == nullptr) return MUON_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(pl->last_stream) != cudaSuccess) return MUON_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, pl->ws.status, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return MUON_ERR_CUDA;
+  if (v != 0 && cudaMemset(pl->ws.status, 0, sizeof(unsigned)) != cudaSuccess) return MUON_ERR_CUDA;
+  if (v & kStatusTimeout) return MUON_ERR_TIMEOUT;
+  if (v & kStatusNonFinite) return MUON_ERR_NONFINITE;
+  return MUON_OK;
+}
+
+void muon_destroy(muon_plan_t pl) {
+  if (pl == nullptr) return;
+  cudaStreamSynchronize(pl->last_stream);
+  cudaGetLastError();
+  free_plan(pl);
+}
+
+muon_status_t muon_profile_enable(muon_plan_t pl, int32_t enable) {
+  if (pl == nullptr) return MUON_ERR_INVALID_ARG;
+  if (enable && pl->events.empty()) {
+    pl->events.resize(kEventPool);
+    for (auto& ev : pl->events)
+      if (cudaEventCreate(&ev) != cudaSuccess) return MUON_ERR_CUDA;
+  }
+  pl->prof = enable != 0;
+  return MUON_OK;
+}
+
+muon_status_t muon_profile_read(muon_plan_t pl, double* phase_ms, int64_t* launches, int32_t* calls) {
+  if (pl == nullptr || phase_ms == nullptr || launches == nullptr || calls == nullptr) return MUON_ERR_INVALID_ARG;
+  prof_flush(pl);
+  for (int k = 0; k < MUON_NUM_PHASES; ++k) {
+    phase_ms[k] += pl->prof_ms[k];
+    launches[k] += pl->prof_launches[k];
+    pl->prof_ms[k] = 0.0;
+    pl->prof_launches[k] = 0;
+  }
+  *calls = pl->prof_calls;
+  pl->prof_calls = 0;
+  return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"

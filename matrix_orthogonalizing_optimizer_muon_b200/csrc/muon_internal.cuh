@@ -1,0 +1,147 @@
+// Internal definitions shared by libmuon's kernels and host code.
+//
+// Data layout in HBM (all owned by the plan unless noted):
+//   user W, M (fp32) and G (bf16/fp32): [R, C] row-major, the caller's buffers.
+//   hi[2], lo (bf16): the Newton-Schulz iterate in the parameter's own
+//       orientation [R, C] with row pitch `ld` (>= C, multiple of 8), stored as
+//       a bf16 pair X = hi + lo.  hi is the tensor-core operand and is double
+//       buffered (the X-update GEMM reads hi while its epilogue writes the
+//       next one); lo is only touched by the epilogue of the tile that owns
+//       the element and is updated in place.
+//   A, B (bf16): symmetric [m, m] matrices (m = min(R, C)), pitch `lda`.
+//   x32[2], a32, b32 (fp32): the same for the fp32 validation path.
+// A matrix with R > C ("tall") is never transposed: its Gram matrix is
+// Y^T Y, read with MN-major (column-contiguous) tensor-core operands, and its
+// X update is Y B, so every buffer keeps the parameter's layout.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace muon {
+
+// ---------------------------------------------------------------- tile shapes
+constexpr int kBM = 128;        // tile rows = UMMA M = TMEM lanes
+constexpr int kBN = 256;        // tile columns = max UMMA N = accumulator columns
+constexpr int kBK = 64;         // K per pipeline stage = one 128-byte swizzle row of bf16
+constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
+constexpr int kStages = 4;      // TMA -> MMA pipeline depth
+constexpr int kBox = 64;        // TMA box is 64 x 64 bf16 = 8 KiB for every operand
+constexpr int kBoxBytes = kBox * kBox * 2;
+constexpr int kStageABytes = kBM * kBK * 2;          // 16 KiB
+constexpr int kStageBBytes = kBN * kBK * 2;          // 32 KiB
+constexpr int kEpiWarps = 4;    // epilogue warps (one per TMEM lane quadrant)
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
+
+constexpr int kChunkElems = 32768;  // elements per momentum/normalise chunk
+constexpr int kEwThreads = 256;
+constexpr int kT32 = 64;           // fp32 path tile edge
+
+// device status bits (sticky, cleared by muon_get_status)
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusNonFinite = 2u;
+
+// bounded device waits: give up after this many nanoseconds of %globaltimer
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+enum Phase : int { kPhaseGram = 0, kPhasePoly = 1, kPhaseUpdate = 2 };
+enum FinalMode : int { kFinalNone = 0, kFinalWeight = 1, kFinalOut = 2 };
+enum K1Mode : int { kK1Momentum = 0, kK1Copy = 1 };
+
+// Per-matrix description, built once by muon_init.
+struct MatInfo {
+  int32_t rows, cols;   // parameter shape [R, C]
+  int32_t m, n;         // min(R, C), max(R, C)
+  int32_t tall;         // R > C
+  int32_t ld;           // pitch of [R, C] workspace arrays (elements)
+  int32_t lda;          // pitch of [m, m] workspace arrays (elements)
+  int32_t chunk_base;   // first chunk of this matrix in the chunk list
+  int32_t nchunks;
+  int32_t rms_tile_base;  // first rms partial slot of the fused final update (tensor-core tiles)
+  int32_t rms_tile_count;
+  int32_t rms32_base;     // same for the fp32 path's 64x64 tiles
+  int32_t rms32_count;
+  int32_t pad_[3];
+  int64_t off_x;        // element offset of this matrix in hi/lo/x32
+  int64_t off_a;        // element offset in A/B/a32/b32
+};
+
+// Per-call pointers of one matrix.
+struct MatPtrs {
+  float* W;             // muon_step: weights; muon_orthogonalize: O_out
+  const void* G;        // gradient or X_in
+  float* M;             // momentum (step only)
+  int32_t g_dtype;      // 0 bf16, 1 fp32
+  int32_t vec_ok;       // all three pointers 16-byte aligned and C % 8 == 0
+};
+
+// Tile of a GEMM phase: .x matrix, .y row0, .z col0, .w n_need (columns that
+// hold useful output, <= kBN).  Symmetric phases list only tiles that touch
+// the lower triangle.
+using TileDesc = int4;
+
+// Momentum/normalise chunk: .x matrix, .y first row, .z number of rows, .w slot
+using ChunkDesc = int4;
+
+struct Workspace {
+  __nv_bfloat16* hi[2];
+  __nv_bfloat16* lo;
+  __nv_bfloat16* A;
+  __nv_bfloat16* B;
+  float* x32[2];
+  float* a32;
+  float* b32;
+  float* s;             // per matrix: 1/||Y||_F, or 0 for a zero matrix
+  double* norm_part;    // per chunk: sum of y^2
+  unsigned* norm_count; // per matrix arrival counter (self-resetting)
+  float* rms_part;      // per tile-warp / chunk: sum of O^2
+  unsigned* status;
+};
+
+struct StepScalars {
+  float lr, wd, mu, a, b, c, rms_scale;
+  int nesterov;
+};
+
+// Arguments of the tensor-core GEMM kernel (one launch = one phase of one
+// Newton-Schulz iteration over every matrix of the plan).
+struct GemmArgs {
+  const TileDesc* tiles;
+  int ntiles;
+  int phase;            // Phase
+  int iter;             // 0-based iteration index (iteration 0 folds in 1/||Y||_F)
+  int cur;              // which hi buffer holds the current iterate
+  int final_mode;       // FinalMode (only for the last kPhaseUpdate)
+  const MatInfo* mats;
+  const MatPtrs* ptrs;
+  const void* tmaps;    // CUtensorMap[4 * nmat]: hi0, hi1, A, B
+  Workspace ws;
+  StepScalars sc;
+};
+
+// Arguments of the fp32 SIMT GEMM kernel.
+struct Gemm32Args {
+  const TileDesc* tiles;
+  int ntiles;
+  int phase, iter, cur, final_mode;
+  const MatInfo* mats;
+  const MatPtrs* ptrs;
+  Workspace ws;
+  StepScalars sc;
+};
+
+// ---------------------------------------------------------------- launchers (host)
+cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
+                      Workspace ws, StepScalars sc, int mode, int fp32_path, cudaStream_t st);
+cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
+                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, cudaStream_t st);
+// which: 0 chunk partials (stand-alone update), 1 tensor-core tiles, 2 fp32 tiles
+cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which,
+                                float* out, cudaStream_t st);
+cudaError_t launch_gemm_tc(const GemmArgs& args, int grid, cudaStream_t st);
+cudaError_t launch_gemm_f32(const Gemm32Args& args, cudaStream_t st);
+int gemm_tc_smem_bytes();
+
+}  // namespace muon

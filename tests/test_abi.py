@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point the header declares, and rejects bad arguments before it
+touches the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from matrix_orthogonalizing_optimizer_muon_b200 import _lib as L
+from matrix_orthogonalizing_optimizer_muon_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_symbols():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        names |= set(re.findall(r"MUON_API\s+[\w\s\*]+?\b(muon_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    assert declared_symbols() == set(L.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_no_other_exported_functions(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {s for s in exported if s.startswith("muon_")} == declared_symbols()
+
+
+def test_status_strings(lib):
+    for code in range(0, 9):
+        assert L.status_string(code)
+    assert L.status_string(0) == "ok"
+    assert L.status_string(123) == "unknown status"
+
+
+def test_default_hparams_are_the_pages_values(lib):
+    hp = L.muon_hparams_default()
+    assert abs(hp.a - 3.4445) < 1e-6 and abs(hp.b + 4.7750) < 1e-6 and abs(hp.c - 2.0315) < 1e-6
+    assert hp.ns_steps == 5 and abs(hp.momentum - 0.95) < 1e-7 and abs(hp.rms_scale - 0.2) < 1e-7
+    assert abs(hp.weight_decay - 0.1) < 1e-7 and abs(hp.lr - 4.2e-4) < 1e-10
+    assert hp.nesterov == 1 and hp.ns_precision == L.MUON_NS_BF16
+    assert lib.muon_hparams_default(None) == L.MUON_ERR_INVALID_ARG
+
+
+def test_init_rejects_bad_arguments_before_any_cuda_call(lib):
+    plan = ctypes.c_void_p()
+    arr = (L.muon_param_t * 2)()
+    arr[0].rows, arr[0].cols = 4, 4
+    arr[1].rows, arr[1].cols = 4, 4
+    assert lib.muon_init(None, arr, 2, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init(ctypes.byref(plan), None, 2, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init(ctypes.byref(plan), arr, 0, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init(ctypes.byref(plan), arr, 2, 0x100, None) == L.MUON_ERR_INVALID_ARG
+    arr[1].cols = 0
+    assert lib.muon_init(ctypes.byref(plan), arr, 2, 0, None) == L.MUON_ERR_INVALID_ARG
+    arr[1].cols = 70000
+    assert lib.muon_init(ctypes.byref(plan), arr, 2, 0, None) == L.MUON_ERR_INVALID_ARG
+    arr[1].cols = 4
+    arr[1].reserved = 1
+    assert lib.muon_init(ctypes.byref(plan), arr, 2, 0, None) == L.MUON_ERR_INVALID_ARG
+    arr[1].reserved = 0
+    # zero-momentum needs every M pointer
+    assert lib.muon_init(ctypes.byref(plan), arr, 2, L.MUON_INIT_ZERO_MOMENTUM, None) == L.MUON_ERR_INVALID_ARG
+    assert plan.value is None
+
+
+def test_null_plan_calls(lib):
+    hp = L.muon_hparams_default()
+    arr = (L.muon_param_t * 1)()
+    assert lib.muon_step(None, arr, 1, ctypes.byref(hp), None, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_workspace_bytes(None) == 0
+    assert lib.muon_get_status(None) == L.MUON_ERR_INVALID_ARG
+    lib.muon_destroy(None)
+    abc = (ctypes.c_float * 3)(1, 0, 0)
+    assert lib.muon_orthogonalize(None, None, None, 1, 0, 5, abc, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_profile_enable(None, 1) == L.MUON_ERR_INVALID_ARG
+
+
+def test_build_flags_target_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in B.ARCH
+    assert "-lineinfo" in B.FLAGS
