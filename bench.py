@@ -1,0 +1,377 @@
+"""Benchmark of the one-GPU Muon step on the 64+2-expert MoE batch.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload moe]
+
+One step = one grouped muon_step over all 198 expert matrices (momentum,
+Nesterov input, Frobenius normalisation, 5 quintic Newton-Schulz iterations,
+weight update and the per-matrix update RMS), on synthetic inputs resident
+in HBM.  Prints one JSON line (rank 0).
+
+Metric: Newton-Schulz TFLOP/s, counted with the algorithmic (symmetry-aware)
+FLOPs N (m(m+1)n + m^2(m+1) + 2 m^2 n) of every matrix with a non-zero
+gradient, divided by the whole step's device time; ms per step alongside.
+
+--gpus N under torchrun runs N independent replicas (the step has no
+exchange between GPUs): value = all ranks' FLOPs / max-over-ranks time.
+--impl reference times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload, in the same unit.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Newton-Schulz TFLOPS (% of B200 bf16 peak) and Muon step ms, 64-expert batch"
+UNIT = "TFLOP/s"
+K1_BYTES_PER_ELEM = 14          # G 2 + M 4 + 4 + hi 2 + lo 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def ns_flops(rows: int, cols: int, steps: int) -> int:
+    m, n = min(rows, cols), max(rows, cols)
+    return steps * (m * (m + 1) * n + m * m * (m + 1) + 2 * m * m * n)
+
+
+def ns_flops_dense(rows: int, cols: int, steps: int) -> int:
+    m, n = min(rows, cols), max(rows, cols)
+    return steps * (4 * m * m * n + 2 * m * m * m)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "matrix_orthogonalizing_optimizer_muon_b200", "csrc", "k_ns_tc.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def ncu_traffic(units: float):
+    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary,
+    scaled to this run's launch size; None unless the summary was taken on
+    the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ns_gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel_sha256_16") != kernel_source_hash():
+        return None
+    return d.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- oracle (CPU) legs
+
+def cpu_sample(wl, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle on whole-matrix steps of the workload until
+    `budget_s` seconds have passed.  Returns (flops, seconds, matrices)."""
+    import numpy as np
+    import oracle.muon_oracle as orc
+    from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
+    rng = np.random.default_rng(seed)
+    order = [i for i in rng.permutation(wl.n).tolist() if i not in wl.zero_grad]
+    flops, spent, done = 0, 0.0, 0
+    for i in order:
+        _, r, c = wl.shapes[i]
+        W = wlm.weight(wl, i).astype(np.float64)
+        G = wlm.bf16_bits_to_f32(wlm.grad_bf16(wl, i, 0)).astype(np.float64)
+        M = np.zeros_like(W)
+        t0 = time.perf_counter()
+        orc.muon_step(W, G, M, lr=4.2e-4, weight_decay=0.1)
+        spent += time.perf_counter() - t0
+        flops += ns_flops(r, c, 5)
+        done += 1
+        if spent >= budget_s:
+            break
+    return flops, spent, done
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((d.get("num_threads") or 0) for d in info) if info else (os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, wl, rank: int):
+    if rank != 0:
+        return
+    budget = float(os.environ.get("MUON_REFERENCE_STEP_S", "2.0"))
+    for _ in range(args.warmup):
+        cpu_sample(wl, 0.5, seed=1)
+    tot_f, tot_s, mats = 0, 0.0, 0
+    for k in range(args.steps):
+        f, s, d = cpu_sample(wl, budget, seed=100 + k)
+        tot_f, tot_s, mats = tot_f + f, tot_s + s, mats + d
+    value = tot_f / tot_s / 1e12
+    sample = (f"{mats} whole-matrix oracle steps (fp64 numpy) drawn from the {wl.n}-matrix workload, "
+              f"~{budget:.0f} s per timed step; FLOPs counted as for the GPU arm")
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    nz = [s for i, s in enumerate(wl.shapes) if i not in wl.zero_grad]
+    return {"workload": f"{wl.name}: {wl.n} matrices ({len(nz)} with non-zero gradient)",
+            "matrices": wl.n, "elements": wl.elements, "ns_steps": 5,
+            "shapes": sorted({(r, c) for _, r, c in wl.shapes}),
+            "inputs": "synthetic: W ~ N(0, 0.02^2) fp32, G ~ N(0, 1e-6) bf16, M_0 = 0",
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": "replicas (no exchange)"}
+
+
+# ---------------------------------------------------------------------- GPU arm
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="moe")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--limit", type=int, default=0, help="keep only the first N matrices (small profiling case)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
+    wl = wlm.get(args.workload)
+    if args.limit > 0:
+        wl.shapes = wl.shapes[:args.limit]
+        wl.zero_grad = {i for i in wl.zero_grad if i < args.limit}
+        wl.name += f"[first {args.limit}]"
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return 0
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from matrix_orthogonalizing_optimizer_muon_b200.api import MuonPlan
+
+    dev = torch.device("cuda", local)
+    shapes = [(r, c) for _, r, c in wl.shapes]
+    sizes = [r * c for r, c in shapes]
+    total = sum(sizes)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    Wbuf = torch.empty(total, device=dev).normal_(0.0, 0.02, generator=gen)
+    Gbuf = torch.empty(total, device=dev).normal_(0.0, 1e-3, generator=gen).to(torch.bfloat16)
+    Mbuf = torch.empty(total, device=dev)
+    Ws, Gs, Ms, off = [], [], [], 0
+    for (r, c), e in zip(shapes, sizes):
+        Ws.append(Wbuf[off:off + e].view(r, c))
+        Gs.append(Gbuf[off:off + e].view(r, c))
+        Ms.append(Mbuf[off:off + e].view(r, c))
+        off += e
+    for i in wl.zero_grad:
+        Gs[i].zero_()
+    plan = MuonPlan(shapes, momenta=Ms)
+    params = list(zip(Ws, Gs, Ms))
+    plan.bind(params)
+    rms = torch.zeros(wl.n, device=dev)
+    hp = dict(lr=4.2e-4, weight_decay=0.1, momentum=0.95, ns_steps=5)
+    nz_flops = sum(ns_flops(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
+    dense_flops = sum(ns_flops_dense(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        plan.step(**hp, update_rms=rms)
+    torch.cuda.synchronize()
+    st = plan.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    # ---- timed region: inputs resident in HBM
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plan.profile(True)
+    plan.profile_read()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            plan.step(**hp, update_rms=rms)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    plan.profile(False)
+    prof = plan.profile_read()
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    value = world * nz_flops / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end: pinned host gradients in, update RMS out, every step
+    e2e = None
+    if not args.no_e2e:
+        Ghost = Gbuf.cpu().pin_memory()
+        rms_host = torch.empty(wl.n, dtype=torch.float32).pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            Gbuf.copy_(Ghost, non_blocking=True)
+            plan.step(**hp, update_rms=rms)
+            rms_host.copy_(rms, non_blocking=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            Gbuf.copy_(Ghost, non_blocking=True)
+            plan.step(**hp, update_rms=rms)
+            rms_host.copy_(rms, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": world * nz_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": Gbuf.numel() * 2, "d2h_bytes_per_step": wl.n * 4,
+               "path": "MuonPlan.step (C ABI muon_step) with G copied from pinned host memory and the "
+                       "update RMS copied back each step"}
+    st = plan.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    if rank != 0:
+        plan.close()
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    calls = max(prof["calls"], 1)
+    gemm_ms = sum(prof["ms"][k] for k in ("gram", "poly", "x_update")) / calls
+    gemm_launches = sum(prof["launches"][k] for k in ("gram", "poly", "x_update")) / calls
+    per_step_launches = sum(prof["launches"].values()) / calls
+    achieved = nz_flops / (gemm_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    k1_ms = prof["ms"]["momentum_normalise"] / calls
+    k1_gbs = total * K1_BYTES_PER_ELEM / (k1_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(gemm_launches)
+
+    cpu = None
+    if world == 1 and args.cpu_budget > 0:
+        f, s, d = cpu_sample(wl, args.cpu_budget)
+        cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{d} whole-matrix fp64 oracle steps of the workload ({s:.1f} s), same FLOP count"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(wl),
+        "ns_ms_per_step": gemm_ms, "ns_tflops": achieved,
+        "ns_pct_of_bf16_peak": 100.0 * achieved / peak,
+        "ns_tflops_dense_equivalent": dense_flops / (gemm_ms * 1e-3) / 1e12,
+        "phase_ms_per_step": {k: v / calls for k, v in prof["ms"].items()},
+        "roofline": {"kernel": "ns_gemm_kernel (tcgen05, all Gram/poly/X-update launches)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"bf16_tflops_sustained ({peak_kind})", "traffic": traffic,
+                     "algorithmic_flops_per_launch": nz_flops / gemm_launches},
+        "elementwise": {"kernel": "k1_kernel (momentum, Nesterov, norm, bf16 split)", "bound": "hbm",
+                        "achieved": k1_gbs, "peak": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                        "unit": "GB/s", "frac": k1_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                        "bytes_per_elem": K1_BYTES_PER_ELEM},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(round(per_step_launches * args.steps)),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    plan.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
