@@ -130,7 +130,8 @@ def test_zero_gradient_matrix_is_pure_decay():
     torch.cuda.synchronize()
     for k in (0, 2):
         want = W0[k] - LR * (WD * W0[k])
-        assert np.max(np.abs(host64(Ws[k]) - want)) <= 1e-9
+        # two fp32 roundings of the decay product and one of the result
+        assert np.max(np.abs(host64(Ws[k]) - want) / np.maximum(np.abs(want), 1e-30)) <= 3 * 2.0 ** -24
         assert float(rms[k]) == 0.0
     assert float(rms[1]) > 0
 
