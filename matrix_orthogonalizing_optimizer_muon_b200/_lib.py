@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so")
+LIB_PATH = os.environ.get("MUON_LIB_PATH") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon.so")
 
 MUON_OK = 0
 MUON_ERR_INVALID_ARG = 1

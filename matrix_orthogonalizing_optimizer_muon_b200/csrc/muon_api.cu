@@ -18,6 +18,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -49,17 +50,19 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // 2-D bf16 tensor map over a [rows, cols] array with row pitch `ld`
-// elements; 64 x 64 boxes with 128-byte swizzle, zero fill outside.
-bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld) {
+// elements and boxes of `box_cols` (contiguous) x 128 rows; zero fill
+// outside.  64-column boxes use the 128-byte swizzle (tensor-core operands),
+// 32-column boxes the 64-byte swizzle (epilogue staging).
+bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld, int box_cols) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBox), static_cast<cuuint32_t>(kBox)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBoxOuter)};
   const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct ProfRec {
@@ -73,6 +76,7 @@ struct ProfRec {
 struct muon_plan_s {
   int device = 0;
   int sm_count = 0;
+  int npairs = 0;  // resident 2-CTA clusters of the tensor-core kernel
   int n = 0;
   uint32_t flags = 0;
   bool fp32_ws = false;
@@ -222,7 +226,7 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
         a.tmaps = pl->tmaps_d;
         a.ws = pl->ws;
         a.sc = sc;
-        e = launch_gemm_tc(a, std::min(pl->sm_count, a.ntiles), st);
+        e = launch_gemm_tc(a, pl->npairs, st);
       }
       if (e != cudaSuccess) return MUON_ERR_CUDA;
       rec.mark(1 + ph);
@@ -310,6 +314,14 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   if (pl == nullptr) return MUON_ERR_NO_MEMORY;
   pl->device = dev;
   pl->sm_count = prop.multiProcessorCount;
+  // persistent grid of the tensor-core kernel: as many 2-CTA clusters as can be
+  // resident (clusters never wait on each other, so more would only queue)
+  pl->npairs = gemm_tc_max_pairs();
+  if (pl->npairs < 1) pl->npairs = std::max(1, pl->sm_count / 2);
+  if (const char* env = std::getenv("MUON_TC_PAIRS")) {  // diagnostic: cap the persistent grid
+    const int v = std::atoi(env);
+    if (v >= 1 && v < pl->npairs) pl->npairs = v;
+  }
   pl->n = n;
   pl->flags = flags;
   pl->fp32_ws = (flags & MUON_INIT_FP32_NS) != 0;
@@ -349,7 +361,7 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
       chunks.push_back(make_int4(i, r, std::min(rows_per_chunk, R - r), static_cast<int>(chunks.size())));
     mi.nchunks = static_cast<int>(chunks.size()) - mi.chunk_base;
     mi.rms_tile_base = rms_tc;
-    mi.rms_tile_count = ((R + kBM - 1) / kBM) * ((C + kBN - 1) / kBN) * kEpiWarps;
+    mi.rms_tile_count = ((R + kTileM - 1) / kTileM) * ((C + kBN - 1) / kBN) * kRmsSlotsPerTile;
     rms_tc += mi.rms_tile_count;
     mi.rms32_base = rms32;
     mi.rms32_count = ((R + kT32 - 1) / kT32) * ((C + kT32 - 1) / kT32);
@@ -357,12 +369,12 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   }
   for (int i : order) {
     const MatInfo& mi = pl->mats[i];
-    for (int r0 = 0; r0 < mi.m; r0 += kBM)
-      for (int c0 = 0; c0 < mi.m && c0 <= r0 + kBM - 1; c0 += kBN) {
-        const int need = std::min({kBN, mi.m - c0, r0 + kBM - c0});
+    for (int r0 = 0; r0 < mi.m; r0 += kTileM)
+      for (int c0 = 0; c0 < mi.m && c0 <= r0 + kTileM - 1; c0 += kBN) {
+        const int need = std::min({kBN, mi.m - c0, r0 + kTileM - c0});
         sym.push_back(make_int4(i, r0, c0, need));
       }
-    for (int r0 = 0; r0 < mi.rows; r0 += kBM)
+    for (int r0 = 0; r0 < mi.rows; r0 += kTileM)
       for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
     if (pl->fp32_ws) {
       for (int r0 = 0; r0 < mi.m; r0 += kT32)
@@ -407,7 +419,7 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   const size_t o_sym32 = take(std::max<size_t>(1, sym32.size()) * sizeof(TileDesc));
   const size_t o_full32 = take(std::max<size_t>(1, full32.size()) * sizeof(TileDesc));
   const size_t o_chunks = take(chunks.size() * sizeof(ChunkDesc));
-  const size_t o_tmaps = take(static_cast<size_t>(n) * 4 * sizeof(CUtensorMap));
+  const size_t o_tmaps = take(static_cast<size_t>(n) * kMapsPerMat * sizeof(CUtensorMap));
   pl->dbytes = off;
   if (cudaMalloc(&pl->dmem, pl->dbytes) != cudaSuccess) {
     cudaGetLastError();
@@ -441,14 +453,19 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   pl->chunks_d = reinterpret_cast<ChunkDesc*>(b + o_chunks);
   pl->tmaps_d = b + o_tmaps;
 
-  // ---- TMA descriptors: hi0, hi1, A, B per matrix
-  std::vector<CUtensorMap> tmaps(static_cast<size_t>(n) * 4);
+  // ---- TMA descriptors: hi0, hi1, A, B, lo per matrix
+  std::vector<CUtensorMap> tmaps(static_cast<size_t>(n) * kMapsPerMat);
   for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];
-    bool ok = encode_bf16_2d(&tmaps[4 * i + 0], ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld) &&
-              encode_bf16_2d(&tmaps[4 * i + 1], ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld) &&
-              encode_bf16_2d(&tmaps[4 * i + 2], ws.A + mi.off_a, mi.m, mi.m, mi.lda) &&
-              encode_bf16_2d(&tmaps[4 * i + 3], ws.B + mi.off_a, mi.m, mi.m, mi.lda);
+    CUtensorMap* t = &tmaps[static_cast<size_t>(kMapsPerMat) * i];
+    bool ok = encode_bf16_2d(t + kMapHi0, ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld, kBoxInner) &&
+              encode_bf16_2d(t + kMapHi1, ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld, kBoxInner) &&
+              encode_bf16_2d(t + kMapA, ws.A + mi.off_a, mi.m, mi.m, mi.lda, kBoxInner) &&
+              encode_bf16_2d(t + kMapB, ws.B + mi.off_a, mi.m, mi.m, mi.lda, kBoxInner) &&
+              encode_bf16_2d(t + kMapEpiHi0, ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols) &&
+              encode_bf16_2d(t + kMapEpiHi1, ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols) &&
+              encode_bf16_2d(t + kMapEpiA, ws.A + mi.off_a, mi.m, mi.m, mi.lda, kEpiBoxCols) &&
+              encode_bf16_2d(t + kMapEpiLo, ws.lo + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols);
     if (!ok) {
       free_plan(pl);
       return MUON_ERR_CUDA;

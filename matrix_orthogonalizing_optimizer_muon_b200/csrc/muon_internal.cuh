@@ -22,22 +22,31 @@
 namespace muon {
 
 // ---------------------------------------------------------------- tile shapes
-constexpr int kBM = 128;        // tile rows = UMMA M = TMEM lanes
-constexpr int kBN = 256;        // tile columns = max UMMA N = accumulator columns
-constexpr int kBK = 64;         // K per pipeline stage = one 128-byte swizzle row of bf16
+// A tensor-core tile is 256 x 256 outputs computed by a pair of CTAs (a
+// 2-CTA cluster on two SMs): each CTA stages 128 rows of the A operand and
+// half of the B operand's N rows, and holds its 128 output rows in TMEM.
+constexpr int kTileM = 256;     // output rows per tile (two CTAs x 128 TMEM lanes)
+constexpr int kHalfM = 128;     // output rows per CTA
+constexpr int kBN = 256;        // output columns per tile = max UMMA N
+constexpr int kBK = 128;        // K per pipeline stage (two 128-byte swizzle atoms of bf16)
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-constexpr int kStages = 4;      // TMA -> MMA pipeline depth
-constexpr int kBox = 64;        // TMA box is 64 x 64 bf16 = 8 KiB for every operand
-constexpr int kBoxBytes = kBox * kBox * 2;
-constexpr int kStageABytes = kBM * kBK * 2;          // 16 KiB
-constexpr int kStageBBytes = kBN * kBK * 2;          // 32 KiB
-constexpr int kEpiWarps = 4;    // epilogue warps (one per TMEM lane quadrant)
-constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
-constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
+constexpr int kBoxInner = 64;   // every TMA box is 64 (contiguous) x 128 bf16 = 16 KiB
+constexpr int kBoxOuter = 128;
+constexpr int kBoxBytes = kBoxInner * kBoxOuter * 2;
+constexpr int kEpiWarps = 8;    // epilogue warps per CTA (two per TMEM lane quadrant)
+constexpr int kRmsSlotsPerTile = 2 * kEpiWarps;
+constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators per CTA
 
 constexpr int kChunkElems = 32768;  // elements per momentum/normalise chunk
 constexpr int kEwThreads = 256;
 constexpr int kT32 = 64;           // fp32 path tile edge
+// TMA descriptors per matrix: main-loop operand maps hi0, hi1, A, B (64 x 128
+// boxes, 128-byte swizzle) and epilogue maps hi0, hi1, A, lo (32 x 128 boxes,
+// 64-byte swizzle)
+constexpr int kMapsPerMat = 8;
+enum MapIndex : int { kMapHi0 = 0, kMapHi1 = 1, kMapA = 2, kMapB = 3, kMapEpiHi0 = 4, kMapEpiHi1 = 5, kMapEpiA = 6,
+                      kMapEpiLo = 7 };
+constexpr int kEpiBoxCols = 32;
 
 // device status bits (sticky, cleared by muon_get_status)
 constexpr uint32_t kStatusTimeout = 1u;
@@ -116,7 +125,7 @@ struct GemmArgs {
   int final_mode;       // FinalMode (only for the last kPhaseUpdate)
   const MatInfo* mats;
   const MatPtrs* ptrs;
-  const void* tmaps;    // CUtensorMap[4 * nmat]: hi0, hi1, A, B
+  const void* tmaps;    // CUtensorMap[kMapsPerMat * nmat], see MapIndex
   Workspace ws;
   StepScalars sc;
 };
@@ -140,7 +149,8 @@ cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatI
 // which: 0 chunk partials (stand-alone update), 1 tensor-core tiles, 2 fp32 tiles
 cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which,
                                 float* out, cudaStream_t st);
-cudaError_t launch_gemm_tc(const GemmArgs& args, int grid, cudaStream_t st);
+cudaError_t launch_gemm_tc(const GemmArgs& args, int npairs, cudaStream_t st);
+int gemm_tc_max_pairs();
 cudaError_t launch_gemm_f32(const Gemm32Args& args, cudaStream_t st);
 int gemm_tc_smem_bytes();
 
