@@ -15,9 +15,10 @@
 // bf16 operands, fp32 accumulators in TMEM) reads 128 A rows and N/2 B rows
 // from each CTA's shared memory, so each SM streams 32 KiB per 64-deep K step
 // for 4.2 MFLOP.  Per CTA:
-//   warp 0      TMA producer: 64 x 64 bf16 boxes (128-byte swizzle) into a
-//               kStages-deep ring; both CTAs' loads complete on the leader
-//               CTA's "full" mbarrier.
+//   warp 0      TMA producer: four lanes each issue one 64 x 128 bf16 box
+//               (128-byte swizzle) per 128-deep K stage into a ring of 3
+//               stages (2 for the X update, which gives its epilogue the
+//               room); both CTAs' loads complete on the leader's "full" barrier.
 //   warp 1      TMEM allocator (both CTAs) and MMA issuer (leader only); two
 //               256-column accumulators so the epilogue of one tile overlaps
 //               the main loop of the next.
@@ -43,7 +44,8 @@ namespace {
 #ifndef MUON_TC_STAGES
 #define MUON_TC_STAGES 3
 #endif
-constexpr int kStages = MUON_TC_STAGES;
+constexpr int kStages = MUON_TC_STAGES;   // stages of the Gram and polynomial phases
+constexpr int kStagesUpd = 2;              // stages of the X-update phase
 constexpr int kStageABytes = kHalfM * kBK * 2;   // 32 KiB: this CTA's 128 A rows x 128 K
 constexpr int kStageBBytes = 128 * kBK * 2;      // 32 KiB: up to 128 B rows (half of N) x 128 K
 // Epilogue: two groups of four warps (one warp per TMEM lane quadrant each);
@@ -60,10 +62,18 @@ constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;      // 32 KiB
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
 constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);
 
+// X-update epilogue: per warp a ring of 3 buffers, each a 32 x 32 hi block and
+// lo block (4 KiB), filled by cp.async.  With 2 main-loop stages the free
+// shared memory is [64 KiB, 96 KiB) and [160 KiB, 224 KiB): 24 buffers.
+constexpr int kUpdBufs = 3;
+constexpr int kUpdBufBytes = 2 * kEpiBlockBytes;
+
 struct SmemLayout {
   static constexpr int kA = 0;
   static constexpr int kB = kA + kStages * kStageABytes;
   static constexpr int kEpi = kB + kStages * kStageBBytes;
+  static constexpr int kUpdLo = kA + kStagesUpd * kStageABytes;  // [64 KiB, 96 KiB)
+  static constexpr int kUpdHi = kB + kStagesUpd * kStageBBytes;  // [160 KiB, 224 KiB)
   static constexpr int kBar = kEpi + kEpiBytes;
   // full[S], empty[S], tfull[2], tempty[2], drain
   static constexpr int kNumBars = 2 * kStages + 5;
@@ -346,6 +356,30 @@ __device__ __forceinline__ void store_block32(const uint8_t* blk, __nv_bfloat16*
   }
 }
 
+// Asynchronous (cp.async, no registers) copy of a 32 x 32 bf16 block
+// src[(g_row0 + rr) * ld + g_col0 + cc] into a staging block, 16 bytes per
+// lane per row segment; completion is tracked by cp.async groups.
+__device__ __forceinline__ void cp_block32(uint8_t* blk, const __nv_bfloat16* src, int ld, int g_row0, int g_col0,
+                                           int lane) {
+  const int c16 = lane & 3;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int rr = 8 * k + (lane >> 2);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(blk + chunk_off(rr, c16))),
+                 "l"(src + static_cast<size_t>(g_row0 + rr) * ld + g_col0 + c16 * 8)
+                 : "memory");
+  }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// wait until at most `pending` of this thread's most recent groups are in flight
+__device__ __forceinline__ void cp_async_wait(int pending) {
+  if (pending <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+  else if (pending == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else asm volatile("cp.async.wait_group 2;" ::: "memory");
+}
+
 // Row i, columns [j0, j0+32) of a [rows, cols] bf16 array, zero outside.
 __device__ __forceinline__ void load_row32_masked(const __nv_bfloat16* src, int ld, int rows, int cols, int i, int j0,
                                                   uint4 (&out)[4]) {
@@ -446,6 +480,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // B box 0, B box 1): TMA throughput per SM grows with the number of
     // threads issuing, so one thread per box keeps the copies in flight
     // concurrently.  Lane 0 owns the barriers.
+    const int nst = (g.phase == kPhaseUpdate) ? kStagesUpd : kStages;
     int stage = 0;
     uint32_t phase = 0;
     long fills = 0;
@@ -483,7 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           else        tma_load_pair(sb + h * kBoxBytes, c.b.tmap, k0 + h * kBoxInner, brow, fb);
         }
         ++fills;
-        if (++stage == kStages) {
+        if (++stage == nst) {
           stage = 0;
           phase ^= 1u;
         }
@@ -493,8 +528,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Drain (leader): both CTAs' loads complete on the leader's barriers,
     // so every stage's most recent fill must have landed before exit.
     if (leader && lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
-        const long cnt = fills / kStages + ((s < fills % kStages) ? 1 : 0);
+      for (int s = 0; s < nst; ++s) {
+        const long cnt = fills / nst + ((s < fills % nst) ? 1 : 0);
         if (cnt > 0 && !wait_bounded(full_bar(s), static_cast<uint32_t>((cnt - 1) & 1), nullptr))
           atomicOr(status, kStatusTimeout);
       }
@@ -502,6 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     if (leader && lane == 0) {
+      const int nst = (g.phase == kPhaseUpdate) ? kStagesUpd : kStages;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -545,7 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // free the stage in both CTAs once these MMAs have read it
           tc_commit(empty_bar(stage));
           tc_commit(map_to_rank(empty_bar(stage), 1));
-          if (++stage == kStages) {
+          if (++stage == nst) {
             stage = 0;
             phase ^= 1u;
           }
@@ -620,8 +656,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           load_block32(in0, ld_in, i_lo, j0, lane, pf0);
           if (nin == 2) load_block32(in1, ld_in, i_lo, j0, lane, pf1);
         };
+        // X update: a per-warp ring of kUpdBufs buffers (hi, lo) fed by cp.async,
+        // up to three chunks ahead; the polynomial prefetches into registers
+        auto upd_buf = [&](int b) -> uint8_t* {
+          const int id = ew * kUpdBufs + b;
+          return smem + (id < 8 ? SmemLayout::kUpdLo + id * kUpdBufBytes : SmemLayout::kUpdHi + (id - 8) * kUpdBufBytes);
+        };
+        int kc = 0;  // chunks of this warp in this tile
+        for (int x = grp; x < c.nch; x += kEpiGroups) ++kc;
+        int issued = 0;
+        auto stage_chunk = [&](int k) {
+          const int chh = grp + k * kEpiGroups;
+          if (block_inside(chh)) {
+            uint8_t* b = upd_buf(k % kUpdBufs);
+            cp_block32(b, in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
+            cp_block32(b + kEpiBlockBytes, in1, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
+          }
+          cp_async_commit();  // one group per chunk, empty for ragged chunks
+        };
         int ch = grp;
-        prefetch(ch);
+        if (upd) {
+          for (; issued < kc && issued < kUpdBufs; ++issued) stage_chunk(issued);
+        } else {
+          prefetch(ch);
+        }
         // one lane waits and the warp follows its verdict, so the warp stays
         // converged for the .sync.aligned TMEM loads
         int ready = 0;
@@ -634,7 +692,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
         const float s = g.ws.s[c.p];
-        for (; ch < c.nch; ch += kEpiGroups) {
+        for (int k = 0; ch < c.nch; ch += kEpiGroups, ++k) {
           const int j0 = c.col0 + ch * kEpiBoxCols;
           if (!needed(ch)) continue;
           const bool inside = block_inside(ch);
@@ -644,7 +702,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // land this chunk's prefetched inputs in the warp's staging blocks,
           // then start fetching the next chunk
           uint4 xa[4], xb[4];  // this thread's row, packed bf16
-          if (nin > 0) {
+          uint8_t* ub = upd ? upd_buf(k % kUpdBufs) : nullptr;
+          if (upd) {
+            if (inside) {
+              cp_async_wait(issued - k - 1);
+              __syncwarp();
+              read_row32(ub, lane, xa);
+              read_row32(ub + kEpiBlockBytes, lane, xb);
+            } else {
+              load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
+              load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
+            }
+          } else if (nin > 0) {
             if (inside) {
               put_block32(blk0, lane, pf0);
               if (nin == 2) put_block32(blk1, lane, pf1);
@@ -657,7 +726,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (nin == 2) load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
             }
           }
-          if (ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
+          if (!upd && ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
           tmem_ld_wait();
           float val[32];
           if (g.phase == kPhaseGram) {
@@ -709,11 +778,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
             __nv_bfloat16* lout = g.ws.lo + mi.off_x;
             if (inside) {
-              write_row32(blk0, lane, h);
-              write_row32(blk1, lane, l);
+              write_row32(ub, lane, h);
+              write_row32(ub + kEpiBlockBytes, lane, l);
               __syncwarp();
-              store_block32(blk0, hout, mi.ld, i_lo, j0, lane);
-              store_block32(blk1, lout, mi.ld, i_lo, j0, lane);
+              store_block32(ub, hout, mi.ld, i_lo, j0, lane);
+              store_block32(ub + kEpiBlockBytes, lout, mi.ld, i_lo, j0, lane);
             } else if (i < mi.rows) {
               const size_t wi = static_cast<size_t>(i) * mi.ld + j0;
 #pragma unroll
@@ -760,6 +829,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               }
             }
           }
+          if (upd && issued < kc) {
+            __syncwarp();  // every lane is done with this buffer before it is refilled
+            stage_chunk(issued);
+            ++issued;
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -777,6 +851,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may land in freed shared memory
   }
 
   tc_fence_before();
