@@ -125,6 +125,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------------- replicas
+
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The largest per-rank value (the slowest replica's time); `v` itself
+    without a process group."""
+    if dist is None or not dist.is_initialized():
+        return v
+    import torch
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tflops(world: int, flops_per_rank: int, ms_step: float) -> float:
+    """Whole-job throughput of `world` independent replicas that each do
+    `flops_per_rank` per step, timed by the slowest one."""
+    return world * flops_per_rank / (ms_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------- oracle (CPU) legs
 
 def cpu_sample(wl, budget_s: float, seed: int = 0):
@@ -260,13 +279,6 @@ def main(argv=None) -> int:
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         plan.step(**hp, update_rms=rms)
     torch.cuda.synchronize()
@@ -290,8 +302,8 @@ def main(argv=None) -> int:
     barrier()
     plan.profile(False)
     prof = plan.profile_read()
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    value = world * nz_flops / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    value = replica_tflops(world, nz_flops, ms_step)
 
     # ---- end to end: pinned host gradients in, update RMS out, every step
     e2e = None
@@ -313,8 +325,8 @@ def main(argv=None) -> int:
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-        e2e = {"value": world * nz_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+        e2e = {"value": replica_tflops(world, nz_flops, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": Gbuf.numel() * 2, "d2h_bytes_per_step": wl.n * 4,
                "path": "MuonPlan.step (C ABI muon_step) with G copied from pinned host memory and the "
                        "update RMS copied back each step"}
