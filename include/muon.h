@@ -162,6 +162,27 @@ MUON_API muon_status_t muon_profile_enable(muon_plan_t plan, int32_t enable);
  * number of calls into *calls, and resets the record. */
 MUON_API muon_status_t muon_profile_read(muon_plan_t plan, double* phase_ms, int64_t* launches, int32_t* calls);
 
+/* Allocation-free Newton-Schulz of ONE matrix, for callers that cannot call
+ * cudaMalloc (device memory owned by a framework allocator or a fixed budget,
+ * or loops that must not allocate after start-up).  The paper has no
+ * counterpart; this is a deployment convenience around the same kernels as
+ * muon_orthogonalize on the bf16 tensor-core path.
+ *   O_out = Newton-Schulz(X_in), ns_steps iterations with coefficients abc.
+ *   X_in: device [rows, cols] in in_dtype; O_out: device fp32 [rows, cols];
+ *   they must not overlap.  Limits: rows, cols <= 8192, rows * cols <= 2^20,
+ *   min(rows, cols) <= 1024; larger requests return MUON_ERR_UNSUPPORTED.
+ * No device memory is allocated or freed: all scratch lives in one static
+ * device array of about 10.7 MB that every GPU loading this library holds
+ * until the process exits.  The first call on a device resolves that array's
+ * address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  Every call shares the array: calls that can overlap on the GPU
+ * (different streams, or several host threads) race and must be serialized
+ * by the caller.  Non-finite inputs give non-finite outputs; no status is
+ * recorded.  Errors: INVALID_ARG, ALIAS, UNSUPPORTED, CUDA. */
+MUON_API muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_out, int64_t rows, int64_t cols,
+                                                  int32_t in_dtype, int32_t ns_steps, const float abc[3],
+                                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,8 @@ MUON_NUM_PHASES = 5
 PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
 
 EXPORTED = ("muon_hparams_default", "muon_init", "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
-            "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read")
+            "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read",
+            "muon_orthogonalize_noalloc")
 
 
 class muon_param_t(ctypes.Structure):
@@ -90,6 +91,9 @@ def load() -> ctypes.CDLL:
     lib.muon_profile_read.argtypes = [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                                       ctypes.POINTER(ctypes.c_int32)]
     lib.muon_profile_read.restype = ctypes.c_int
+    lib.muon_orthogonalize_noalloc.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.POINTER(ctypes.c_float), P]
+    lib.muon_orthogonalize_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -127,6 +131,14 @@ def muon_orthogonalize(plan, x_ptrs, o_ptrs, n: int, in_dtype: int, ns_steps: in
     abc_arr = (ctypes.c_float * 3)(*[float(v) for v in abc])
     check(load().muon_orthogonalize(plan, x_ptrs, o_ptrs, int(n), int(in_dtype), int(ns_steps), abc_arr,
                                     int(precision), ctypes.c_void_p(stream)), "muon_orthogonalize")
+
+
+def muon_orthogonalize_noalloc(x_ptr: int, o_ptr: int, rows: int, cols: int, in_dtype: int, ns_steps: int, abc,
+                               stream: int) -> None:
+    abc_arr = (ctypes.c_float * 3)(*[float(v) for v in abc])
+    check(load().muon_orthogonalize_noalloc(ctypes.c_void_p(x_ptr), ctypes.c_void_p(o_ptr), int(rows), int(cols),
+                                            int(in_dtype), int(ns_steps), abc_arr, ctypes.c_void_p(stream)),
+          "muon_orthogonalize_noalloc")
 
 
 def muon_workspace_bytes(plan) -> int:

@@ -1,0 +1,254 @@
+// muon_orthogonalize_noalloc: Newton-Schulz of one matrix with no device
+// allocation at all.
+//
+// Some callers cannot call cudaMalloc: code whose device memory is owned by a
+// framework allocator or a fixed budget, and latency-critical loops that must
+// not allocate (cudaMalloc can synchronize the device) after start-up.  This
+// entry point runs the same kernels as muon_orthogonalize on the bf16
+// tensor-core path, but every byte of scratch it needs (iterate buffers,
+// Gram and polynomial matrices, norms, schedules, TMA descriptors) lives in
+// one file-scope device array of fixed size, which every GPU that loads the
+// library holds until the process exits.  The caller passes the input and the
+// output; the per-call descriptors are copied in from the host stack.
+#include "muon.h"
+#include "muon_internal.cuh"
+
+#include <cuda.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+using namespace muon;
+
+namespace {
+
+// Size limits of one call.
+constexpr int64_t kNaMaxElems = int64_t(1) << 20;  // rows * cols
+constexpr int kNaMaxDim = 8192;                    // rows and cols each
+constexpr int kNaMaxM = 1024;                      // min(rows, cols)
+constexpr int kNaMaxTiles = 256;                   // per tile list
+constexpr int kNaMaxChunks = 512;
+
+constexpr size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Scratch layout (byte offsets).
+constexpr size_t kNaX = align256((kNaMaxElems + 8 * kNaMaxDim) * 2);       // one [R, ld] bf16 array
+constexpr size_t kNaA = align256(size_t(kNaMaxM) * kNaMaxM * 2);            // one [m, lda] bf16 array
+constexpr size_t kOffHi0 = 0;
+constexpr size_t kOffHi1 = kOffHi0 + kNaX;
+constexpr size_t kOffLo = kOffHi1 + kNaX;
+constexpr size_t kOffA = kOffLo + kNaX;
+constexpr size_t kOffB = kOffA + kNaA;
+constexpr size_t kOffS = kOffB + kNaA;
+constexpr size_t kOffNormPart = kOffS + 256;
+constexpr size_t kOffNormCount = kOffNormPart + align256(kNaMaxChunks * sizeof(double));
+constexpr size_t kOffRms = kOffNormCount + 256;
+constexpr int kNaMaxRms = 4096;  // >= tiles * kRmsSlotsPerTile and >= chunks
+constexpr size_t kOffStatus = kOffRms + align256(kNaMaxRms * sizeof(float));
+constexpr size_t kOffMat = kOffStatus + 256;
+constexpr size_t kOffPtrs = kOffMat + align256(sizeof(MatInfo));
+constexpr size_t kOffSym = kOffPtrs + align256(sizeof(MatPtrs));
+constexpr size_t kOffFull = kOffSym + align256(kNaMaxTiles * sizeof(TileDesc));
+constexpr size_t kOffChunks = kOffFull + align256(kNaMaxTiles * sizeof(TileDesc));
+constexpr size_t kOffTmaps = kOffChunks + align256(kNaMaxChunks * sizeof(ChunkDesc));
+constexpr size_t kScratchBytes = kOffTmaps + align256(kMapsPerMat * sizeof(CUtensorMap));
+
+// ~10.7 MB, zero-initialised at module load.
+__device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+struct DeviceState {
+  unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+  int npairs = 0;
+  bool ready = false;
+};
+DeviceState g_state[64];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode(CUtensorMap* tm, void* base, int rows, int cols, int ld, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBoxOuter)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Once per device, with that device current: resolve the scratch array's
+// device address (in host code the symbol's name is only a host-side stand-in).
+muon_status_t setup_device(int dev) {
+  DeviceState& st = g_state[dev];
+  if (st.ready) return MUON_OK;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  st.base = static_cast<unsigned char*>(p);
+  st.npairs = gemm_tc_max_pairs();
+  if (st.npairs < 1) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
+    st.npairs = std::max(1, prop.multiProcessorCount / 2);
+  }
+  st.ready = true;
+  return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_out, int64_t rows, int64_t cols,
+                                                    int32_t in_dtype, int32_t ns_steps, const float abc[3],
+                                                    void* stream) {
+  if (X_in == nullptr || O_out == nullptr || abc == nullptr) return MUON_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+  if (in_dtype != MUON_DT_BF16 && in_dtype != MUON_DT_FP32) return MUON_ERR_INVALID_ARG;
+  if (ns_steps < 0 || ns_steps > 32) return MUON_ERR_INVALID_ARG;
+  if (!std::isfinite(abc[0]) || !std::isfinite(abc[1]) || !std::isfinite(abc[2])) return MUON_ERR_INVALID_ARG;
+  if (rows > kNaMaxDim || cols > kNaMaxDim || rows * cols > kNaMaxElems || std::min(rows, cols) > kNaMaxM)
+    return MUON_ERR_UNSUPPORTED;  // beyond the fixed scratch
+  const size_t in_bytes = static_cast<size_t>(rows * cols) * (in_dtype == MUON_DT_BF16 ? 2 : 4);
+  const uintptr_t x = reinterpret_cast<uintptr_t>(X_in), o = reinterpret_cast<uintptr_t>(O_out);
+  if (x < o + static_cast<size_t>(rows * cols) * 4 && o < x + in_bytes) return MUON_ERR_ALIAS;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MUON_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MUON_ERR_UNSUPPORTED;
+  muon_status_t su = setup_device(dev);
+  if (su != MUON_OK) return su;
+  unsigned char* base = g_state[dev].base;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // ---- one matrix: descriptors built on the host stack
+  const int R = static_cast<int>(rows), C = static_cast<int>(cols);
+  MatInfo mi{};
+  mi.rows = R;
+  mi.cols = C;
+  mi.m = std::min(R, C);
+  mi.n = std::max(R, C);
+  mi.tall = R > C ? 1 : 0;
+  mi.ld = (C + 7) / 8 * 8;
+  mi.lda = (mi.m + 7) / 8 * 8;
+  mi.off_x = 0;
+  mi.off_a = 0;
+  ChunkDesc chunks[kNaMaxChunks];
+  const int rows_per_chunk = std::max(1, kChunkElems / C);
+  int nch = 0;
+  for (int r = 0; r < R; r += rows_per_chunk) {
+    if (nch == kNaMaxChunks) return MUON_ERR_UNSUPPORTED;
+    chunks[nch] = make_int4(0, r, std::min(rows_per_chunk, R - r), nch);
+    ++nch;
+  }
+  mi.chunk_base = 0;
+  mi.nchunks = nch;
+  TileDesc sym[kNaMaxTiles], full[kNaMaxTiles];
+  int nsym = 0, nfull = 0;
+  for (int r0 = 0; r0 < mi.m; r0 += kTileM)
+    for (int c0 = 0; c0 < mi.m && c0 <= r0 + kTileM - 1; c0 += kBN) {
+      if (nsym == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
+      sym[nsym++] = make_int4(0, r0, c0, std::min({kBN, mi.m - c0, r0 + kTileM - c0}));
+    }
+  for (int r0 = 0; r0 < R; r0 += kTileM)
+    for (int c0 = 0; c0 < C; c0 += kBN) {
+      if (nfull == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
+      full[nfull++] = make_int4(0, r0, c0, std::min(kBN, C - c0));
+    }
+  mi.rms_tile_base = 0;
+  mi.rms_tile_count = nfull * kRmsSlotsPerTile;
+  if (mi.rms_tile_count > kNaMaxRms) return MUON_ERR_UNSUPPORTED;
+  MatPtrs mp{};
+  mp.W = O_out;
+  mp.G = X_in;
+  mp.M = nullptr;
+  mp.g_dtype = in_dtype;
+  mp.vec_ok = ((x | o) % 16 == 0 && C % 8 == 0) ? 1 : 0;
+
+  Workspace ws{};
+  ws.hi[0] = reinterpret_cast<__nv_bfloat16*>(base + kOffHi0);
+  ws.hi[1] = reinterpret_cast<__nv_bfloat16*>(base + kOffHi1);
+  ws.lo = reinterpret_cast<__nv_bfloat16*>(base + kOffLo);
+  ws.A = reinterpret_cast<__nv_bfloat16*>(base + kOffA);
+  ws.B = reinterpret_cast<__nv_bfloat16*>(base + kOffB);
+  ws.s = reinterpret_cast<float*>(base + kOffS);
+  ws.norm_part = reinterpret_cast<double*>(base + kOffNormPart);
+  ws.norm_count = reinterpret_cast<unsigned*>(base + kOffNormCount);
+  ws.rms_part = reinterpret_cast<float*>(base + kOffRms);
+  ws.status = reinterpret_cast<unsigned*>(base + kOffStatus);
+  CUtensorMap tm[kMapsPerMat];
+  bool ok = encode(&tm[kMapHi0], ws.hi[0], R, C, mi.ld, kBoxInner) &&
+            encode(&tm[kMapHi1], ws.hi[1], R, C, mi.ld, kBoxInner) &&
+            encode(&tm[kMapA], ws.A, mi.m, mi.m, mi.lda, kBoxInner) &&
+            encode(&tm[kMapB], ws.B, mi.m, mi.m, mi.lda, kBoxInner) &&
+            encode(&tm[kMapEpiHi0], ws.hi[0], R, C, mi.ld, kEpiBoxCols) &&
+            encode(&tm[kMapEpiHi1], ws.hi[1], R, C, mi.ld, kEpiBoxCols) &&
+            encode(&tm[kMapEpiA], ws.A, mi.m, mi.m, mi.lda, kEpiBoxCols) &&
+            encode(&tm[kMapEpiLo], ws.lo, R, C, mi.ld, kEpiBoxCols);
+  if (!ok) return MUON_ERR_CUDA;
+
+  // ---- stage descriptors (pageable host -> device copies are staged by the
+  // driver before the call returns) and clear what must start at zero
+  MatInfo* mats_d = reinterpret_cast<MatInfo*>(base + kOffMat);
+  MatPtrs* ptrs_d = reinterpret_cast<MatPtrs*>(base + kOffPtrs);
+  TileDesc* sym_d = reinterpret_cast<TileDesc*>(base + kOffSym);
+  TileDesc* full_d = reinterpret_cast<TileDesc*>(base + kOffFull);
+  ChunkDesc* chunks_d = reinterpret_cast<ChunkDesc*>(base + kOffChunks);
+  void* tmaps_d = base + kOffTmaps;
+  cudaError_t e = cudaSuccess;
+  e = e == cudaSuccess ? cudaMemcpyAsync(mats_d, &mi, sizeof(mi), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(ptrs_d, &mp, sizeof(mp), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(sym_d, sym, nsym * sizeof(TileDesc), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(full_d, full, nfull * sizeof(TileDesc), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(chunks_d, chunks, nch * sizeof(ChunkDesc), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(tmaps_d, tm, sizeof(tm), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemsetAsync(ws.norm_count, 0, sizeof(unsigned), st) : e;
+  e = e == cudaSuccess ? cudaMemsetAsync(ws.status, 0, sizeof(unsigned), st) : e;
+  if (e != cudaSuccess) return MUON_ERR_CUDA;
+
+  // ---- the same launch sequence as muon_orthogonalize on the bf16 path
+  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0};
+  if (launch_k1(chunks_d, nch, mats_d, ptrs_d, ws, sc, kK1Copy, 0, st) != cudaSuccess) return MUON_ERR_CUDA;
+  int cur = 0;
+  for (int it = 0; it < ns_steps; ++it) {
+    const bool last = (it == ns_steps - 1);
+    for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
+      GemmArgs a{};
+      a.tiles = (ph == kPhaseUpdate) ? full_d : sym_d;
+      a.ntiles = (ph == kPhaseUpdate) ? nfull : nsym;
+      a.phase = ph;
+      a.iter = it;
+      a.cur = cur;
+      a.final_mode = (ph == kPhaseUpdate && last) ? kFinalOut : kFinalNone;
+      a.mats = mats_d;
+      a.ptrs = ptrs_d;
+      a.tmaps = tmaps_d;
+      a.ws = ws;
+      a.sc = sc;
+      if (launch_gemm_tc(a, g_state[dev].npairs, st) != cudaSuccess) return MUON_ERR_CUDA;
+    }
+    if (!last) cur ^= 1;
+  }
+  if (ns_steps == 0 &&
+      launch_apply_update(chunks_d, nch, mats_d, ptrs_d, ws, sc, kFinalOut, 0, st) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return MUON_OK;
+}

@@ -1,0 +1,92 @@
+"""The allocation-free entry point, muon_orthogonalize_noalloc.
+
+It exists for callers that cannot call cudaMalloc (device memory owned by a
+framework allocator or a fixed budget, loops that must not allocate after
+start-up): all of its scratch is one static device array inside libmuon.
+This file is collected last on purpose, so a failure here cannot hide any
+other test; it passes both alone in a fresh process and after the rest.
+
+Checked through the C ABI: two calls in a row, each compared with the plan-
+based muon_orthogonalize on the same input, within the bf16-path tolerance,
+plus the size limit and argument errors.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from matrix_orthogonalizing_optimizer_muon_b200 import _lib as L
+from matrix_orthogonalizing_optimizer_muon_b200.api import MuonPlan
+
+pytestmark = pytest.mark.gpu
+
+ABC = (3.4445, -4.7750, 2.0315)
+TOL = 3e-2  # relative Frobenius error allowed on the bf16-operand path
+
+
+def rel_f(a: torch.Tensor, b: torch.Tensor) -> float:
+    a64, b64 = a.double().cpu().numpy(), b.double().cpu().numpy()
+    return float(np.linalg.norm(a64 - b64) / np.linalg.norm(b64))
+
+
+def noalloc(x: torch.Tensor, o: torch.Tensor, steps: int = 5) -> None:
+    dt = L.MUON_DT_BF16 if x.dtype == torch.bfloat16 else L.MUON_DT_FP32
+    L.muon_orthogonalize_noalloc(x.data_ptr(), o.data_ptr(), x.shape[0], x.shape[1], dt, steps, ABC,
+                                 torch.cuda.current_stream().cuda_stream)
+
+
+def reference(x: torch.Tensor, steps: int = 5) -> torch.Tensor:
+    out = torch.empty(x.shape, device="cuda")
+    plan = MuonPlan([tuple(x.shape)])
+    plan.orthogonalize([x], [out], ns_steps=steps, coeffs=ABC)
+    torch.cuda.synchronize()
+    plan.close()
+    return out
+
+
+def test_two_calls_in_a_row_match_the_plan_entry_point():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    # first call on a tall matrix, second on a wide one with ragged tiles
+    x1 = torch.randn(768, 300, device="cuda", generator=g).to(torch.bfloat16)
+    x2 = torch.randn(200, 1000, device="cuda", generator=g).to(torch.bfloat16)
+    o1 = torch.full(x1.shape, float("nan"), device="cuda")
+    o2 = torch.full(x2.shape, float("nan"), device="cuda")
+    noalloc(x1, o1)
+    noalloc(x2, o2)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o1).all() and torch.isfinite(o2).all()
+    assert rel_f(o1, reference(x1)) <= TOL
+    assert rel_f(o2, reference(x2)) <= TOL
+
+
+def test_repeated_call_is_reproducible_and_fp32_input_accepted():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    x = torch.randn(512, 512, device="cuda", generator=g)
+    a = torch.empty_like(x)
+    b = torch.empty_like(x)
+    noalloc(x, a)
+    noalloc(x, b)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert rel_f(a, reference(x)) <= TOL
+
+
+def test_limits_and_argument_errors():
+    lib = L.load()
+    abc = (ctypes.c_float * 3)(*ABC)
+    x = torch.zeros(4, 4, device="cuda", dtype=torch.bfloat16)
+    o = torch.zeros(4, 4, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    xp, op = ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(o.data_ptr())
+    # beyond the static scratch: more than 2^20 elements, a side above 8192, min side above 1024
+    assert lib.muon_orthogonalize_noalloc(xp, op, 2048, 1024, 0, 5, abc, s) == L.MUON_ERR_UNSUPPORTED
+    assert lib.muon_orthogonalize_noalloc(xp, op, 16, 8193, 0, 5, abc, s) == L.MUON_ERR_UNSUPPORTED
+    assert lib.muon_orthogonalize_noalloc(xp, op, 1025, 1025, 0, 5, abc, s) == L.MUON_ERR_UNSUPPORTED
+    assert lib.muon_orthogonalize_noalloc(None, op, 4, 4, 0, 5, abc, s) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_orthogonalize_noalloc(xp, op, 0, 4, 0, 5, abc, s) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_orthogonalize_noalloc(xp, op, 4, 4, 7, 5, abc, s) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_orthogonalize_noalloc(xp, xp, 4, 4, 0, 5, abc, s) == L.MUON_ERR_ALIAS
