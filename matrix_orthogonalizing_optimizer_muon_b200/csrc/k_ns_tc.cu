@@ -13,8 +13,8 @@
 // Structure: persistent 2-CTA clusters (one CTA per SM).  A pair owns a
 // 256 x 256 output tile; tcgen05.mma.cta_group::2 (M = 256, N <= 256, K = 16,
 // bf16 operands, fp32 accumulators in TMEM) reads 128 A rows and N/2 B rows
-// from each CTA's shared memory, so each SM streams 32 KiB per 64-deep K step
-// for 4.2 MFLOP.  Per CTA:
+// from each CTA's shared memory, so each SM streams 64 KiB per 128-deep K
+// stage for 16.8 MFLOP of the pair.  Per CTA:
 //   warp 0      TMA producer: four lanes each issue one 64 x 128 bf16 box
 //               (128-byte swizzle) per 128-deep K stage into a ring of 3
 //               stages (2 for the X update, which gives its epilogue the
@@ -22,18 +22,11 @@
 //   warp 1      TMEM allocator (both CTAs) and MMA issuer (leader only); two
 //               256-column accumulators so the epilogue of one tile overlaps
 //               the main loop of the next.
-//   warp 2      epilogue loader: TMA-prefetches the tiles the epilogue reads
-//               (A for the polynomial; the hi/lo iterate for the X update)
-//               into a ring of 64-column slots, ahead of the accumulator.
-//   warps 3..10 epilogue: two warps per TMEM lane quadrant, each taking one
-//               32-column half of every 64-column chunk: tcgen05.ld, fused
-//               arithmetic, vector stores.
-// K-major or MN-major operands are a descriptor choice, so tall matrices are
-// never transposed.  Symmetric outputs (A, B) are computed only for tiles
-// that touch the lower triangle; each entry is written exactly once, directly
-// (i >= j) or through its mirror (i > j), so the result is symmetric bit for
-// bit.  Every mbarrier wait is bounded by time; on timeout the CTA raises a
-// status bit, stops issuing, drains what it has in flight, frees TMEM, exits.
+//   warps 2..9  epilogue: two warps per TMEM lane quadrant, each owning whole
+//               32 x 32 blocks (tcgen05.ld of 32 columns, one row per thread),
+//               fused arithmetic, and coalesced 64-byte row-segment stores
+//               through warp-private swizzled staging blocks.  The X update
+//               feeds its hi/lo inputs through a per-warp cp.async ring.
 #include "muon_internal.cuh"
 
 #include <cuda.h>
@@ -125,10 +118,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
 // arrive on a barrier given by its shared::cluster address (may be the peer's)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -173,15 +162,6 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* tmap, in
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
       "%3}], [%4];" ::"r"(dst),
       "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
-      : "memory");
-}
-
-// TMA load completing on this CTA's own barrier.
-__device__ __forceinline__ void tma_load_local(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
 
@@ -395,35 +375,6 @@ __device__ __forceinline__ void load_row32_masked(const __nv_bfloat16* src, int 
 __device__ __forceinline__ float bf_at(const uint4 (&p)[4], int q) {
   const uint32_t w = reinterpret_cast<const uint32_t*>(&p[q >> 3])[(q & 7) >> 1];
   return __uint_as_float((q & 1) ? (w & 0xFFFF0000u) : (w << 16));
-}
-
-__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const __nv_bfloat16* v) {
-  *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(v);
-}
-
-// Symmetric output: row i, columns j0..j0+31 of an [m, m] matrix.
-__device__ __forceinline__ void store_sym_chunk(__nv_bfloat16* out, int lda, int m, int i, int j0,
-                                                const float* val) {
-  __align__(16) __nv_bfloat16 h[32];
-#pragma unroll
-  for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
-  __nv_bfloat16* row = out + static_cast<size_t>(i) * lda;
-  if (j0 + 31 <= i && j0 + 32 <= m) {
-#pragma unroll
-    for (int q = 0; q < 32; q += 8) store_bf16x8(row + j0 + q, h + q);
-  } else {
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int j = j0 + q;
-      if (j <= i && j < m) row[j] = h[q];
-    }
-  }
-  // mirror of the strictly lower part: out[j, i] for j < i
-#pragma unroll
-  for (int q = 0; q < 32; ++q) {
-    const int j = j0 + q;
-    if (j < i && j < m) out[static_cast<size_t>(j) * lda + i] = h[q];
-  }
 }
 
 // ---------------------------------------------------------------- the kernel
