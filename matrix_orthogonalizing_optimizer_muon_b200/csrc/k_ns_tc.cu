@@ -13,20 +13,25 @@
 // Structure: persistent 2-CTA clusters (one CTA per SM).  A pair owns a
 // 256 x 256 output tile; tcgen05.mma.cta_group::2 (M = 256, N <= 256, K = 16,
 // bf16 operands, fp32 accumulators in TMEM) reads 128 A rows and N/2 B rows
-// from each CTA's shared memory, so each SM streams 64 KiB per 128-deep K
-// stage for 16.8 MFLOP of the pair.  Per CTA:
-//   warp 0      TMA producer: four lanes each issue one 64 x 128 bf16 box
-//               (128-byte swizzle) per 128-deep K stage into a ring of 3
-//               stages (2 for the X update, which gives its epilogue the
-//               room); both CTAs' loads complete on the leader's "full" barrier.
+// from each CTA's shared memory, so each SM streams 32 KiB per 64-deep K
+// stage for 8.4 MFLOP of the pair.  The operand stream is latency bound (a
+// stage takes about two stage-times of MMA to arrive), so the ring is as deep
+// as shared memory allows: 6 stages for the Gram and polynomial phases, 4 for
+// the X update, whose epilogue also stages its hi/lo inputs.  Per CTA:
+//   warps 0, 10 TMA producers for the even and the odd stages: up to four
+//               lanes issue one box each per stage in a single instruction
+//               (a 64 x 128 K-major box, or 64 x 64 boxes for MN-major
+//               operands and narrow K-major ones); both CTAs' loads complete
+//               on the leader's "full" barrier.
 //   warp 1      TMEM allocator (both CTAs) and MMA issuer (leader only); two
 //               256-column accumulators so the epilogue of one tile overlaps
 //               the main loop of the next.
 //   warps 2..9  epilogue: two warps per TMEM lane quadrant, each owning whole
-//               32 x 32 blocks (tcgen05.ld of 32 columns, one row per thread),
-//               fused arithmetic, and coalesced 64-byte row-segment stores
-//               through warp-private swizzled staging blocks.  The X update
-//               feeds its hi/lo inputs through a per-warp cp.async ring.
+//               32 x 32 blocks (tcgen05.ld of 32 columns, one row per thread)
+//               and the fused arithmetic.  Results go through a warp-private
+//               swizzled staging block to TMA bulk stores, so the load/store
+//               units and the L1 path stay free for the inputs (the X
+//               update's hi/lo via a per-warp cp.async ring).
 #include "muon_internal.cuh"
 
 #include <cuda.h>
@@ -34,45 +39,51 @@
 namespace muon {
 namespace {
 
-#ifndef MUON_TC_STAGES
-#define MUON_TC_STAGES 3
+#ifndef MUON_TC_STAGES_SYM
+#define MUON_TC_STAGES_SYM 6
 #endif
-constexpr int kStages = MUON_TC_STAGES;   // stages of the Gram and polynomial phases
-constexpr int kStagesUpd = 2;              // stages of the X-update phase
-constexpr int kStageABytes = kHalfM * kBK * 2;   // 32 KiB: this CTA's 128 A rows x 128 K
-constexpr int kStageBBytes = 128 * kBK * 2;      // 32 KiB: up to 128 B rows (half of N) x 128 K
+#ifndef MUON_TC_STAGES_UPD
+#define MUON_TC_STAGES_UPD 4
+#endif
+constexpr int kStagesSym = MUON_TC_STAGES_SYM;  // stages of the Gram and polynomial phases
+constexpr int kStagesUpd = MUON_TC_STAGES_UPD;  // stages of the X-update phase
+constexpr int kStagesMax = kStagesSym > kStagesUpd ? kStagesSym : kStagesUpd;
+constexpr int kOpBytes = kHalfM * kBK * 2;      // 16 KiB: one operand's share of a stage in one CTA
+constexpr int kStageBytes = 2 * kOpBytes;       // A then B
+constexpr int kBox128Bytes = kBoxInner * 128 * 2;  // 16 KiB
+constexpr int kBox64Bytes = kBoxInner * 64 * 2;    // 8 KiB
 // Epilogue: two groups of four warps (one warp per TMEM lane quadrant each);
 // group g takes the 32-column chunks g, g+2, ... of every tile, so each warp
-// owns whole 32 x 32 blocks.  Each warp has 4 KiB of shared memory: two
-// 32 x 32 bf16 blocks through which its inputs and outputs are transposed
-// between coalesced global accesses (64-byte row segments) and the
-// row-per-thread layout of the TMEM accumulator.  The epilogue uses no TMA,
-// so its traffic never queues behind the main loop's operand copies.
+// owns whole 32 x 32 blocks.  Each warp has 4 KiB of staging: two 32 x 32 bf16
+// blocks in the 64-byte-swizzled layout of a 32 x 32 TMA store box.
 constexpr int kEpiGroups = 2;
 constexpr int kEpiBlockBytes = 32 * 32 * 2;               // 2 KiB
 constexpr int kEpiWarpBytes = 2 * kEpiBlockBytes;         // 4 KiB
 constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;      // 32 KiB
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
-constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);
+constexpr int kWarpProducer2 = kWarpEpi0 + kEpiWarps;  // second producer warp (odd stages)
+constexpr int kThreads = 32 * (kWarpProducer2 + 1);
+static_assert(MUON_TC_STAGES_SYM % 2 == 0 && MUON_TC_STAGES_UPD % 2 == 0,
+              "the two producer warps own the even and the odd stages");
 
-// X-update epilogue: per warp a ring of 3 buffers, each a 32 x 32 hi block and
-// lo block (4 KiB), filled by cp.async.  With 2 main-loop stages the free
-// shared memory is [64 KiB, 96 KiB) and [160 KiB, 224 KiB): 24 buffers.
-constexpr int kUpdBufs = 3;
+// X-update inputs: per warp a ring of 2 buffers, each a 32 x 32 hi block and
+// lo block (4 KiB), filled by cp.async two chunks ahead.
+constexpr int kUpdBufs = 2;
 constexpr int kUpdBufBytes = 2 * kEpiBlockBytes;
 
 struct SmemLayout {
-  static constexpr int kA = 0;
-  static constexpr int kB = kA + kStages * kStageABytes;
-  static constexpr int kEpi = kB + kStages * kStageBBytes;
-  static constexpr int kUpdLo = kA + kStagesUpd * kStageABytes;  // [64 KiB, 96 KiB)
-  static constexpr int kUpdHi = kB + kStagesUpd * kStageBBytes;  // [160 KiB, 224 KiB)
+  static constexpr int kStages = 0;                                   // stage s at s * kStageBytes
+  static constexpr int kUpdRing = kStagesUpd * kStageBytes;           // X update only
+  static constexpr int kEpi = kStagesSym * kStageBytes;               // staging blocks
   static constexpr int kBar = kEpi + kEpiBytes;
   // full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kNumBars = 2 * kStagesMax + 5;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort (int)
   static constexpr int kBytes = kMisc + 16;
 };
+static_assert(SmemLayout::kUpdRing + kEpiWarps * kUpdBufs * kUpdBufBytes <= SmemLayout::kEpi,
+              "X-update ring overlaps the staging blocks");
+static_assert(kStagesUpd * kStageBytes <= SmemLayout::kEpi, "stages overlap the staging blocks");
 constexpr int kSmemBytes = SmemLayout::kBytes + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -165,6 +176,26 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* tmap, in
       : "memory");
 }
 
+// Bring a tensor map into the TMA descriptor cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// TMA bulk store of a staged box: shared::cta -> global, tracked by this
+// thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap), "r"(x),
+               "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every committed bulk store of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -200,11 +231,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout.
-// A stage holds each operand as two 16 KiB TMA boxes (64 contiguous x 128).
-//   K-major : box h holds K [64h, 64h+64) for 128 rows, one 128-byte row per
-//             MN index; SBO = 1024 B between 8-row groups, LBO unused (16 B).
-//   MN-major: box h holds MN [64h, 64h+64) for all 128 k, one 128-byte row per
-//             k; SBO = 1024 B between 8-k groups, LBO = 16 KiB between boxes.
+// A stage holds each operand's 64-deep K slice in 16 KiB:
+//   K-major : one box, K [0, 64) for up to 128 rows, one 128-byte row per MN
+//             index; SBO = 1024 B between 8-row groups, LBO unused (16 B).
+//   MN-major: box h (8 KiB) holds MN [64h, 64h+64) for the 64 k, one 128-byte
+//             row per k; SBO = 1024 B between 8-k groups, LBO = 8 KiB between
+//             boxes.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
@@ -223,18 +255,40 @@ __device__ __forceinline__ uint32_t make_idesc(int n, int a_mn, int b_mn) {
 }
 
 // ---------------------------------------------------------------- tile decoding
+// One operand's per-CTA share of a stage: `nbox` boxes of `box_bytes` each,
+// loaded from `tmap`.
 struct Operand {
   const void* tmap;
-  int mn;  // 1: MN-major (column-contiguous), 0: K-major
+  int mn;         // 1: MN-major (column-contiguous), 0: K-major
+  int nbox;       // 1 or 2
+  int box_bytes;  // kBox128Bytes or kBox64Bytes
 };
 
 struct TileCfg {
-  int p, row0, col0, n_need, n_mma, half, nb_b, nk, nch, skip;
+  int p, row0, col0, n_need, n_mma, half, nk, nch, skip;
   Operand a, b;
 };
 
 __device__ __forceinline__ const void* tmap_of(const GemmArgs& g, int p, int which) {
   return static_cast<const uint8_t*>(g.tmaps) + (static_cast<size_t>(p) * kMapsPerMat + which) * 128;
+}
+
+// Operand over the array with 128-row map `map128` (its 64-row map is
+// map128 + 4) spanning `extent` MN indices in this CTA.
+__device__ __forceinline__ Operand make_operand(const GemmArgs& g, int p, int map128, int mn, int extent) {
+  Operand o;
+  o.mn = mn;
+  if (mn) {
+    o.tmap = tmap_of(g, p, map128 + 4);
+    o.nbox = extent > kBoxInner ? 2 : 1;
+    o.box_bytes = kBox64Bytes;
+  } else {
+    const bool narrow = extent <= 64;
+    o.tmap = tmap_of(g, p, narrow ? map128 + 4 : map128);
+    o.nbox = 1;
+    o.box_bytes = narrow ? kBox64Bytes : kBox128Bytes;
+  }
+  return o;
 }
 
 __device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) {
@@ -248,28 +302,27 @@ __device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) {
   c.half = c.n_mma >> 1;
   c.nch = (c.n_need + kEpiBoxCols - 1) / kEpiBoxCols;
   const MatInfo& mi = g.mats[c.p];
-  const int hi = g.cur;  // tensor maps 0/1 = hi buffers
+  const int hi = kMapHi0 + g.cur;
   int K;
   if (g.phase == kPhaseGram) {
     K = mi.n;
-    c.a = {tmap_of(g, c.p, hi), mi.tall};
-    c.b = c.a;
+    c.a = make_operand(g, c.p, hi, mi.tall, kHalfM);
+    c.b = make_operand(g, c.p, hi, mi.tall, c.half);
   } else if (g.phase == kPhasePoly) {
     K = mi.m;
-    c.a = {tmap_of(g, c.p, 2), 0};
-    c.b = c.a;
+    c.a = make_operand(g, c.p, kMapA, 0, kHalfM);
+    c.b = make_operand(g, c.p, kMapA, 0, c.half);
   } else {
     K = mi.m;
     if (mi.tall) {
-      c.a = {tmap_of(g, c.p, hi), 0};
-      c.b = {tmap_of(g, c.p, 3), 0};
+      c.a = make_operand(g, c.p, hi, 0, kHalfM);
+      c.b = make_operand(g, c.p, kMapB, 0, c.half);
     } else {
-      c.a = {tmap_of(g, c.p, 3), 0};
-      c.b = {tmap_of(g, c.p, hi), 1};
+      c.a = make_operand(g, c.p, kMapB, 0, kHalfM);
+      c.b = make_operand(g, c.p, hi, 1, c.half);
     }
   }
   c.nk = (K + kBK - 1) / kBK;
-  c.nb_b = c.b.mn ? (c.half + kBoxInner - 1) / kBoxInner : 2;  // B boxes per CTA
   c.skip = (g.ws.s[c.p] == 0.0f) ? 1 : 0;
   return c;
 }
@@ -323,19 +376,6 @@ __device__ __forceinline__ void put_block32(uint8_t* blk, int lane, const uint4 
   for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(blk + chunk_off(8 * k + (lane >> 2), c16)) = in[k];
 }
 
-// Copy a staged 32 x 32 block to out[(g_row0 + rr) * ld + g_col0 + cc]: every
-// warp store writes eight full 64-byte row segments.
-__device__ __forceinline__ void store_block32(const uint8_t* blk, __nv_bfloat16* out, int ld, int g_row0, int g_col0,
-                                              int lane) {
-  const int c16 = lane & 3;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int rr = 8 * k + (lane >> 2);
-    const uint4 v = *reinterpret_cast<const uint4*>(blk + chunk_off(rr, c16));
-    *reinterpret_cast<uint4*>(out + static_cast<size_t>(g_row0 + rr) * ld + g_col0 + c16 * 8) = v;
-  }
-}
-
 // Asynchronous (cp.async, no registers) copy of a 32 x 32 bf16 block
 // src[(g_row0 + rr) * ld + g_col0 + cc] into a staging block, 16 bytes per
 // lane per row segment; completion is tracked by cp.async groups.
@@ -385,10 +425,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + SmemLayout::kBar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStagesMax + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStagesMax + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStagesMax + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kStagesMax + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::kMisc + 4);
 
@@ -398,9 +438,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool leader = (rank == 0);
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
+  const int nst = (g.phase == kPhaseUpdate) ? kStagesUpd : kStagesSym;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesMax; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
@@ -425,25 +466,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   unsigned* status = g.ws.status;
 
-  if (warp == kWarpProducer) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    // Lanes 0..3 each issue one 16 KiB box per stage (A k-half 0, A k-half 1,
-    // B box 0, B box 1): TMA throughput per SM grows with the number of
-    // threads issuing, so one thread per box keeps the copies in flight
-    // concurrently.  Lane 0 owns the barriers.
-    const int nst = (g.phase == kPhaseUpdate) ? kStagesUpd : kStages;
-    int stage = 0;
-    uint32_t phase = 0;
-    long fills = 0;
+  if (warp == kWarpProducer || warp == kWarpProducer2) {
+    // ------------------------------------------------------------ TMA producers (both CTAs)
+    // Two warps take alternate stages, so two stage fills are being issued at
+    // any time (one thread issues about one TMA instruction per few hundred
+    // ns).  Within a warp, lane l < nbox_a loads A box l and the next lanes the
+    // B boxes, all in one instruction; lane 0 owns the barriers.
+    const int pp = (warp == kWarpProducer) ? 0 : 1;
+    long fills = 0;  // fills of both producers, in order
     for (int t = pair; t < g.ntiles; t += npairs) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
       const TileCfg c = decode_tile(g, t);
       if (c.skip) continue;
-      const uint32_t bytes = static_cast<uint32_t>(2 * (2 + c.nb_b) * kBoxBytes);
+      const uint32_t bytes =
+          static_cast<uint32_t>(2 * (c.a.nbox * c.a.box_bytes + c.b.nbox * c.b.box_bytes));
       const int arow = c.row0 + static_cast<int>(rank) * kHalfM;
       const int brow = c.col0 + static_cast<int>(rank) * c.half;
+      if (lane == 0) prefetch_tensormap(c.a.tmap);
+      if (lane == 1) prefetch_tensormap(c.b.tmap);
       bool ok = true;
-      for (int kb = 0; kb < c.nk; ++kb) {
+      for (int kb = 0; kb < c.nk; ++kb, ++fills) {
+        if ((fills & 1) != pp) continue;
+        const int stage = static_cast<int>(fills % nst);
+        const uint32_t phase = static_cast<uint32_t>((fills / nst) & 1);
         int ready = 0;
         if (lane == 0) {
           ready = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag) ? 1 : 0;
@@ -456,30 +501,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t fb = map_to_rank(full_bar(stage), 0);
-        const uint32_t sa = sbase + SmemLayout::kA + stage * kStageABytes;
-        const uint32_t sb = sbase + SmemLayout::kB + stage * kStageBBytes;
+        const uint32_t sa = sbase + SmemLayout::kStages + stage * kStageBytes;
+        const uint32_t sb = sa + kOpBytes;
         const int k0 = kb * kBK;
-        if (lane < 2) {
-          const int h = lane;
-          if (c.a.mn) tma_load_pair(sa + h * kBoxBytes, c.a.tmap, arow + h * kBoxInner, k0, fb);
-          else        tma_load_pair(sa + h * kBoxBytes, c.a.tmap, k0 + h * kBoxInner, arow, fb);
-        } else if (lane < 2 + c.nb_b) {
-          const int h = lane - 2;
-          if (c.b.mn) tma_load_pair(sb + h * kBoxBytes, c.b.tmap, brow + h * kBoxInner, k0, fb);
-          else        tma_load_pair(sb + h * kBoxBytes, c.b.tmap, k0 + h * kBoxInner, brow, fb);
-        }
-        ++fills;
-        if (++stage == nst) {
-          stage = 0;
-          phase ^= 1u;
+        const bool is_a = lane < c.a.nbox;
+        const Operand& o = is_a ? c.a : c.b;
+        const int h = is_a ? lane : lane - c.a.nbox;
+        if (lane < c.a.nbox + c.b.nbox) {
+          const int mn0 = (is_a ? arow : brow) + h * kBoxInner;
+          const uint32_t dst = (is_a ? sa : sb) + h * kBox64Bytes;
+          tma_load_pair(dst, o.tmap, o.mn ? mn0 : k0, o.mn ? k0 : mn0 - h * kBoxInner, fb);
         }
       }
       if (!ok) break;
     }
     // Drain (leader): both CTAs' loads complete on the leader's barriers,
-    // so every stage's most recent fill must have landed before exit.
+    // so the most recent fill of each of this warp's stages must have landed
+    // before exit.
     if (leader && lane == 0) {
-      for (int s = 0; s < nst; ++s) {
+      for (int s = pp; s < nst; s += 2) {
         const long cnt = fills / nst + ((s < fills % nst) ? 1 : 0);
         if (cnt > 0 && !wait_bounded(full_bar(s), static_cast<uint32_t>((cnt - 1) & 1), nullptr))
           atomicOr(status, kStatusTimeout);
@@ -488,7 +528,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     if (leader && lane == 0) {
-      const int nst = (g.phase == kPhaseUpdate) ? kStagesUpd : kStages;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -504,16 +543,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         const uint32_t idesc = make_idesc(c.n_mma, c.a.mn, c.b.mn);
-        const uint32_t a_lbo = c.a.mn ? kBoxBytes : 16u, b_lbo = c.b.mn ? kBoxBytes : 16u;
+        const uint32_t a_lbo = c.a.mn ? kBox64Bytes : 16u, b_lbo = c.b.mn ? kBox64Bytes : 16u;
         // descriptor start-address fields advance by (byte offset >> 4); shared
         // addresses stay below 256 KiB, so the 14-bit field never carries
-        const uint64_t a_desc0 = smem_desc(sbase + SmemLayout::kA, a_lbo, 1024u);
-        const uint64_t b_desc0 = smem_desc(sbase + SmemLayout::kB, b_lbo, 1024u);
+        const uint64_t a_desc0 = smem_desc(sbase + SmemLayout::kStages, a_lbo, 1024u);
+        const uint64_t b_desc0 = smem_desc(sbase + SmemLayout::kStages + kOpBytes, b_lbo, 1024u);
         // byte offset of MMA k-step kk (16 deep) inside a stage: MN-major moves
-        // down 16 rows of 128 B; K-major moves 32 B inside a box, then to box 1
+        // down 16 rows of 128 B, K-major 32 B along the swizzled row
         auto koff = [](int mn, int kk) -> uint64_t {
-          return mn ? static_cast<uint64_t>(kk * 2048) >> 4
-                    : static_cast<uint64_t>((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+          return static_cast<uint64_t>(mn ? kk * 2048 : kk * 32) >> 4;
         };
         bool ok = true;
         for (int kb = 0; kb < c.nk; ++kb) {
@@ -523,11 +561,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * kStageABytes) >> 4);
-          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * kStageBBytes) >> 4);
+          const uint64_t so = static_cast<uint64_t>((stage * kStageBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-            tc_mma_pair(d_tmem, ad + koff(c.a.mn, kk), bd + koff(c.b.mn, kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_pair(d_tmem, a_desc0 + so + koff(c.a.mn, kk), b_desc0 + so + koff(c.b.mn, kk), idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
           issued = true;
           // free the stage in both CTAs once these MMAs have read it
           tc_commit(empty_bar(stage));
@@ -553,9 +591,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int ew = warp - kWarpEpi0;          // 0..kEpiWarps-1
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
     const int grp = ew >> 2;                  // chunk group: 32-column chunks grp, grp + 2, ...
-    // warp-private staging: two 32 x 32 bf16 blocks (64-byte rows, swizzled)
+    // warp-private staging for the TMA stores: two 32 x 32 bf16 blocks
     uint8_t* blk0 = smem + SmemLayout::kEpi + ew * kEpiWarpBytes;
     uint8_t* blk1 = blk0 + kEpiBlockBytes;
+    const uint32_t blk0_s = smem_u32(blk0), blk1_s = smem_u32(blk1);
+    // the staging blocks may be rewritten once this warp's earlier bulk
+    // stores have read them (lane 0 issues and tracks them)
+    auto staging_free = [&]() {
+      if (lane == 0) bulk_wait_read();
+      __syncwarp();
+    };
+    // stage this thread's row of both blocks, then store them (lane 0)
+    auto publish = [&](const void* map0, int x0, int y0, const void* map1, int x1, int y1) {
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(map0, blk0_s, x0, y0);
+        tma_store_2d(map1, blk1_s, x1, y1);
+        bulk_commit();
+      }
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     const float a_c = g.sc.a, b_c = g.sc.b, c_c = g.sc.c;
@@ -592,26 +647,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const __nv_bfloat16* in1 = g.ws.lo + mi.off_x;
         const int ld_in = upd ? mi.ld : mi.lda;
         const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
-        const int nin = (g.phase == kPhaseGram) ? 0 : (upd ? 2 : 1);
+        const bool poly = (g.phase == kPhasePoly);
         // a chunk needs work unless it is a block strictly above the diagonal
         // of a symmetric output (its mirror writes it)
         auto needed = [&](int ch) { return !(sym && (c.col0 + ch * kEpiBoxCols > i_lo + 31)); };
         auto block_inside = [&](int ch) {
           return i_lo + 31 < rows_in && c.col0 + ch * kEpiBoxCols + 32 <= cols_in;
         };
-        // coalesced prefetch of one chunk's input blocks into registers
-        uint4 pf0[4], pf1[4];
+        // polynomial: coalesced prefetch of the next A block into registers
+        uint4 pf0[4];
         auto prefetch = [&](int ch) {
-          if (nin == 0 || !needed(ch) || !block_inside(ch)) return;
-          const int j0 = c.col0 + ch * kEpiBoxCols;
-          load_block32(in0, ld_in, i_lo, j0, lane, pf0);
-          if (nin == 2) load_block32(in1, ld_in, i_lo, j0, lane, pf1);
+          if (!poly || !needed(ch) || !block_inside(ch)) return;
+          load_block32(in0, ld_in, i_lo, c.col0 + ch * kEpiBoxCols, lane, pf0);
         };
-        // X update: a per-warp ring of kUpdBufs buffers (hi, lo) fed by cp.async,
-        // up to three chunks ahead; the polynomial prefetches into registers
+        // X update: ring of kUpdBufs (hi, lo) buffers fed by cp.async; chunk k
+        // of this warp lives in buffer k % kUpdBufs
         auto upd_buf = [&](int b) -> uint8_t* {
-          const int id = ew * kUpdBufs + b;
-          return smem + (id < 8 ? SmemLayout::kUpdLo + id * kUpdBufBytes : SmemLayout::kUpdHi + (id - 8) * kUpdBufBytes);
+          return smem + SmemLayout::kUpdRing + (ew * kUpdBufs + b) * kUpdBufBytes;
         };
         int kc = 0;  // chunks of this warp in this tile
         for (int x = grp; x < c.nch; x += kEpiGroups) ++kc;
@@ -650,41 +702,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(t_row + static_cast<uint32_t>(ch * kEpiBoxCols), v);  // completes at tmem_ld_wait
-          // land this chunk's prefetched inputs in the warp's staging blocks,
-          // then start fetching the next chunk
-          uint4 xa[4], xb[4];  // this thread's row, packed bf16
-          uint8_t* ub = upd ? upd_buf(k % kUpdBufs) : nullptr;
+          uint4 xa[4], xb[4];  // this thread's row of the inputs, packed bf16
           if (upd) {
             if (inside) {
               cp_async_wait(issued - k - 1);
               __syncwarp();
-              read_row32(ub, lane, xa);
-              read_row32(ub + kEpiBlockBytes, lane, xb);
+              read_row32(upd_buf(k % kUpdBufs), lane, xa);
+              read_row32(upd_buf(k % kUpdBufs) + kEpiBlockBytes, lane, xb);
+              __syncwarp();
             } else {
               load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
               load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
             }
-          } else if (nin > 0) {
+            // this buffer is free again: fetch the chunk two ahead into it
+            if (issued < kc) {
+              stage_chunk(issued);
+              ++issued;
+            }
+          } else if (poly) {
             if (inside) {
+              staging_free();
               put_block32(blk0, lane, pf0);
-              if (nin == 2) put_block32(blk1, lane, pf1);
               __syncwarp();
               read_row32(blk0, lane, xa);
-              if (nin == 2) read_row32(blk1, lane, xb);
               __syncwarp();
             } else {
               load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
-              if (nin == 2) load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
             }
+            if (ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
           }
-          if (!upd && ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
           tmem_ld_wait();
           float val[32];
           if (g.phase == kPhaseGram) {
             const bool first = (g.iter == 0);
 #pragma unroll
             for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
-          } else if (g.phase == kPhasePoly) {
+          } else if (poly) {
 #pragma unroll
             for (int q = 0; q < 32; ++q) val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q));
           } else {
@@ -693,21 +746,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q) + bf_at(xb, q), u2f(v[q]));
           }
           if (sym) {
-            __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
             __align__(16) __nv_bfloat16 h[32];
 #pragma unroll
             for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
             if (inside && j0 + 31 < i_lo) {
               // strictly lower block: stage it and its transpose, store both
-              // as 64-byte row segments
+              staging_free();
               write_row32(blk0, lane, h);
 #pragma unroll
               for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
-              __syncwarp();
-              store_block32(blk0, out, mi.lda, i_lo, j0, lane);
-              store_block32(blk1, out, mi.lda, j0, i_lo, lane);
+              const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
+              publish(map, j0, i_lo, map, i_lo, j0);
             } else {
               // diagonal or ragged block: element-wise with masks
+              __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
               __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
 #pragma unroll
               for (int q = 0; q < 32; ++q) {
@@ -726,15 +778,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               h[q] = __float2bfloat16_rn(val[q]);
               l[q] = __float2bfloat16_rn(val[q] - __bfloat162float(h[q]));
             }
-            __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
-            __nv_bfloat16* lout = g.ws.lo + mi.off_x;
             if (inside) {
-              write_row32(ub, lane, h);
-              write_row32(ub + kEpiBlockBytes, lane, l);
-              __syncwarp();
-              store_block32(ub, hout, mi.ld, i_lo, j0, lane);
-              store_block32(ub + kEpiBlockBytes, lout, mi.ld, i_lo, j0, lane);
+              staging_free();
+              write_row32(blk0, lane, h);
+              write_row32(blk1, lane, l);
+              publish(tmap_of(g, c.p, kMapStHi0 + (g.cur ^ 1)), j0, i_lo, tmap_of(g, c.p, kMapStLo), j0, i_lo);
             } else if (i < mi.rows) {
+              __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
+              __nv_bfloat16* lout = g.ws.lo + mi.off_x;
               const size_t wi = static_cast<size_t>(i) * mi.ld + j0;
 #pragma unroll
               for (int q = 0; q < 32; ++q)
@@ -780,11 +831,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               }
             }
           }
-          if (upd && issued < kc) {
-            __syncwarp();  // every lane is done with this buffer before it is refilled
-            stage_chunk(issued);
-            ++issued;
-          }
         }
         tc_fence_before();
         __syncwarp();
@@ -802,7 +848,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may land in freed shared memory
+    // nothing may still read or land in shared memory once the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+    asm volatile("cp.async.wait_all;" ::: "memory");
   }
 
   tc_fence_before();

@@ -50,20 +50,45 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // 2-D bf16 tensor map over a [rows, cols] array with row pitch `ld`
-// elements and boxes of `box_cols` (contiguous) x 128 rows; zero fill
-// outside.  64-column boxes use the 128-byte swizzle (tensor-core operands),
-// 32-column boxes the 64-byte swizzle (epilogue staging).
-bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld, int box_cols) {
+// elements; boxes of box_cols (contiguous) x box_rows, zero fill outside.
+// 64-column boxes use the 128-byte swizzle (tensor-core operands), 32-column
+// boxes the 64-byte swizzle (epilogue staging blocks).
+bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld, int box_cols, int box_rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBoxOuter)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle swz = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+// Operand maps (64 x 128 and 64 x 64 boxes) and epilogue store maps (32 x 32)
+// of one matrix's workspace arrays, in MapIndex order.
+bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0, __nv_bfloat16* hi1,
+                              __nv_bfloat16* lo, __nv_bfloat16* A, __nv_bfloat16* B) {
+  CUtensorMap* t = static_cast<CUtensorMap*>(maps);
+  const int R = mi.rows, C = mi.cols, m = mi.m;
+  return encode_bf16_2d(t + kMapHi0, hi0, R, C, mi.ld, kBoxInner, 128) &&
+         encode_bf16_2d(t + kMapHi1, hi1, R, C, mi.ld, kBoxInner, 128) &&
+         encode_bf16_2d(t + kMapA, A, m, m, mi.lda, kBoxInner, 128) &&
+         encode_bf16_2d(t + kMapB, B, m, m, mi.lda, kBoxInner, 128) &&
+         encode_bf16_2d(t + kMapHi0S, hi0, R, C, mi.ld, kBoxInner, 64) &&
+         encode_bf16_2d(t + kMapHi1S, hi1, R, C, mi.ld, kBoxInner, 64) &&
+         encode_bf16_2d(t + kMapAS, A, m, m, mi.lda, kBoxInner, 64) &&
+         encode_bf16_2d(t + kMapBS, B, m, m, mi.lda, kBoxInner, 64) &&
+         encode_bf16_2d(t + kMapStHi0, hi0, R, C, mi.ld, kEpiBoxCols, 32) &&
+         encode_bf16_2d(t + kMapStHi1, hi1, R, C, mi.ld, kEpiBoxCols, 32) &&
+         encode_bf16_2d(t + kMapStLo, lo, R, C, mi.ld, kEpiBoxCols, 32) &&
+         encode_bf16_2d(t + kMapStA, A, m, m, mi.lda, kEpiBoxCols, 32) &&
+         encode_bf16_2d(t + kMapStB, B, m, m, mi.lda, kEpiBoxCols, 32);
+}
+
+namespace {
 
 struct ProfRec {
   int first_event;
@@ -453,20 +478,12 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   pl->chunks_d = reinterpret_cast<ChunkDesc*>(b + o_chunks);
   pl->tmaps_d = b + o_tmaps;
 
-  // ---- TMA descriptors: hi0, hi1, A, B, lo per matrix
+  // ---- TMA descriptors per matrix
   std::vector<CUtensorMap> tmaps(static_cast<size_t>(n) * kMapsPerMat);
   for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];
-    CUtensorMap* t = &tmaps[static_cast<size_t>(kMapsPerMat) * i];
-    bool ok = encode_bf16_2d(t + kMapHi0, ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld, kBoxInner) &&
-              encode_bf16_2d(t + kMapHi1, ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld, kBoxInner) &&
-              encode_bf16_2d(t + kMapA, ws.A + mi.off_a, mi.m, mi.m, mi.lda, kBoxInner) &&
-              encode_bf16_2d(t + kMapB, ws.B + mi.off_a, mi.m, mi.m, mi.lda, kBoxInner) &&
-              encode_bf16_2d(t + kMapEpiHi0, ws.hi[0] + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols) &&
-              encode_bf16_2d(t + kMapEpiHi1, ws.hi[1] + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols) &&
-              encode_bf16_2d(t + kMapEpiA, ws.A + mi.off_a, mi.m, mi.m, mi.lda, kEpiBoxCols) &&
-              encode_bf16_2d(t + kMapEpiLo, ws.lo + mi.off_x, mi.rows, mi.cols, mi.ld, kEpiBoxCols);
-    if (!ok) {
+    if (!encode_matrix_maps(&tmaps[static_cast<size_t>(kMapsPerMat) * i], mi, ws.hi[0] + mi.off_x,
+                            ws.hi[1] + mi.off_x, ws.lo + mi.off_x, ws.A + mi.off_a, ws.B + mi.off_a)) {
       free_plan(pl);
       return MUON_ERR_CUDA;
     }

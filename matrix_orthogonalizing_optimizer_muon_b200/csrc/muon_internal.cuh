@@ -28,11 +28,9 @@ namespace muon {
 constexpr int kTileM = 256;     // output rows per tile (two CTAs x 128 TMEM lanes)
 constexpr int kHalfM = 128;     // output rows per CTA
 constexpr int kBN = 256;        // output columns per tile = max UMMA N
-constexpr int kBK = 128;        // K per pipeline stage (two 128-byte swizzle atoms of bf16)
+constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle atom of bf16)
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-constexpr int kBoxInner = 64;   // every TMA box is 64 (contiguous) x 128 bf16 = 16 KiB
-constexpr int kBoxOuter = 128;
-constexpr int kBoxBytes = kBoxInner * kBoxOuter * 2;
+constexpr int kBoxInner = 64;   // operand boxes: 64 contiguous bf16 (128 bytes) x 128 or 64 rows
 constexpr int kEpiWarps = 8;    // epilogue warps per CTA (two per TMEM lane quadrant)
 constexpr int kRmsSlotsPerTile = 2 * kEpiWarps;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators per CTA
@@ -40,12 +38,17 @@ constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators per CTA
 constexpr int kChunkElems = 32768;  // elements per momentum/normalise chunk
 constexpr int kEwThreads = 256;
 constexpr int kT32 = 64;           // fp32 path tile edge
-// TMA descriptors per matrix: main-loop operand maps hi0, hi1, A, B (64 x 128
-// boxes, 128-byte swizzle) and epilogue maps hi0, hi1, A, lo (32 x 128 boxes,
-// 64-byte swizzle)
-constexpr int kMapsPerMat = 8;
-enum MapIndex : int { kMapHi0 = 0, kMapHi1 = 1, kMapA = 2, kMapB = 3, kMapEpiHi0 = 4, kMapEpiHi1 = 5, kMapEpiA = 6,
-                      kMapEpiLo = 7 };
+// TMA descriptors per matrix (128 bytes each):
+//   kMapHi0..kMapB     operand boxes of 64 x 128 rows, 128-byte swizzle (K-major loads)
+//   kMapHi0S..kMapBS   operand boxes of 64 x 64 rows, 128-byte swizzle (MN-major loads,
+//                      and K-major loads of at most 64 rows)
+//   kMapStHi0..kMapStB epilogue store boxes of 32 x 32, 64-byte swizzle
+enum MapIndex : int {
+  kMapHi0 = 0, kMapHi1 = 1, kMapA = 2, kMapB = 3,
+  kMapHi0S = 4, kMapHi1S = 5, kMapAS = 6, kMapBS = 7,
+  kMapStHi0 = 8, kMapStHi1 = 9, kMapStLo = 10, kMapStA = 11, kMapStB = 12,
+  kMapsPerMat = 13
+};
 constexpr int kEpiBoxCols = 32;
 
 // device status bits (sticky, cleared by muon_get_status)
@@ -150,6 +153,10 @@ cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatI
 cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which,
                                 float* out, cudaStream_t st);
 cudaError_t launch_gemm_tc(const GemmArgs& args, int npairs, cudaStream_t st);
+// Encode the kMapsPerMat TMA descriptors of one matrix (host); false if the
+// driver entry point is missing or rejects a descriptor.
+bool encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0, __nv_bfloat16* hi1, __nv_bfloat16* lo,
+                        __nv_bfloat16* A, __nv_bfloat16* B);
 int gemm_tc_max_pairs();
 cudaError_t launch_gemm_f32(const Gemm32Args& args, cudaStream_t st);
 int gemm_tc_smem_bytes();

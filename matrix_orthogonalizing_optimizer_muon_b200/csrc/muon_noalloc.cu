@@ -64,34 +64,6 @@ struct DeviceState {
 };
 DeviceState g_state[64];
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-bool encode(CUtensorMap* tm, void* base, int rows, int cols, int ld, int box_cols) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBoxOuter)};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle swz = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Once per device, with that device current: resolve the scratch array's
 // device address (in host code the symbol's name is only a host-side stand-in).
 muon_status_t setup_device(int dev) {
@@ -195,14 +167,7 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   ws.rms_part = reinterpret_cast<float*>(base + kOffRms);
   ws.status = reinterpret_cast<unsigned*>(base + kOffStatus);
   CUtensorMap tm[kMapsPerMat];
-  bool ok = encode(&tm[kMapHi0], ws.hi[0], R, C, mi.ld, kBoxInner) &&
-            encode(&tm[kMapHi1], ws.hi[1], R, C, mi.ld, kBoxInner) &&
-            encode(&tm[kMapA], ws.A, mi.m, mi.m, mi.lda, kBoxInner) &&
-            encode(&tm[kMapB], ws.B, mi.m, mi.m, mi.lda, kBoxInner) &&
-            encode(&tm[kMapEpiHi0], ws.hi[0], R, C, mi.ld, kEpiBoxCols) &&
-            encode(&tm[kMapEpiHi1], ws.hi[1], R, C, mi.ld, kEpiBoxCols) &&
-            encode(&tm[kMapEpiA], ws.A, mi.m, mi.m, mi.lda, kEpiBoxCols) &&
-            encode(&tm[kMapEpiLo], ws.lo, R, C, mi.ld, kEpiBoxCols);
+  const bool ok = encode_matrix_maps(tm, mi, ws.hi[0], ws.hi[1], ws.lo, ws.A, ws.B);
   if (!ok) return MUON_ERR_CUDA;
 
   // ---- stage descriptors (pageable host -> device copies are staged by the
