@@ -188,6 +188,11 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int
                "r"(y), "r"(src)
                : "memory");
 }
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(tmap), "r"(x),
+               "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until every committed bulk store of this thread has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -782,7 +787,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               staging_free();
               write_row32(blk0, lane, h);
               write_row32(blk1, lane, l);
-              publish(tmap_of(g, c.p, kMapStHi0 + (g.cur ^ 1)), j0, i_lo, tmap_of(g, c.p, kMapStLo), j0, i_lo);
+              // blk1 follows blk0: one 3-D store writes the hi block and the lo block
+              fence_proxy_async();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(tmap_of(g, c.p, kMapStHiLo0 + (g.cur ^ 1)), blk0_s, j0, i_lo, 0);
+                bulk_commit();
+              }
             } else if (i < mi.rows) {
               __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
               __nv_bfloat16* lout = g.ws.lo + mi.off_x;

@@ -65,10 +65,26 @@ bool encode_bf16_2d(CUtensorMap* tm, void* base, int rows, int cols, int ld, int
             swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over two [rows, cols] arrays with the same pitch `ld`,
+// the second `pair_bytes` after the first: boxes {32, 32, 2} move a 32 x 32
+// block of both arrays at once; 64-byte swizzle.
+bool encode_bf16_pair(CUtensorMap* tm, void* base, int rows, int cols, int ld, long long pair_bytes) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr || pair_bytes <= 0 || pair_bytes % 16 != 0) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(pair_bytes)};
+  const cuuint32_t box[3] = {32, 32, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
-// Operand maps (64 x 128 and 64 x 64 boxes) and epilogue store maps (32 x 32)
-// of one matrix's workspace arrays, in MapIndex order.
+// Operand maps (64 x 128 and 64 x 64 boxes) and epilogue store maps (32 x 32,
+// hi and lo together) of one matrix's workspace arrays, in MapIndex order.
+// lo must lie after hi0 and hi1 in memory.
 bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0, __nv_bfloat16* hi1,
                               __nv_bfloat16* lo, __nv_bfloat16* A, __nv_bfloat16* B) {
   CUtensorMap* t = static_cast<CUtensorMap*>(maps);
@@ -81,9 +97,8 @@ bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0,
          encode_bf16_2d(t + kMapHi1S, hi1, R, C, mi.ld, kBoxInner, 64) &&
          encode_bf16_2d(t + kMapAS, A, m, m, mi.lda, kBoxInner, 64) &&
          encode_bf16_2d(t + kMapBS, B, m, m, mi.lda, kBoxInner, 64) &&
-         encode_bf16_2d(t + kMapStHi0, hi0, R, C, mi.ld, kEpiBoxCols, 32) &&
-         encode_bf16_2d(t + kMapStHi1, hi1, R, C, mi.ld, kEpiBoxCols, 32) &&
-         encode_bf16_2d(t + kMapStLo, lo, R, C, mi.ld, kEpiBoxCols, 32) &&
+         encode_bf16_pair(t + kMapStHiLo0, hi0, R, C, mi.ld, reinterpret_cast<char*>(lo) - reinterpret_cast<char*>(hi0)) &&
+         encode_bf16_pair(t + kMapStHiLo1, hi1, R, C, mi.ld, reinterpret_cast<char*>(lo) - reinterpret_cast<char*>(hi1)) &&
          encode_bf16_2d(t + kMapStA, A, m, m, mi.lda, kEpiBoxCols, 32) &&
          encode_bf16_2d(t + kMapStB, B, m, m, mi.lda, kEpiBoxCols, 32);
 }

@@ -39,15 +39,18 @@ constexpr int kChunkElems = 32768;  // elements per momentum/normalise chunk
 constexpr int kEwThreads = 256;
 constexpr int kT32 = 64;           // fp32 path tile edge
 // TMA descriptors per matrix (128 bytes each):
-//   kMapHi0..kMapB     operand boxes of 64 x 128 rows, 128-byte swizzle (K-major loads)
-//   kMapHi0S..kMapBS   operand boxes of 64 x 64 rows, 128-byte swizzle (MN-major loads,
-//                      and K-major loads of at most 64 rows)
-//   kMapStHi0..kMapStB epilogue store boxes of 32 x 32, 64-byte swizzle
+//   kMapHi0..kMapB        operand boxes of 64 x 128 rows, 128-byte swizzle (K-major loads)
+//   kMapHi0S..kMapBS      operand boxes of 64 x 64 rows, 128-byte swizzle (MN-major loads,
+//                         and K-major loads of at most 64 rows)
+//   kMapStHiLo0/1         epilogue store of a 32 x 32 block of hi[0/1] and the same block of
+//                         lo in one 3-D box {32, 32, 2} (the third dimension steps from hi to
+//                         lo), 64-byte swizzle
+//   kMapStA, kMapStB      epilogue store boxes of 32 x 32, 64-byte swizzle
 enum MapIndex : int {
   kMapHi0 = 0, kMapHi1 = 1, kMapA = 2, kMapB = 3,
   kMapHi0S = 4, kMapHi1S = 5, kMapAS = 6, kMapBS = 7,
-  kMapStHi0 = 8, kMapStHi1 = 9, kMapStLo = 10, kMapStA = 11, kMapStB = 12,
-  kMapsPerMat = 13
+  kMapStHiLo0 = 8, kMapStHiLo1 = 9, kMapStA = 10, kMapStB = 11,
+  kMapsPerMat = 12
 };
 constexpr int kEpiBoxCols = 32;
 
