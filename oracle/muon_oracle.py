@@ -26,7 +26,9 @@ are taken:
   (no epsilon anywhere), so the step reduces to pure weight decay.
 * Update scale: 0.2 * sqrt(max(A, B)) with [A, B] the parameter's shape
   (Sec. 2.2, Eq. 4, the "Adjusted LR" rule of Sec. 3.1, Eq. 7); the decay term
-  reads W_{t-1} (decoupled, Eq. 3).
+  reads W_{t-1} (decoupled, Eq. 3).  The two alternatives Sec. 3.1 compares
+  are also provided: 0.2 * sqrt(H) (Eq. 5) and 0.2 / RMS(O) (Eq. 6), the
+  latter 0 for O = 0.
 * Update RMS: sqrt(mean(u^2)) of the orthogonalised update u, the quantity
   Algorithm 1 ("Distributed Muon", Sec. 2.3) returns for logging.
 """
@@ -46,6 +48,11 @@ DEFAULT_NS_STEPS = 5
 DEFAULT_MOMENTUM = 0.95
 # Sec. 2.2, Eq. 4: the update RMS is matched to AdamW's at 0.2.
 DEFAULT_RMS_SCALE = 0.2
+
+# Ways of scaling the orthogonalised update (Sec. 3.1, "Consistent update RMS")
+SCALE_MAX_DIM = 0      # 0.2 * sqrt(max(A, B))          Eq. 4 = Eq. 7 ("Adjusted LR"), the method's rule
+SCALE_HIDDEN = 1       # 0.2 * sqrt(H), H hidden size    Eq. 5 ("Baseline")
+SCALE_UPDATE_NORM = 2  # 0.2 / RMS(O)                    Eq. 6 ("Update Norm")
 
 
 def _f64(x) -> np.ndarray:
@@ -121,6 +128,22 @@ def update_scale(rows: int, cols: int, rms_scale: float = DEFAULT_RMS_SCALE) -> 
     return float(rms_scale) * math.sqrt(float(max(rows, cols)))
 
 
+def update_scale_hidden(hidden_dim: float, rms_scale: float = DEFAULT_RMS_SCALE) -> float:
+    """0.2 * sqrt(H) with H the model's hidden dimension, the same for every
+    matrix (Sec. 3.1, Eq. 5, "Baseline")."""
+    if not hidden_dim > 0:
+        raise ValueError("Eq. 5 needs the hidden dimension H > 0")
+    return float(rms_scale) * math.sqrt(float(hidden_dim))
+
+
+def update_norm_scale(O, rms_scale: float = DEFAULT_RMS_SCALE) -> float:
+    """Factor that makes the update's RMS exactly 0.2: 0.2 / RMS(O) (Sec. 3.1,
+    Eq. 6, "Update Norm").  Reading: for O = 0 (zero input) the factor is 0,
+    so the step stays pure weight decay as in the other rules."""
+    r = update_rms(O)
+    return 0.0 if r == 0.0 else float(rms_scale) / r
+
+
 def apply_update(W, O, lr: float, weight_decay: float, scale: float) -> np.ndarray:
     """W_t = W_{t-1} - eta_t (scale * O_t + lambda W_{t-1})  (Sec. 2.2, Eq. 4;
     with scale = 1 this is Eq. 3)."""
@@ -147,14 +170,17 @@ class StepResult:
 
 def muon_step(W, G, M_prev, *, lr: float, weight_decay: float, momentum_coef: float = DEFAULT_MOMENTUM,
               ns_steps: int = DEFAULT_NS_STEPS, coeffs=DEFAULT_COEFFS,
-              rms_scale: float = DEFAULT_RMS_SCALE, nesterov: bool = True) -> StepResult:
+              rms_scale: float = DEFAULT_RMS_SCALE, nesterov: bool = True,
+              scale_mode: int = SCALE_MAX_DIM, hidden_dim: float = 0.0) -> StepResult:
     """One Muon step for one matrix parameter (Sec. 2.1 Eq. 1 with the
     Nesterov input, Eq. 2, and the Sec. 2.2 Eq. 4 update).
 
     1. M_t = mu M_{t-1} + G_t
     2. Y   = mu M_t + G_t   (or Y = M_t without Nesterov, plain Eq. 1)
     3. O_t = Newton-Schulz(Y)
-    4. W_t = W_{t-1} - eta (rms_scale sqrt(max(A,B)) O_t + lambda W_{t-1})
+    4. W_t = W_{t-1} - eta (scale O_t + lambda W_{t-1}), with scale
+       rms_scale sqrt(max(A,B)) (Eq. 4), rms_scale sqrt(H) (Sec. 3.1 Eq. 5)
+       or rms_scale / RMS(O_t) (Sec. 3.1 Eq. 6) by `scale_mode`.
     """
     W = _f64(W)
     if W.ndim != 2:
@@ -162,7 +188,14 @@ def muon_step(W, G, M_prev, *, lr: float, weight_decay: float, momentum_coef: fl
     M_t = momentum(M_prev, G, momentum_coef)
     Y = nesterov_input(M_t, G, momentum_coef) if nesterov else M_t
     O = newton_schulz(Y, ns_steps, coeffs)
-    scale = update_scale(W.shape[0], W.shape[1], rms_scale)
+    if scale_mode == SCALE_MAX_DIM:
+        scale = update_scale(W.shape[0], W.shape[1], rms_scale)
+    elif scale_mode == SCALE_HIDDEN:
+        scale = update_scale_hidden(hidden_dim, rms_scale)
+    elif scale_mode == SCALE_UPDATE_NORM:
+        scale = update_norm_scale(O, rms_scale)
+    else:
+        raise ValueError(f"unknown scale_mode {scale_mode}")
     W_t = apply_update(W, O, lr, weight_decay, scale)
     return StepResult(W=W_t, M=M_t, O=O, rms=update_rms(O), Y=Y)
 

@@ -259,6 +259,63 @@ def test_full_step_against_svd_route(shape):
         assert abs(outs[t].rms - math.sqrt(np.mean(O * O))) < 1e-13
 
 
+# ------------------------------------------------------------------ update-scale alternatives (Sec. 3.1)
+
+def _one_step(shape, seed, **hp):
+    W0 = rand(shape, seed)
+    G = rand(shape, seed + 1)
+    return W0, orc.muon_step(W0, G, np.zeros(shape), **hp)
+
+
+def _update_part(W0, r, lr, wd):
+    """u with W_t = W_{t-1} - lr (u + wd W_{t-1})."""
+    return (W0 * (1 - lr * wd) - r.W) / lr
+
+
+def test_hidden_dim_scale_matches_eq4_on_square_and_printed_ratio():
+    # Sec. 3.1: for most matrices max(A, B) = H, so Eq. 5 and Eq. 4 agree on
+    # [H, H]; for [H, 4H] the Eq. 4 update is twice the Eq. 5 one (finding 2)
+    lr, wd = 0.1, 0.1
+    H = 24
+    W0, r4 = _one_step((H, H), 7, lr=lr, weight_decay=wd, scale_mode=orc.SCALE_MAX_DIM)
+    _, r5 = _one_step((H, H), 7, lr=lr, weight_decay=wd, scale_mode=orc.SCALE_HIDDEN, hidden_dim=H)
+    assert np.max(np.abs(r4.W - r5.W)) < 1e-15
+    g = json.load(open(GOLDEN))["mlp_vs_attention_update_ratio"]
+    shape = (H, 4 * H)
+    W0, r4 = _one_step(shape, 8, lr=lr, weight_decay=wd, scale_mode=orc.SCALE_MAX_DIM)
+    _, r5 = _one_step(shape, 8, lr=lr, weight_decay=wd, scale_mode=orc.SCALE_HIDDEN, hidden_dim=H)
+    u4, u5 = _update_part(W0, r4, lr, wd), _update_part(W0, r5, lr, wd)
+    assert abs(np.linalg.norm(u4) / np.linalg.norm(u5) - g["value"]) < 1e-12
+
+
+@pytest.mark.parametrize("shape", [(6, 17), (17, 6), (9, 9)])
+def test_update_norm_makes_update_rms_exactly_rms_scale(shape):
+    lr, wd = 0.05, 0.1
+    W0, r = _one_step(shape, 11, lr=lr, weight_decay=wd, scale_mode=orc.SCALE_UPDATE_NORM)
+    u = _update_part(W0, r, lr, wd)
+    assert abs(math.sqrt(np.mean(u * u)) - 0.2) < 1e-12
+    # the logged RMS stays that of O itself
+    assert abs(r.rms - math.sqrt(np.mean(r.O * r.O))) < 1e-15
+
+
+@pytest.mark.parametrize("shape", [(16, 64), (64, 16)])
+def test_update_norm_equals_eq4_for_exact_polar_factor(shape):
+    # Lemma 1: a full-rank polar factor has RMS 1/sqrt(max(A, B)), so Eq. 6
+    # and Eq. 4 give the same step; the cubic iteration (1.5, -0.5, 0) run
+    # long reaches the polar factor
+    hp = dict(lr=0.1, weight_decay=0.1, ns_steps=60, coeffs=(1.5, -0.5, 0.0))
+    _, r4 = _one_step(shape, 21, scale_mode=orc.SCALE_MAX_DIM, **hp)
+    _, r6 = _one_step(shape, 21, scale_mode=orc.SCALE_UPDATE_NORM, **hp)
+    assert np.max(np.abs(r4.W - r6.W)) < 1e-10
+
+
+def test_update_norm_zero_gradient_is_pure_decay():
+    W0 = rand((5, 7), 31)
+    r = orc.muon_step(W0, np.zeros((5, 7)), np.zeros((5, 7)), lr=0.01, weight_decay=0.1,
+                      scale_mode=orc.SCALE_UPDATE_NORM)
+    assert np.max(np.abs(r.W - (1 - 0.01 * 0.1) * W0)) < 1e-16
+
+
 # ------------------------------------------------------------------ planted mistakes
 
 def _pins_hold() -> bool:
@@ -274,6 +331,10 @@ def _pins_hold() -> bool:
         test_full_step_against_svd_route((12, 20))
         test_full_step_against_svd_route((20, 12))
         test_zero_gradient_is_pure_decoupled_weight_decay()
+        test_hidden_dim_scale_matches_eq4_on_square_and_printed_ratio()
+        test_update_norm_makes_update_rms_exactly_rms_scale((6, 17))
+        test_update_norm_equals_eq4_for_exact_polar_factor((16, 64))
+        test_update_norm_zero_gradient_is_pure_decay()
     except Exception:
         return False
     return True
@@ -290,6 +351,10 @@ MUTATIONS = {
     "no_nesterov": ("nesterov_input", lambda M, G, mu: np.asarray(M, float)),
     "damped_momentum": ("momentum", lambda M, G, mu: mu * np.asarray(M, float) + (1 - mu) * np.asarray(G, float)),
     "scale_uses_min": ("update_scale", lambda r, c, s=0.2: s * math.sqrt(min(r, c))),
+    "hidden_scale_without_sqrt": ("update_scale_hidden", lambda H, s=0.2: s * float(H)),
+    "update_norm_by_mean_abs": ("update_norm_scale",
+                                lambda O, s=0.2: s / float(np.mean(np.abs(O))) if np.any(O) else 0.0),
+    "update_norm_inverted": ("update_norm_scale", lambda O, s=0.2: s * orc.update_rms(O)),
     "decay_after_update": ("apply_update",
                            lambda W, O, lr, weight_decay, scale: (np.asarray(W, float) - lr * scale * O) * (1 - lr * weight_decay)),
 }
