@@ -179,6 +179,45 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def blas_vendor() -> str:
+    try:
+        from threadpoolctl import threadpool_info
+        import numpy  # noqa: F401  (loads its BLAS so threadpoolctl can see it)
+        info = [d for d in threadpool_info() if d.get("user_api") == "blas"]
+        return ", ".join(sorted({f"{d.get('internal_api')} {d.get('version') or ''}".strip() for d in info})) or "unknown"
+    except Exception:
+        return "unknown"
+
+
+def torch_eager_ns_ms(Gs, zero, steps: int, abc, reps: int = 3) -> float:
+    """Same-box context point, not part of the product: the quintic iteration
+    written with torch.mm in bf16 (library GEMMs, no symmetry, one matrix at a
+    time) over the same gradients, wide orientation.  Returns ms per pass."""
+    import torch
+    a, b, c = abc
+
+    def one(G):
+        X = G.t() if G.shape[0] > G.shape[1] else G
+        X = (X.float() / X.float().norm()).to(torch.bfloat16)
+        for _ in range(steps):
+            A = X @ X.t()
+            B = b * A + c * (A @ A)
+            X = a * X + B @ X
+        return X
+
+    mats = [G for i, G in enumerate(Gs) if i not in zero]
+    one(mats[0])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        for G in mats:
+            one(G)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def run_reference(args, wl, rank: int):
     if rank != 0:
         return
@@ -197,7 +236,8 @@ def run_reference(args, wl, rank: int):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(wl),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                             "host_cpus": os.cpu_count(), "blas": blas_vendor()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -221,6 +261,9 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="moe")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-context", action="store_true", help="skip the PyTorch eager comparison point")
+    ap.add_argument("--scale", default="max_dim", choices=["max_dim", "hidden", "update_norm"],
+                    help="update scale of Sec. 3.1: Eq. 4 (default), Eq. 5 with H = 2048, Eq. 6")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--limit", type=int, default=0, help="keep only the first N matrices (small profiling case)")
     args = ap.parse_args(argv)
@@ -271,7 +314,7 @@ def main(argv=None) -> int:
     params = list(zip(Ws, Gs, Ms))
     plan.bind(params)
     rms = torch.zeros(wl.n, device=dev)
-    hp = dict(lr=4.2e-4, weight_decay=0.1, momentum=0.95, ns_steps=5)
+    hp = dict(lr=4.2e-4, weight_decay=0.1, momentum=0.95, ns_steps=5, scale=args.scale, hidden_dim=2048.0)
     nz_flops = sum(ns_flops(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
     dense_flops = sum(ns_flops_dense(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
 
@@ -351,16 +394,35 @@ def main(argv=None) -> int:
     k1_gbs = total * K1_BYTES_PER_ELEM / (k1_ms * 1e-3) / 1e9
     traffic = ncu_traffic(gemm_launches)
 
+    context = None
+    if not args.no_context:
+        t_eager = torch_eager_ns_ms(Gs, wl.zero_grad, 5, (3.4445, -4.7750, 2.0315))
+        context = {"what": "PyTorch eager Newton-Schulz (torch.mm bf16, one matrix at a time, no symmetry), "
+                           "same gradients; context only",
+                   "ns_ms_per_step": t_eager, "tflops_algorithmic": nz_flops / (t_eager * 1e-3) / 1e12,
+                   "tflops_dense_equivalent": dense_flops / (t_eager * 1e-3) / 1e12}
+
     cpu = None
     if world == 1 and args.cpu_budget > 0:
         f, s, d = cpu_sample(wl, args.cpu_budget)
         cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{d} whole-matrix fp64 oracle steps of the workload ({s:.1f} s), same FLOP count"}
+               "sample": f"{d} whole-matrix fp64 oracle steps of the workload ({s:.1f} s), same FLOP count",
+               "host_cpus": os.cpu_count(), "blas": blas_vendor()}
 
+    config = workload_config(wl)
+    config["update_scale"] = {"max_dim": "Eq. 4: 0.2 sqrt(max(A,B))", "hidden": "Eq. 5: 0.2 sqrt(H), H = 2048",
+                              "update_norm": "Eq. 6: 0.2 / RMS(O)"}[args.scale]
+    if args.scale == "update_norm":
+        fin_ms = prof["ms"]["finalize"] / calls
+        config["update_norm_passes"] = {
+            "kernels": "update_norm_kernel (RMS(O): reads hi+lo, 4 B/elem) + apply_update_kernel "
+                       "(hi+lo 4 + W 8 B/elem)", "ms_per_step": fin_ms,
+            "gbs": total * 16 / (fin_ms * 1e-3) / 1e9,
+            "frac_of_hbm": total * 16 / (fin_ms * 1e-3) / 1e9 / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(wl),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
         "ns_ms_per_step": gemm_ms, "ns_tflops": achieved,
         "ns_pct_of_bf16_peak": 100.0 * achieved / peak,
         "ns_tflops_dense_equivalent": dense_flops / (gemm_ms * 1e-3) / 1e12,
@@ -374,6 +436,7 @@ def main(argv=None) -> int:
                         "unit": "GB/s", "frac": k1_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
                         "bytes_per_elem": K1_BYTES_PER_ELEM},
         "cpu_baseline": cpu,
+        "context_torch_eager_ns": context,
         "e2e": e2e,
         "gpu_launches": int(round(per_step_launches * args.steps)),
         "clocks": clk.summary(),

@@ -62,6 +62,17 @@ typedef enum { MUON_DT_BF16 = 0, MUON_DT_FP32 = 1 } muon_dtype_t;
  *                 validation path, needs MUON_INIT_FP32_NS at plan creation. */
 typedef enum { MUON_NS_BF16 = 0, MUON_NS_FP32 = 1 } muon_ns_precision_t;
 
+/* How the orthogonalised update O is scaled before it is applied ("Muon is
+ * Scalable for LLM Training", Sec. 3.1, "Consistent update RMS", which
+ * compares the three rules; the method itself uses the first).
+ *   MUON_SCALE_MAX_DIM     rms_scale * sqrt(max(rows, cols))   Eq. 4 (= Eq. 7), the default
+ *   MUON_SCALE_HIDDEN      rms_scale * sqrt(hidden_dim)        Eq. 5, "Baseline": one H for all
+ *   MUON_SCALE_UPDATE_NORM rms_scale / RMS(O), 0 when O = 0    Eq. 6, "Update Norm": every
+ *                          matrix's update has RMS exactly rms_scale.  Needs RMS(O) before any
+ *                          weight changes, so the step adds a reduction pass and an apply pass
+ *                          over the iterate instead of the update fused into the last product. */
+typedef enum { MUON_SCALE_MAX_DIM = 0, MUON_SCALE_HIDDEN = 1, MUON_SCALE_UPDATE_NORM = 2 } muon_scale_mode_t;
+
 /* muon_init flags */
 #define MUON_INIT_ZERO_MOMENTUM 0x1u /* zero every M on `stream` (M_0 = 0, Sec. 2.1) */
 #define MUON_INIT_FP32_NS       0x2u /* also reserve the workspace of the fp32 path */
@@ -89,6 +100,8 @@ typedef struct {
   float   rms_scale;     /* the 0.2 of Eq. 4                                                   */
   int32_t nesterov;      /* 1: Newton-Schulz input mu M_t + G_t; 0: M_t (plain Eq. 1)          */
   int32_t ns_precision;  /* muon_ns_precision_t                                                */
+  int32_t scale_mode;    /* muon_scale_mode_t                                                  */
+  float   hidden_dim;    /* H of Eq. 5 (> 0 with MUON_SCALE_HIDDEN, ignored otherwise)          */
 } muon_hparams_t;
 
 typedef struct muon_plan_s* muon_plan_t;
@@ -96,7 +109,7 @@ typedef struct muon_plan_s* muon_plan_t;
 /* Fill `hp` with the pages' values: lr 4.2e-4 (Sec. 3.3 peak), weight_decay 0.1
  * (Sec. 3.3), momentum 0.95, ns_steps 5 (Sec. 2.2), (a, b, c) =
  * (3.4445, -4.7750, 2.0315) (Sec. 2.1), rms_scale 0.2 (Eq. 4), nesterov 1,
- * ns_precision MUON_NS_BF16.  Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
+ * ns_precision MUON_NS_BF16, scale_mode MUON_SCALE_MAX_DIM, hidden_dim 0.  Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
 MUON_API muon_status_t muon_hparams_default(muon_hparams_t* hp);
 
 /* Build a plan for `n` matrices with the shapes in params[0..n).  The plan

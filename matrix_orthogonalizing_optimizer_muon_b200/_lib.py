@@ -29,6 +29,7 @@ MUON_NS_BF16 = 0
 MUON_NS_FP32 = 1
 MUON_INIT_ZERO_MOMENTUM = 0x1
 MUON_INIT_FP32_NS = 0x2
+MUON_SCALE_MAX_DIM, MUON_SCALE_HIDDEN, MUON_SCALE_UPDATE_NORM = 0, 1, 2
 MUON_NUM_PHASES = 5
 PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
 
@@ -47,7 +48,7 @@ class muon_hparams_t(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("weight_decay", ctypes.c_float), ("momentum", ctypes.c_float),
                 ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float), ("b", ctypes.c_float),
                 ("c", ctypes.c_float), ("rms_scale", ctypes.c_float), ("nesterov", ctypes.c_int32),
-                ("ns_precision", ctypes.c_int32)]
+                ("ns_precision", ctypes.c_int32), ("scale_mode", ctypes.c_int32), ("hidden_dim", ctypes.c_float)]
 
 
 class MuonError(RuntimeError):

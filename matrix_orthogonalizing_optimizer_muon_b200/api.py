@@ -88,15 +88,25 @@ class MuonPlan:
 
     def step(self, params=None, *, lr: float, weight_decay: float, momentum: float = 0.95, ns_steps: int = 5,
              coeffs=DEFAULT_COEFFS, rms_scale: float = 0.2, nesterov: bool = True, precision: str = "bf16",
-             update_rms: torch.Tensor | None = None, stream=None) -> None:
-        """One Muon step over every matrix (in place on W and M)."""
+             update_rms: torch.Tensor | None = None, scale: str = "max_dim", hidden_dim: float = 0.0,
+             stream=None) -> None:
+        """One Muon step over every matrix (in place on W and M).
+
+        `scale` picks how O is scaled (Sec. 3.1): "max_dim" rms_scale sqrt(max(A, B))
+        (Eq. 4), "hidden" rms_scale sqrt(hidden_dim) (Eq. 5) or "update_norm"
+        rms_scale / RMS(O) (Eq. 6)."""
+        modes = {"max_dim": L.MUON_SCALE_MAX_DIM, "hidden": L.MUON_SCALE_HIDDEN,
+                 "update_norm": L.MUON_SCALE_UPDATE_NORM}
+        if scale not in modes:
+            raise ValueError(f"scale must be one of {sorted(modes)}")
         if params is not None:
             self.bind(params)
         elif self._key is None:
             raise ValueError("no parameters bound")
         hp = L.muon_hparams_t(lr, weight_decay, momentum, int(ns_steps), coeffs[0], coeffs[1], coeffs[2],
                               rms_scale, 1 if nesterov else 0,
-                              L.MUON_NS_FP32 if precision == "fp32" else L.MUON_NS_BF16)
+                              L.MUON_NS_FP32 if precision == "fp32" else L.MUON_NS_BF16, modes[scale],
+                              float(hidden_dim))
         rms_ptr = None
         if update_rms is not None:
             _check_tensor(update_rms, torch.float32, "update_rms", (self.n,))

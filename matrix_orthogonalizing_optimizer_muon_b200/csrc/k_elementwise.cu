@@ -10,9 +10,15 @@
 //     counter) reduces the chunk partials in chunk order and writes
 //     s = 1 / ||Y||_F (0 for an all-zero Y, NaN plus a status bit if the sum
 //     is not finite).
-// apply_update: W <- W - lr (rms_scale sqrt(n) O + wd W) with O = s X, used
-//     when there are no Newton-Schulz iterations (N = 0); the N > 0 path fuses
-//     this update into the last GEMM epilogue (Sec. 2.2, Eq. 4).
+// apply_update: W <- W - lr (scale O + wd W) (Sec. 2.2, Eq. 4; Sec. 3.1,
+//     Eq. 5/6 for the other scales), or O itself, from the iterate the last
+//     X update left in workspace, with O = s X when there are no
+//     Newton-Schulz iterations (N = 0).  A separate, fully coalesced pass: a
+//     fused row-per-thread fp32 read-modify-write in the last GEMM epilogue
+//     measured about twice as slow as this pass plus the extra iterate write.
+// update_norm: RMS(O) per matrix and the Eq. 6 factor rms_scale / RMS(O)
+//     (Sec. 3.1, "Update Norm"), chunk partials in fp64 reduced in chunk
+//     order by the last CTA of each matrix.
 // rms_finalize: sqrt(mean(O^2)) per matrix from per-tile partial sums
 //     (Sec. 2.3, Algorithm 1, returned value).
 #include "muon_internal.cuh"
@@ -172,49 +178,191 @@ __global__ void __launch_bounds__(kEwThreads) k1_kernel(const ChunkDesc* __restr
   }
 }
 
+// The iterate X in workspace: fp32 x32 on the fp32 path, else the bf16 pair hi + lo.
+struct XView {
+  const float* x32;
+  const __nv_bfloat16* hi;
+  const __nv_bfloat16* lo;
+};
+
+__device__ __forceinline__ XView x_view(const Workspace& ws, int fp32_path, int xbuf) {
+  // selects, not an indexed load: a runtime index into a kernel-parameter
+  // array would copy the whole struct to local memory
+  return fp32_path ? XView{xbuf ? ws.x32[1] : ws.x32[0], nullptr, nullptr}
+                   : XView{nullptr, xbuf ? ws.hi[1] : ws.hi[0], ws.lo};
+}
+
+// Eight consecutive values of X at workspace index wi (16-byte aligned).
+__device__ __forceinline__ void load_x8(XView xv, size_t wi, float* x) {
+  if (xv.x32 != nullptr) {
+    const float4* q = reinterpret_cast<const float4*>(xv.x32 + wi);
+    const float4 u = q[0], v = q[1];
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+  } else {
+    const uint4 h = *reinterpret_cast<const uint4*>(xv.hi + wi);
+    const uint4 l = *reinterpret_cast<const uint4*>(xv.lo + wi);
+    const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&h);
+    const __nv_bfloat162* ll = reinterpret_cast<const __nv_bfloat162*>(&l);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fh = __bfloat1622float2(hh[i]), fl = __bfloat1622float2(ll[i]);
+      x[2 * i] = fh.x + fl.x;
+      x[2 * i + 1] = fh.y + fl.y;
+    }
+  }
+}
+
+__device__ __forceinline__ float load_x1(XView xv, size_t wi) {
+  return xv.x32 != nullptr ? xv.x32[wi] : __bfloat162float(xv.hi[wi]) + __bfloat162float(xv.lo[wi]);
+}
+
 __global__ void __launch_bounds__(kEwThreads) apply_update_kernel(const ChunkDesc* __restrict__ chunks,
                                                                   const MatInfo* __restrict__ mats,
                                                                   const MatPtrs* __restrict__ ptrs, Workspace ws,
-                                                                  StepScalars sc, int final_mode, int fp32_path) {
+                                                                  StepScalars sc, int final_mode, int fp32_path,
+                                                                  int xbuf, int mul_s) {
   __shared__ float red[kEwThreads / 32];
   const ChunkDesc ch = chunks[blockIdx.x];
   const int p = ch.x;
   const MatInfo mi = mats[p];
   const MatPtrs pt = ptrs[p];
   const int C = mi.cols, r0 = ch.y, nr = ch.z;
-  const float s = ws.s[p];
-  const float scale = sc.rms_scale * sqrtf((float)mi.n);
+  // s == 0 marks Y == 0: O = 0, and the Newton-Schulz launches skipped this
+  // matrix, so its iterate buffer holds nothing of this step
+  const float sp = ws.s[p];
+  const bool zero = (sp == 0.0f);
+  const float s = zero ? 0.0f : (mul_s ? sp : 1.0f);
+  const float scale = zero ? 0.0f : (sc.scale_mode == kScaleUpdateNorm ? ws.unorm[p] : update_scale_of(sc, mi.n));
+  const bool weight = (final_mode == kFinalWeight);
+  const XView xv = x_view(ws, fp32_path, xbuf);
   float acc = 0.0f;
   const int64_t total = (int64_t)nr * C;
-  for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
-    const int rr = (int)(e / C);
-    const int c = (int)(e - (int64_t)rr * C);
-    const int r = r0 + rr;
-    const size_t gi = (size_t)r * C + c;
-    const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c;
-    const float x = fp32_path ? ws.x32[0][wi] : __bfloat162float(ws.hi[0][wi]) + __bfloat162float(ws.lo[wi]);
-    const float o = s * x;
-    acc = fmaf(o, o, acc);
-    if (final_mode == kFinalWeight) {
-      const float w = pt.W[gi];
-      pt.W[gi] = w - sc.lr * fmaf(scale, o, sc.wd * w);
-    } else {
-      pt.W[gi] = o;
+  if (pt.vec_ok) {
+    for (int64_t e = (int64_t)threadIdx.x * 8; e < total; e += (int64_t)blockDim.x * 8) {
+      const int rr = (int)(e / C);
+      const int c = (int)(e - (int64_t)rr * C);
+      const int r = r0 + rr;
+      const size_t gi = (size_t)r * C + c;
+      const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c;
+      float o[8] = {};
+      if (!zero) load_x8(xv, wi, o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i] *= s;
+        acc = fmaf(o[i], o[i], acc);
+      }
+      float4* w4 = reinterpret_cast<float4*>(pt.W + gi);
+      float4 wa = w4[0], wb = w4[1];
+      if (weight) {
+        wa.x = wa.x - sc.lr * fmaf(scale, o[0], sc.wd * wa.x);
+        wa.y = wa.y - sc.lr * fmaf(scale, o[1], sc.wd * wa.y);
+        wa.z = wa.z - sc.lr * fmaf(scale, o[2], sc.wd * wa.z);
+        wa.w = wa.w - sc.lr * fmaf(scale, o[3], sc.wd * wa.w);
+        wb.x = wb.x - sc.lr * fmaf(scale, o[4], sc.wd * wb.x);
+        wb.y = wb.y - sc.lr * fmaf(scale, o[5], sc.wd * wb.y);
+        wb.z = wb.z - sc.lr * fmaf(scale, o[6], sc.wd * wb.z);
+        wb.w = wb.w - sc.lr * fmaf(scale, o[7], sc.wd * wb.w);
+      } else {
+        wa = make_float4(o[0], o[1], o[2], o[3]);
+        wb = make_float4(o[4], o[5], o[6], o[7]);
+      }
+      w4[0] = wa;
+      w4[1] = wb;
+    }
+  } else {
+    for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+      const int rr = (int)(e / C);
+      const int c = (int)(e - (int64_t)rr * C);
+      const int r = r0 + rr;
+      const size_t gi = (size_t)r * C + c;
+      const size_t wi = (size_t)mi.off_x + (size_t)r * mi.ld + c;
+      const float o = zero ? 0.0f : s * load_x1(xv, wi);
+      acc = fmaf(o, o, acc);
+      if (weight) {
+        const float w = pt.W[gi];
+        pt.W[gi] = w - sc.lr * fmaf(scale, o, sc.wd * w);
+      } else {
+        pt.W[gi] = o;
+      }
     }
   }
   const float part = block_sum(acc, red);
   if (threadIdx.x == 0) ws.rms_part[ch.w] = part;
 }
 
+__global__ void __launch_bounds__(kEwThreads) update_norm_kernel(const ChunkDesc* __restrict__ chunks,
+                                                                 const MatInfo* __restrict__ mats, Workspace ws,
+                                                                 StepScalars sc, int fp32_path, int xbuf, int mul_s,
+                                                                 float* __restrict__ update_rms) {
+  __shared__ double red[kEwThreads / 32];
+  __shared__ bool am_last;
+  const ChunkDesc ch = chunks[blockIdx.x];
+  const int p = ch.x;
+  const MatInfo mi = mats[p];
+  const int C = mi.cols, r0 = ch.y, nr = ch.z;
+  const float sp = ws.s[p];
+  const float s = mul_s ? sp : 1.0f;
+  const XView xv = x_view(ws, fp32_path, xbuf);
+  double acc = 0.0;
+  const int64_t total = (int64_t)nr * C;
+  if (sp == 0.0f) {
+    // Y == 0: O = 0 (the iterate buffer was not written this step)
+  } else if (C % 8 == 0) {
+    for (int64_t e = (int64_t)threadIdx.x * 8; e < total; e += (int64_t)blockDim.x * 8) {
+      const int rr = (int)(e / C);
+      const int c = (int)(e - (int64_t)rr * C);
+      float o[8];
+      load_x8(xv, (size_t)mi.off_x + (size_t)(r0 + rr) * mi.ld + c, o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float v = s * o[i];
+        acc = fma((double)v, (double)v, acc);
+      }
+    }
+  } else {
+    for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+      const int rr = (int)(e / C);
+      const int c = (int)(e - (int64_t)rr * C);
+      const float v = s * load_x1(xv, (size_t)mi.off_x + (size_t)(r0 + rr) * mi.ld + c);
+      acc = fma((double)v, (double)v, acc);
+    }
+  }
+  const double part = block_sum(acc, red);
+  if (threadIdx.x == 0) {
+    ws.norm_part[ch.w] = part;
+    __threadfence();
+    const unsigned prev = atomicAdd(ws.norm_count + p, 1u);
+    am_last = (prev == (unsigned)(mi.nchunks - 1));
+  }
+  __syncthreads();
+  if (!am_last) return;
+  __threadfence();
+  double t = 0.0;
+  for (int i = threadIdx.x; i < mi.nchunks; i += blockDim.x) t += __ldcg(ws.norm_part + mi.chunk_base + i);
+  const double sum = block_sum(t, red);
+  if (threadIdx.x == 0) {
+    const double rms = sqrt(sum / ((double)mi.rows * (double)mi.cols));
+    float f;
+    if (!isfinite(rms)) {
+      f = __int_as_float(0x7fc00000);
+      atomicOr(ws.status, kStatusNonFinite);
+    } else {
+      f = rms > 0.0 ? (float)((double)sc.rms_scale / rms) : 0.0f;
+    }
+    ws.unorm[p] = f;
+    if (update_rms != nullptr) update_rms[p] = (float)rms;
+    ws.norm_count[p] = 0u;
+  }
+}
+
 __global__ void __launch_bounds__(kEwThreads) rms_finalize_kernel(const MatInfo* __restrict__ mats,
-                                                                  const float* __restrict__ part, int which,
+                                                                  const float* __restrict__ part,
                                                                   float* __restrict__ out) {
   __shared__ double red[kEwThreads / 32];
   const MatInfo mi = mats[blockIdx.x];
-  const int base = which == 1 ? mi.rms_tile_base : which == 2 ? mi.rms32_base : mi.chunk_base;
-  const int count = which == 1 ? mi.rms_tile_count : which == 2 ? mi.rms32_count : mi.nchunks;
   double t = 0.0;
-  for (int i = threadIdx.x; i < count; i += blockDim.x) t += (double)part[base + i];
+  for (int i = threadIdx.x; i < mi.nchunks; i += blockDim.x) t += (double)part[mi.chunk_base + i];
   const double sum = block_sum(t, red);
   if (threadIdx.x == 0) out[blockIdx.x] = (float)sqrt(sum / ((double)mi.rows * (double)mi.cols));
 }
@@ -228,14 +376,22 @@ cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats,
 }
 
 cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
-                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, cudaStream_t st) {
-  apply_update_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, final_mode, fp32_path);
+                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, int xbuf, int mul_s,
+                                cudaStream_t st) {
+  apply_update_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, final_mode, fp32_path, xbuf,
+                                                      mul_s);
   return cudaGetLastError();
 }
 
-cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which, float* out,
-                                cudaStream_t st) {
-  rms_finalize_kernel<<<nmat, kEwThreads, 0, st>>>(mats, part, which, out);
+cudaError_t launch_update_norm(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, Workspace ws,
+                               StepScalars sc, int fp32_path, int xbuf, int mul_s, float* update_rms,
+                               cudaStream_t st) {
+  update_norm_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ws, sc, fp32_path, xbuf, mul_s, update_rms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, float* out, cudaStream_t st) {
+  rms_finalize_kernel<<<nmat, kEwThreads, 0, st>>>(mats, part, out);
   return cudaGetLastError();
 }
 

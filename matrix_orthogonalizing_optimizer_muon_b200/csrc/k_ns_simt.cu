@@ -29,12 +29,10 @@ __device__ __forceinline__ float fetch(const Src& s, int i, int k, int K) {
 __global__ void __launch_bounds__(256) ns_gemm_f32_kernel(const __grid_constant__ Gemm32Args g) {
   __shared__ float As[kKS][kT32 + 4];
   __shared__ float Bs[kKS][kT32 + 4];
-  __shared__ float red[8];
   const TileDesc td = g.tiles[blockIdx.x];
   const int p = td.x, row0 = td.y, col0 = td.z;
   const MatInfo mi = g.mats[p];
   const float s = g.ws.s[p];
-  const int final_tile = (g.phase == kPhaseUpdate && g.final_mode != kFinalNone);
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
 
   const float* xcur = g.ws.x32[g.cur] + mi.off_x;
@@ -93,11 +91,10 @@ __global__ void __launch_bounds__(256) ns_gemm_f32_kernel(const __grid_constant_
       }
       __syncthreads();
     }
-  } else if (!final_tile) {
-    return;  // Y == 0: nothing downstream reads this matrix
+  } else {
+    return;  // Y == 0: nothing downstream reads this matrix (the update pass treats it as O = 0)
   }
 
-  float rms = 0.0f;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int i = row0 + ty * 4 + u;
@@ -115,33 +112,8 @@ __global__ void __launch_bounds__(256) ns_gemm_f32_kernel(const __grid_constant_
       } else {
         const size_t o = static_cast<size_t>(i) * mi.ld + j;
         const float alpha = g.iter == 0 ? s : 1.0f;
-        const float x = (s != 0.0f) ? alpha * fmaf(g.sc.a, xcur[o], r) : 0.0f;
-        if (!final_tile) {
-          g.ws.x32[g.cur ^ 1][mi.off_x + o] = x;
-        } else {
-          const MatPtrs pt = g.ptrs[p];
-          float* w = pt.W + static_cast<size_t>(i) * mi.cols + j;
-          rms = fmaf(x, x, rms);
-          if (g.final_mode == kFinalWeight) {
-            const float scale = g.sc.rms_scale * sqrtf(static_cast<float>(mi.n));
-            *w = *w - g.sc.lr * fmaf(scale, x, g.sc.wd * *w);
-          } else {
-            *w = x;
-          }
-        }
+        g.ws.x32[g.cur ^ 1][mi.off_x + o] = alpha * fmaf(g.sc.a, xcur[o], r);
       }
-    }
-  }
-  if (final_tile) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) rms += __shfl_xor_sync(0xffffffffu, rms, o);
-    if ((tid & 31) == 0) red[tid >> 5] = rms;
-    __syncthreads();
-    if (tid == 0) {
-      float t = 0.0f;
-      for (int w = 0; w < 8; ++w) t += red[w];
-      const int tiles_c = (mi.cols + kT32 - 1) / kT32;
-      g.ws.rms_part[mi.rms32_base + (row0 / kT32) * tiles_c + col0 / kT32] = t;
     }
   }
 }

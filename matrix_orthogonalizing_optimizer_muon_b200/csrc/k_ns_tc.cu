@@ -8,7 +8,7 @@
 //   kPhaseUpdate X' = alpha (a X + B X)      (wide)   or Y' = alpha (a Y + Y B) (tall)
 // with scale = s^2 and alpha = s on iteration 0 (s = 1/||Y||_F folds the
 // normalisation X_0 = Y/||Y||_F into the first products), 1 afterwards.  The
-// last X update instead applies the weight update of Eq. 4 (or stores O).
+// weight update of Eq. 4 is a separate elementwise pass over the last iterate.
 //
 // Structure: persistent 2-CTA clusters (one CTA per SM).  A pair owns a
 // 256 x 256 output tile; tcgen05.mma.cta_group::2 (M = 256, N <= 256, K = 16,
@@ -625,239 +625,176 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;  // warp-uniform exit
       const TileCfg c = decode_tile(g, t);
       const MatInfo& mi = g.mats[c.p];
-      const int final_tile = (g.phase == kPhaseUpdate && g.final_mode != kFinalNone);
-      if (c.skip && !final_tile) continue;
+      if (c.skip) continue;  // Y == 0: nothing downstream reads this matrix
       const int i_lo = c.row0 + static_cast<int>(rank) * kHalfM + quad * 32;  // first row of this warp
       const int i = i_lo + lane;
-      float rms = 0.0f;
-      if (c.skip) {
-        // Y == 0: O = 0, so the step is pure weight decay (or a zero output).
-        // Rows go to warps and columns to lanes so the stores coalesce.
-        const MatPtrs pt = g.ptrs[c.p];
-        const int rbase = c.row0 + static_cast<int>(rank) * kHalfM;
-        for (int rr = ew; rr < kHalfM; rr += kEpiWarps) {
-          const int r = rbase + rr;
-          if (r >= mi.rows) break;
-          float* wrow = pt.W + static_cast<size_t>(r) * mi.cols;
-          for (int j = c.col0 + lane; j < c.col0 + c.n_need; j += 32) {
-            if (g.final_mode == kFinalWeight) wrow[j] = wrow[j] - g.sc.lr * (g.sc.wd * wrow[j]);
-            else wrow[j] = 0.0f;
-          }
+      const bool upd = (g.phase == kPhaseUpdate);
+      const bool sym = !upd;
+      // inputs the epilogue reads: A (polynomial) or the hi/lo iterate (X update)
+      const __nv_bfloat16* in0 = upd ? g.ws.hi[g.cur] + mi.off_x : g.ws.A + mi.off_a;
+      const __nv_bfloat16* in1 = g.ws.lo + mi.off_x;
+      const int ld_in = upd ? mi.ld : mi.lda;
+      const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
+      const bool poly = (g.phase == kPhasePoly);
+      // a chunk needs work unless it is a block strictly above the diagonal
+      // of a symmetric output (its mirror writes it)
+      auto needed = [&](int ch) { return !(sym && (c.col0 + ch * kEpiBoxCols > i_lo + 31)); };
+      auto block_inside = [&](int ch) {
+        return i_lo + 31 < rows_in && c.col0 + ch * kEpiBoxCols + 32 <= cols_in;
+      };
+      // polynomial: coalesced prefetch of the next A block into registers
+      uint4 pf0[4];
+      auto prefetch = [&](int ch) {
+        if (!poly || !needed(ch) || !block_inside(ch)) return;
+        load_block32(in0, ld_in, i_lo, c.col0 + ch * kEpiBoxCols, lane, pf0);
+      };
+      // X update: ring of kUpdBufs (hi, lo) buffers fed by cp.async; chunk k
+      // of this warp lives in buffer k % kUpdBufs
+      auto upd_buf = [&](int b) -> uint8_t* {
+        return smem + SmemLayout::kUpdRing + (ew * kUpdBufs + b) * kUpdBufBytes;
+      };
+      int kc = 0;  // chunks of this warp in this tile
+      for (int x = grp; x < c.nch; x += kEpiGroups) ++kc;
+      int issued = 0;
+      auto stage_chunk = [&](int k) {
+        const int chh = grp + k * kEpiGroups;
+        if (block_inside(chh)) {
+          uint8_t* b = upd_buf(k % kUpdBufs);
+          cp_block32(b, in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
+          cp_block32(b + kEpiBlockBytes, in1, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
         }
+        cp_async_commit();  // one group per chunk, empty for ragged chunks
+      };
+      int ch = grp;
+      if (upd) {
+        for (; issued < kc && issued < kUpdBufs; ++issued) stage_chunk(issued);
       } else {
-        const bool upd = (g.phase == kPhaseUpdate);
-        const bool sym = !upd;
-        // inputs the epilogue reads: A (polynomial) or the hi/lo iterate (X update)
-        const __nv_bfloat16* in0 = upd ? g.ws.hi[g.cur] + mi.off_x : g.ws.A + mi.off_a;
-        const __nv_bfloat16* in1 = g.ws.lo + mi.off_x;
-        const int ld_in = upd ? mi.ld : mi.lda;
-        const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
-        const bool poly = (g.phase == kPhasePoly);
-        // a chunk needs work unless it is a block strictly above the diagonal
-        // of a symmetric output (its mirror writes it)
-        auto needed = [&](int ch) { return !(sym && (c.col0 + ch * kEpiBoxCols > i_lo + 31)); };
-        auto block_inside = [&](int ch) {
-          return i_lo + 31 < rows_in && c.col0 + ch * kEpiBoxCols + 32 <= cols_in;
-        };
-        // polynomial: coalesced prefetch of the next A block into registers
-        uint4 pf0[4];
-        auto prefetch = [&](int ch) {
-          if (!poly || !needed(ch) || !block_inside(ch)) return;
-          load_block32(in0, ld_in, i_lo, c.col0 + ch * kEpiBoxCols, lane, pf0);
-        };
-        // X update: ring of kUpdBufs (hi, lo) buffers fed by cp.async; chunk k
-        // of this warp lives in buffer k % kUpdBufs
-        auto upd_buf = [&](int b) -> uint8_t* {
-          return smem + SmemLayout::kUpdRing + (ew * kUpdBufs + b) * kUpdBufBytes;
-        };
-        int kc = 0;  // chunks of this warp in this tile
-        for (int x = grp; x < c.nch; x += kEpiGroups) ++kc;
-        int issued = 0;
-        auto stage_chunk = [&](int k) {
-          const int chh = grp + k * kEpiGroups;
-          if (block_inside(chh)) {
-            uint8_t* b = upd_buf(k % kUpdBufs);
-            cp_block32(b, in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
-            cp_block32(b + kEpiBlockBytes, in1, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
-          }
-          cp_async_commit();  // one group per chunk, empty for ragged chunks
-        };
-        int ch = grp;
+        prefetch(ch);
+      }
+      // one lane waits and the warp follows its verdict, so the warp stays
+      // converged for the .sync.aligned TMEM loads
+      int ready = 0;
+      if (lane == 0) ready = wait_bounded(tfull_bar(acc), acc_phase, abort_flag) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) {
+        if (lane == 0) raise_abort(abort_flag, status);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
+      const float s = g.ws.s[c.p];
+      for (int k = 0; ch < c.nch; ch += kEpiGroups, ++k) {
+        const int j0 = c.col0 + ch * kEpiBoxCols;
+        if (!needed(ch)) continue;
+        const bool inside = block_inside(ch);
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(t_row + static_cast<uint32_t>(ch * kEpiBoxCols), v);  // completes at tmem_ld_wait
+        uint4 xa[4], xb[4];  // this thread's row of the inputs, packed bf16
         if (upd) {
-          for (; issued < kc && issued < kUpdBufs; ++issued) stage_chunk(issued);
-        } else {
-          prefetch(ch);
-        }
-        // one lane waits and the warp follows its verdict, so the warp stays
-        // converged for the .sync.aligned TMEM loads
-        int ready = 0;
-        if (lane == 0) ready = wait_bounded(tfull_bar(acc), acc_phase, abort_flag) ? 1 : 0;
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (!ready) {
-          if (lane == 0) raise_abort(abort_flag, status);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
-        const float s = g.ws.s[c.p];
-        for (int k = 0; ch < c.nch; ch += kEpiGroups, ++k) {
-          const int j0 = c.col0 + ch * kEpiBoxCols;
-          if (!needed(ch)) continue;
-          const bool inside = block_inside(ch);
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(t_row + static_cast<uint32_t>(ch * kEpiBoxCols), v);  // completes at tmem_ld_wait
-          uint4 xa[4], xb[4];  // this thread's row of the inputs, packed bf16
-          if (upd) {
-            if (inside) {
-              cp_async_wait(issued - k - 1);
-              __syncwarp();
-              read_row32(upd_buf(k % kUpdBufs), lane, xa);
-              read_row32(upd_buf(k % kUpdBufs) + kEpiBlockBytes, lane, xb);
-              __syncwarp();
-            } else {
-              load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
-              load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
-            }
-            // this buffer is free again: fetch the chunk two ahead into it
-            if (issued < kc) {
-              stage_chunk(issued);
-              ++issued;
-            }
-          } else if (poly) {
-            if (inside) {
-              staging_free();
-              put_block32(blk0, lane, pf0);
-              __syncwarp();
-              read_row32(blk0, lane, xa);
-              __syncwarp();
-            } else {
-              load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
-            }
-            if (ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
-          }
-          tmem_ld_wait();
-          float val[32];
-          if (g.phase == kPhaseGram) {
-            const bool first = (g.iter == 0);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
-          } else if (poly) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q));
+          if (inside) {
+            cp_async_wait(issued - k - 1);
+            __syncwarp();
+            read_row32(upd_buf(k % kUpdBufs), lane, xa);
+            read_row32(upd_buf(k % kUpdBufs) + kEpiBlockBytes, lane, xb);
+            __syncwarp();
           } else {
-            const float alpha = (g.iter == 0) ? s : 1.0f;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q) + bf_at(xb, q), u2f(v[q]));
+            load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
+            load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
           }
-          if (sym) {
-            __align__(16) __nv_bfloat16 h[32];
+          // this buffer is free again: fetch the chunk two ahead into it
+          if (issued < kc) {
+            stage_chunk(issued);
+            ++issued;
+          }
+        } else if (poly) {
+          if (inside) {
+            staging_free();
+            put_block32(blk0, lane, pf0);
+            __syncwarp();
+            read_row32(blk0, lane, xa);
+            __syncwarp();
+          } else {
+            load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
+          }
+          if (ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
+        }
+        tmem_ld_wait();
+        float val[32];
+        if (g.phase == kPhaseGram) {
+          const bool first = (g.iter == 0);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
-            if (inside && j0 + 31 < i_lo) {
-              // strictly lower block: stage it and its transpose, store both
-              staging_free();
-              write_row32(blk0, lane, h);
+          for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
+        } else if (poly) {
 #pragma unroll
-              for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
-              const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
-              publish(map, j0, i_lo, map, i_lo, j0);
-            } else {
-              // diagonal or ragged block: element-wise with masks
-              __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
-              __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
+          for (int q = 0; q < 32; ++q) val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q));
+        } else {
+          const float alpha = (g.iter == 0) ? s : 1.0f;
 #pragma unroll
-              for (int q = 0; q < 32; ++q) {
-                const int j = j0 + q;
-                if (i < mi.m && j < mi.m) {
-                  if (j <= i) row[j] = h[q];
-                  if (j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
-                }
-              }
-            }
-          } else if (g.final_mode == kFinalNone) {
-            __align__(16) __nv_bfloat16 h[32];
-            __align__(16) __nv_bfloat16 l[32];
+          for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q) + bf_at(xb, q), u2f(v[q]));
+        }
+        if (sym) {
+          __align__(16) __nv_bfloat16 h[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
+          if (inside && j0 + 31 < i_lo) {
+            // strictly lower block: stage it and its transpose, store both
+            staging_free();
+            write_row32(blk0, lane, h);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
+            const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
+            publish(map, j0, i_lo, map, i_lo, j0);
+          } else {
+            // diagonal or ragged block: element-wise with masks
+            __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
+            __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              h[q] = __float2bfloat16_rn(val[q]);
-              l[q] = __float2bfloat16_rn(val[q] - __bfloat162float(h[q]));
-            }
-            if (inside) {
-              staging_free();
-              write_row32(blk0, lane, h);
-              write_row32(blk1, lane, l);
-              // blk1 follows blk0: one 3-D store writes the hi block and the lo block
-              fence_proxy_async();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_3d(tmap_of(g, c.p, kMapStHiLo0 + (g.cur ^ 1)), blk0_s, j0, i_lo, 0);
-                bulk_commit();
-              }
-            } else if (i < mi.rows) {
-              __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
-              __nv_bfloat16* lout = g.ws.lo + mi.off_x;
-              const size_t wi = static_cast<size_t>(i) * mi.ld + j0;
-#pragma unroll
-              for (int q = 0; q < 32; ++q)
-                if (j0 + q < mi.cols) {
-                  hout[wi + q] = h[q];
-                  lout[wi + q] = l[q];
-                }
-            }
-          } else if (i < mi.rows) {
-            const MatPtrs pt = g.ptrs[c.p];
-            float* wrow = pt.W + static_cast<size_t>(i) * mi.cols + j0;
-            const float scale = g.sc.rms_scale * sqrtf(static_cast<float>(mi.n));
-            const bool full = (j0 + 32 <= mi.cols);
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (j0 + q < mi.cols) rms = fmaf(val[q], val[q], rms);
-            if (full && pt.vec_ok) {
-              float4* w4 = reinterpret_cast<float4*>(wrow);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                float4 w = w4[q];
-                if (g.final_mode == kFinalWeight) {
-                  w.x = w.x - g.sc.lr * fmaf(scale, val[4 * q + 0], g.sc.wd * w.x);
-                  w.y = w.y - g.sc.lr * fmaf(scale, val[4 * q + 1], g.sc.wd * w.y);
-                  w.z = w.z - g.sc.lr * fmaf(scale, val[4 * q + 2], g.sc.wd * w.z);
-                  w.w = w.w - g.sc.lr * fmaf(scale, val[4 * q + 3], g.sc.wd * w.w);
-                } else {
-                  w = make_float4(val[4 * q], val[4 * q + 1], val[4 * q + 2], val[4 * q + 3]);
-                }
-                w4[q] = w;
-              }
-            } else {
-#pragma unroll
-              for (int q = 0; q < 32; ++q) {
-                if (j0 + q < mi.cols) {
-                  if (g.final_mode == kFinalWeight) {
-                    const float w = wrow[q];
-                    wrow[q] = w - g.sc.lr * fmaf(scale, val[q], g.sc.wd * w);
-                  } else {
-                    wrow[q] = val[q];
-                  }
-                }
+              const int j = j0 + q;
+              if (i < mi.m && j < mi.m) {
+                if (j <= i) row[j] = h[q];
+                if (j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
               }
             }
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      }
-      if (final_tile) {
+        } else {
+          __align__(16) __nv_bfloat16 h[32];
+          __align__(16) __nv_bfloat16 l[32];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) rms += __shfl_xor_sync(0xffffffffu, rms, o);
-        if (lane == 0) {
-          const int tiles_c = (mi.cols + kBN - 1) / kBN;
-          const int local = (c.row0 / kTileM) * tiles_c + c.col0 / kBN;
-          g.ws.rms_part[mi.rms_tile_base + local * kRmsSlotsPerTile + static_cast<int>(rank) * kEpiWarps + ew] = rms;
+          for (int q = 0; q < 32; ++q) {
+            h[q] = __float2bfloat16_rn(val[q]);
+            l[q] = __float2bfloat16_rn(val[q] - __bfloat162float(h[q]));
+          }
+          if (inside) {
+            staging_free();
+            write_row32(blk0, lane, h);
+            write_row32(blk1, lane, l);
+            // blk1 follows blk0: one 3-D store writes the hi block and the lo block
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(tmap_of(g, c.p, kMapStHiLo0 + (g.cur ^ 1)), blk0_s, j0, i_lo, 0);
+              bulk_commit();
+            }
+          } else if (i < mi.rows) {
+            __nv_bfloat16* hout = g.ws.hi[g.cur ^ 1] + mi.off_x;
+            __nv_bfloat16* lout = g.ws.lo + mi.off_x;
+            const size_t wi = static_cast<size_t>(i) * mi.ld + j0;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (j0 + q < mi.cols) {
+                hout[wi + q] = h[q];
+                lout[wi + q] = l[q];
+              }
+          }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
     }
     // nothing may still read or land in shared memory once the CTA exits
     if (lane == 0) bulk_wait_all();

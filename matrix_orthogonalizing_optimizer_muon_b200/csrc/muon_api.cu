@@ -230,16 +230,14 @@ struct Recorder {
 // ------------------------------------------------------------ the launch sequence
 muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int precision, int final_mode,
                      int k1_mode, float* update_rms, cudaStream_t st) {
-  Recorder rec(pl, st, 3 * ns_steps + 3);
+  Recorder rec(pl, st, 3 * ns_steps + 4);
   const int fp32 = precision == MUON_NS_FP32 ? 1 : 0;
   cudaError_t e = launch_k1(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, k1_mode, fp32, st);
   if (e != cudaSuccess) return MUON_ERR_CUDA;
   rec.mark(0);
   int cur = 0;
   for (int it = 0; it < ns_steps; ++it) {
-    const bool last = (it == ns_steps - 1);
     for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
-      const int fm = (ph == kPhaseUpdate && last) ? final_mode : kFinalNone;
       if (fp32) {
         Gemm32Args a{};
         a.tiles = (ph == kPhaseUpdate) ? pl->full32_d : pl->sym32_d;
@@ -247,7 +245,6 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
         a.phase = ph;
         a.iter = it;
         a.cur = cur;
-        a.final_mode = fm;
         a.mats = pl->mats_d;
         a.ptrs = pl->ptrs_d;
         a.ws = pl->ws;
@@ -260,7 +257,6 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
         a.phase = ph;
         a.iter = it;
         a.cur = cur;
-        a.final_mode = fm;
         a.mats = pl->mats_d;
         a.ptrs = pl->ptrs_d;
         a.tmaps = pl->tmaps_d;
@@ -271,21 +267,26 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
       if (e != cudaSuccess) return MUON_ERR_CUDA;
       rec.mark(1 + ph);
     }
-    if (!last) cur ^= 1;
+    cur ^= 1;  // the X update wrote the other buffer
   }
-  int which = fp32 ? 2 : 1;
-  if (ns_steps == 0) {
-    e = launch_apply_update(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, final_mode, fp32, st);
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
-    rec.mark(4);
-    which = 0;
-  }
-  if (update_rms != nullptr) {
-    e = launch_rms_finalize(pl->mats_d, pl->n, pl->ws.rms_part, which, update_rms, st);
+  // The last iterate is in hi[cur]/lo (x32[cur]); O = s X when N = 0.  Eq. 6
+  // needs RMS(O) before any weight changes, so it adds a reduction pass.
+  const int mul_s = ns_steps == 0 ? 1 : 0;
+  const bool norm_pass = (final_mode == kFinalWeight && sc.scale_mode == kScaleUpdateNorm);
+  if (norm_pass) {
+    e = launch_update_norm(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ws, sc, fp32, cur, mul_s, update_rms, st);
     if (e != cudaSuccess) return MUON_ERR_CUDA;
     rec.mark(4);
   }
-  pl->last_stream = st;
+  e = launch_apply_update(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, final_mode, fp32, cur,
+                          mul_s, st);
+  if (e != cudaSuccess) return MUON_ERR_CUDA;
+  rec.mark(4);
+  if (update_rms != nullptr && !norm_pass) {
+    e = launch_rms_finalize(pl->mats_d, pl->n, pl->ws.rms_part, update_rms, st);
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    rec.mark(4);
+  }
   return MUON_OK;
 }
 
@@ -329,6 +330,8 @@ muon_status_t muon_hparams_default(muon_hparams_t* hp) {
   hp->rms_scale = 0.2f;
   hp->nesterov = 1;
   hp->ns_precision = MUON_NS_BF16;
+  hp->scale_mode = MUON_SCALE_MAX_DIM;
+  hp->hidden_dim = 0.0f;
   return MUON_OK;
 }
 
@@ -371,7 +374,6 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   std::vector<TileDesc> sym, full, sym32, full32;
   std::vector<ChunkDesc> chunks;
   size_t total_x = 0, total_a = 0;
-  int rms_tc = 0, rms32 = 0;
   // LPT order of matrices for the GEMM schedules (largest Newton-Schulz work first)
   std::vector<int> order(n);
   for (int i = 0; i < n; ++i) order[i] = i;
@@ -400,12 +402,6 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
     for (int r = 0; r < R; r += rows_per_chunk)
       chunks.push_back(make_int4(i, r, std::min(rows_per_chunk, R - r), static_cast<int>(chunks.size())));
     mi.nchunks = static_cast<int>(chunks.size()) - mi.chunk_base;
-    mi.rms_tile_base = rms_tc;
-    mi.rms_tile_count = ((R + kTileM - 1) / kTileM) * ((C + kBN - 1) / kBN) * kRmsSlotsPerTile;
-    rms_tc += mi.rms_tile_count;
-    mi.rms32_base = rms32;
-    mi.rms32_count = ((R + kT32 - 1) / kT32) * ((C + kT32 - 1) / kT32);
-    rms32 += mi.rms32_count;
   }
   for (int i : order) {
     const MatInfo& mi = pl->mats[i];
@@ -445,13 +441,13 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
     o_a32 = take(total_a * 4);
     o_b32 = take(total_a * 4);
   }
-  const size_t n_rms = std::max({static_cast<size_t>(pl->nchunks), static_cast<size_t>(rms_tc),
-                                 static_cast<size_t>(rms32)});
+  const size_t n_rms = static_cast<size_t>(pl->nchunks);
   const size_t o_s = take(n * sizeof(float));
   const size_t o_np = take(pl->nchunks * sizeof(double));
   const size_t o_nc = take(n * sizeof(unsigned));
   const size_t o_rms = take(n_rms * sizeof(float));
   const size_t o_status = take(sizeof(unsigned));
+  const size_t o_unorm = take(n * sizeof(float));
   const size_t o_mats = take(n * sizeof(MatInfo));
   const size_t o_ptrs = take(n * sizeof(MatPtrs));
   const size_t o_sym = take(std::max<size_t>(1, sym.size()) * sizeof(TileDesc));
@@ -484,6 +480,7 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   ws.norm_count = reinterpret_cast<unsigned*>(b + o_nc);
   ws.rms_part = reinterpret_cast<float*>(b + o_rms);
   ws.status = reinterpret_cast<unsigned*>(b + o_status);
+  ws.unorm = reinterpret_cast<float*>(b + o_unorm);
   pl->mats_d = reinterpret_cast<MatInfo*>(b + o_mats);
   pl->ptrs_d = reinterpret_cast<MatPtrs*>(b + o_ptrs);
   pl->sym_d = reinterpret_cast<TileDesc*>(b + o_sym);
@@ -553,6 +550,11 @@ muon_status_t muon_step(muon_plan_t pl, const muon_param_t* params, int32_t n, c
     return MUON_ERR_INVALID_ARG;
   if (hp->ns_steps < 0 || hp->ns_steps > kMaxNsSteps) return MUON_ERR_INVALID_ARG;
   if (hp->nesterov != 0 && hp->nesterov != 1) return MUON_ERR_INVALID_ARG;
+  if (hp->scale_mode != MUON_SCALE_MAX_DIM && hp->scale_mode != MUON_SCALE_HIDDEN &&
+      hp->scale_mode != MUON_SCALE_UPDATE_NORM)
+    return MUON_ERR_INVALID_ARG;
+  if (hp->scale_mode == MUON_SCALE_HIDDEN && !(finite(hp->hidden_dim) && hp->hidden_dim > 0.0f))
+    return MUON_ERR_INVALID_ARG;
   if (hp->ns_precision != MUON_NS_BF16 && hp->ns_precision != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
   if (hp->ns_precision == MUON_NS_FP32 && !pl->fp32_ws) return MUON_ERR_UNSUPPORTED;
   std::vector<MatPtrs> t(n);
@@ -586,7 +588,9 @@ muon_status_t muon_step(muon_plan_t pl, const muon_param_t* params, int32_t n, c
   if (cudaGetDevice(&cur_dev) != cudaSuccess || cur_dev != pl->device) return MUON_ERR_INVALID_ARG;
   muon_status_t s = upload_ptrs(pl, t, st);
   if (s != MUON_OK) return s;
-  StepScalars sc{hp->lr, hp->weight_decay, hp->momentum, hp->a, hp->b, hp->c, hp->rms_scale, hp->nesterov};
+  StepScalars sc{hp->lr, hp->weight_decay, hp->momentum, hp->a, hp->b, hp->c, hp->rms_scale, hp->nesterov,
+                 hp->scale_mode, 0.0f};
+  if (hp->scale_mode == MUON_SCALE_HIDDEN) sc.const_scale = hp->rms_scale * std::sqrt(hp->hidden_dim);
   return run_ns(pl, sc, hp->ns_steps, hp->ns_precision, kFinalWeight, kK1Momentum, update_rms, st);
 }
 
@@ -622,7 +626,7 @@ muon_status_t muon_orthogonalize(muon_plan_t pl, const void* const* X_in, float*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   muon_status_t s = upload_ptrs(pl, t, st);
   if (s != MUON_OK) return s;
-  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0};
+  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0, kScaleMaxDim, 0.0f};
   return run_ns(pl, sc, ns_steps, ns_precision, kFinalOut, kK1Copy, nullptr, st);
 }
 

@@ -32,7 +32,6 @@ constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle at
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
 constexpr int kBoxInner = 64;   // operand boxes: 64 contiguous bf16 (128 bytes) x 128 or 64 rows
 constexpr int kEpiWarps = 8;    // epilogue warps per CTA (two per TMEM lane quadrant)
-constexpr int kRmsSlotsPerTile = 2 * kEpiWarps;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators per CTA
 
 constexpr int kChunkElems = 32768;  // elements per momentum/normalise chunk
@@ -64,6 +63,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 enum Phase : int { kPhaseGram = 0, kPhasePoly = 1, kPhaseUpdate = 2 };
 enum FinalMode : int { kFinalNone = 0, kFinalWeight = 1, kFinalOut = 2 };
 enum K1Mode : int { kK1Momentum = 0, kK1Copy = 1 };
+// scaling of the update O (Sec. 3.1): Eq. 4, Eq. 5, Eq. 6
+enum ScaleMode : int { kScaleMaxDim = 0, kScaleHidden = 1, kScaleUpdateNorm = 2 };
 
 // Per-matrix description, built once by muon_init.
 struct MatInfo {
@@ -74,11 +75,7 @@ struct MatInfo {
   int32_t lda;          // pitch of [m, m] workspace arrays (elements)
   int32_t chunk_base;   // first chunk of this matrix in the chunk list
   int32_t nchunks;
-  int32_t rms_tile_base;  // first rms partial slot of the fused final update (tensor-core tiles)
-  int32_t rms_tile_count;
-  int32_t rms32_base;     // same for the fp32 path's 64x64 tiles
-  int32_t rms32_count;
-  int32_t pad_[3];
+  int32_t pad_;
   int64_t off_x;        // element offset of this matrix in hi/lo/x32
   int64_t off_a;        // element offset in A/B/a32/b32
 };
@@ -113,12 +110,22 @@ struct Workspace {
   unsigned* norm_count; // per matrix arrival counter (self-resetting)
   float* rms_part;      // per tile-warp / chunk: sum of O^2
   unsigned* status;
+  float* unorm;         // per matrix: rms_scale / RMS(O) of the Eq. 6 update norm
 };
 
 struct StepScalars {
   float lr, wd, mu, a, b, c, rms_scale;
   int nesterov;
+  int scale_mode;       // ScaleMode
+  float const_scale;    // rms_scale * sqrt(H) for kScaleHidden
 };
+
+// Factor of O in the weight update of matrix `n` = max(rows, cols) for
+// kScaleMaxDim and kScaleHidden (kScaleUpdateNorm takes its per-matrix factor
+// from Workspace::unorm).
+__host__ __device__ __forceinline__ float update_scale_of(const StepScalars& sc, int n) {
+  return sc.scale_mode == kScaleHidden ? sc.const_scale : sc.rms_scale * sqrtf(static_cast<float>(n));
+}
 
 // Arguments of the tensor-core GEMM kernel (one launch = one phase of one
 // Newton-Schulz iteration over every matrix of the plan).
@@ -127,8 +134,7 @@ struct GemmArgs {
   int ntiles;
   int phase;            // Phase
   int iter;             // 0-based iteration index (iteration 0 folds in 1/||Y||_F)
-  int cur;              // which hi buffer holds the current iterate
-  int final_mode;       // FinalMode (only for the last kPhaseUpdate)
+  int cur;              // which hi buffer holds the current iterate (the X update writes the other)
   const MatInfo* mats;
   const MatPtrs* ptrs;
   const void* tmaps;    // CUtensorMap[kMapsPerMat * nmat], see MapIndex
@@ -140,7 +146,7 @@ struct GemmArgs {
 struct Gemm32Args {
   const TileDesc* tiles;
   int ntiles;
-  int phase, iter, cur, final_mode;
+  int phase, iter, cur;
   const MatInfo* mats;
   const MatPtrs* ptrs;
   Workspace ws;
@@ -150,11 +156,19 @@ struct Gemm32Args {
 // ---------------------------------------------------------------- launchers (host)
 cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
                       Workspace ws, StepScalars sc, int mode, int fp32_path, cudaStream_t st);
+// Weight update (or O output) from the iterate in hi[xbuf]/lo (x32[xbuf] on the
+// fp32 path); O = s * X when mul_s (ns_steps = 0), else O = X.  Per-chunk
+// sums of O^2 go to rms_part.
 cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
-                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, cudaStream_t st);
-// which: 0 chunk partials (stand-alone update), 1 tensor-core tiles, 2 fp32 tiles
-cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, int which,
-                                float* out, cudaStream_t st);
+                                Workspace ws, StepScalars sc, int final_mode, int fp32_path, int xbuf, int mul_s,
+                                cudaStream_t st);
+// Eq. 6: per matrix RMS(O) of the same iterate, unorm = rms_scale / RMS(O)
+// (0 when O = 0), and RMS(O) into update_rms when it is not null.
+cudaError_t launch_update_norm(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, Workspace ws,
+                               StepScalars sc, int fp32_path, int xbuf, int mul_s, float* update_rms,
+                               cudaStream_t st);
+// sqrt(mean(O^2)) per matrix from the per-chunk partial sums of the update pass
+cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, float* out, cudaStream_t st);
 cudaError_t launch_gemm_tc(const GemmArgs& args, int npairs, cudaStream_t st);
 // Encode the kMapsPerMat TMA descriptors of one matrix (host); false if the
 // driver entry point is missing or rejects a descriptor.

@@ -44,7 +44,7 @@ constexpr size_t kOffS = kOffB + kNaA;
 constexpr size_t kOffNormPart = kOffS + 256;
 constexpr size_t kOffNormCount = kOffNormPart + align256(kNaMaxChunks * sizeof(double));
 constexpr size_t kOffRms = kOffNormCount + 256;
-constexpr int kNaMaxRms = 4096;  // >= tiles * kRmsSlotsPerTile and >= chunks
+constexpr int kNaMaxRms = kNaMaxChunks;  // one update partial per chunk
 constexpr size_t kOffStatus = kOffRms + align256(kNaMaxRms * sizeof(float));
 constexpr size_t kOffMat = kOffStatus + 256;
 constexpr size_t kOffPtrs = kOffMat + align256(sizeof(MatInfo));
@@ -145,9 +145,6 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
       if (nfull == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
       full[nfull++] = make_int4(0, r0, c0, std::min(kBN, C - c0));
     }
-  mi.rms_tile_base = 0;
-  mi.rms_tile_count = nfull * kRmsSlotsPerTile;
-  if (mi.rms_tile_count > kNaMaxRms) return MUON_ERR_UNSUPPORTED;
   MatPtrs mp{};
   mp.W = O_out;
   mp.G = X_in;
@@ -190,11 +187,10 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   if (e != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- the same launch sequence as muon_orthogonalize on the bf16 path
-  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0};
+  StepScalars sc{0.0f, 0.0f, 0.0f, abc[0], abc[1], abc[2], 0.0f, 0, kScaleMaxDim, 0.0f};
   if (launch_k1(chunks_d, nch, mats_d, ptrs_d, ws, sc, kK1Copy, 0, st) != cudaSuccess) return MUON_ERR_CUDA;
   int cur = 0;
   for (int it = 0; it < ns_steps; ++it) {
-    const bool last = (it == ns_steps - 1);
     for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
       GemmArgs a{};
       a.tiles = (ph == kPhaseUpdate) ? full_d : sym_d;
@@ -202,7 +198,6 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
       a.phase = ph;
       a.iter = it;
       a.cur = cur;
-      a.final_mode = (ph == kPhaseUpdate && last) ? kFinalOut : kFinalNone;
       a.mats = mats_d;
       a.ptrs = ptrs_d;
       a.tmaps = tmaps_d;
@@ -210,10 +205,11 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
       a.sc = sc;
       if (launch_gemm_tc(a, g_state[dev].npairs, st) != cudaSuccess) return MUON_ERR_CUDA;
     }
-    if (!last) cur ^= 1;
+    cur ^= 1;  // the X update wrote the other buffer
   }
-  if (ns_steps == 0 &&
-      launch_apply_update(chunks_d, nch, mats_d, ptrs_d, ws, sc, kFinalOut, 0, st) != cudaSuccess)
+  // O = X from hi[cur] + lo, or s Y when there are no iterations
+  if (launch_apply_update(chunks_d, nch, mats_d, ptrs_d, ws, sc, kFinalOut, 0, cur, ns_steps == 0 ? 1 : 0, st) !=
+      cudaSuccess)
     return MUON_ERR_CUDA;
   return MUON_OK;
 }

@@ -49,13 +49,18 @@ def random_bf16(shape, seed, scale=1.0):
 
 
 def check_step(W_prev, M_prev, G, W_new, M_new, rms_gpu, *, lr, wd, mu, ns_steps=5, coeffs=ABC32,
-               precision="bf16", nesterov=True):
+               precision="bf16", nesterov=True, scale_mode=orc.SCALE_MAX_DIM, hidden_dim=0.0):
     """Compare one GPU step of one matrix with the oracle run from the GPU's
     own W_{t-1} and M_{t-1}.  Returns a dict of the measured errors."""
     R, C = W_prev.shape
     ref = orc.muon_step(W_prev, G, M_prev, lr=lr, weight_decay=wd, momentum_coef=mu, ns_steps=ns_steps,
-                        coeffs=coeffs, nesterov=nesterov)
-    scale = orc.update_scale(R, C)
+                        coeffs=coeffs, nesterov=nesterov, scale_mode=scale_mode, hidden_dim=hidden_dim)
+    if scale_mode == orc.SCALE_HIDDEN:
+        scale = orc.update_scale_hidden(hidden_dim)
+    elif scale_mode == orc.SCALE_UPDATE_NORM:
+        scale = orc.update_norm_scale(ref.O)
+    else:
+        scale = orc.update_scale(R, C)
     dW_gpu = W_new - W_prev
     dW_ref = ref.W - W_prev
     bound = TOL_DW * lr * scale

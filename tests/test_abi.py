@@ -58,7 +58,23 @@ def test_default_hparams_are_the_pages_values(lib):
     assert hp.ns_steps == 5 and abs(hp.momentum - 0.95) < 1e-7 and abs(hp.rms_scale - 0.2) < 1e-7
     assert abs(hp.weight_decay - 0.1) < 1e-7 and abs(hp.lr - 4.2e-4) < 1e-10
     assert hp.nesterov == 1 and hp.ns_precision == L.MUON_NS_BF16
+    assert hp.scale_mode == L.MUON_SCALE_MAX_DIM and hp.hidden_dim == 0.0
     assert lib.muon_hparams_default(None) == L.MUON_ERR_INVALID_ARG
+
+
+def test_binding_layouts_and_enums_match_the_header():
+    import re
+    hdr = open(os.path.join(ROOT, "include", "muon.h")).read()
+    # every field of muon_hparams_t is 4 bytes wide, in declaration order
+    end = hdr.index("} muon_hparams_t;")
+    body = hdr[hdr.rindex("typedef struct {", 0, end) + len("typedef struct {"):end]
+    names = re.findall(r"^\s*(?:float|int32_t)\s+([\w, ]+);", body, re.M)
+    fields = [n.strip() for group in names for n in group.split(",")]
+    assert fields == [f for f, _ in L.muon_hparams_t._fields_]
+    assert ctypes.sizeof(L.muon_hparams_t) == 4 * len(fields)
+    for name in ("MUON_SCALE_MAX_DIM", "MUON_SCALE_HIDDEN", "MUON_SCALE_UPDATE_NORM", "MUON_NS_BF16", "MUON_NS_FP32"):
+        m = re.search(name + r"\s*=\s*(\d+)", hdr)
+        assert m and int(m.group(1)) == getattr(L, name), name
 
 
 def test_init_rejects_bad_arguments_before_any_cuda_call(lib):
