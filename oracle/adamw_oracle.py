@@ -8,7 +8,7 @@ with the CUDA path.
 2025) updates the parameters that are not matrices -- RMSNorm gains, the
 embedding and the LM head -- with AdamW, sharing the learning rate and the
 weight decay with Muon (Sec. 2.2, "Matching update RMS of AdamW"; weight decay
-on the RMSNorm gains, Appendix C).  The pages cite AdamW (Loshchilov and
+on the RMSNorm gains, Appendix D, "Training stability").  The pages cite AdamW (Loshchilov and
 Hutter 2019) without restating it, so this is the algorithm of that paper with
 decoupled weight decay and bias correction:
 
