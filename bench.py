@@ -144,6 +144,47 @@ def replica_tflops(world: int, flops_per_rank: int, ms_step: float) -> float:
     return world * flops_per_rank / (ms_step * 1e-3) / 1e12
 
 
+# ---------------------------------------------------------------------- AdamW companion leg
+
+ADAMW_NUMELS = [65536 * 2048, 65536 * 2048] + [2048] * 16   # embedding, LM head, 16 RMSNorm gains
+ADAMW_BYTES_PER_ELEM = 26                                    # P 4+4, m 4+4, v 4+4, G (bf16) 2
+
+
+def bench_adamw(dev, steps: int = 20, warmup: int = 3):
+    """Time the fused AdamW step on synthetic non-matrix parameters (inputs
+    larger than L2); returns the bench line's `adamw_companion` object."""
+    import torch
+    from matrix_orthogonalizing_optimizer_muon_b200.api import AdamWPlan
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(77)
+    ts = []
+    for e in ADAMW_NUMELS:
+        P = torch.empty(e, device=dev).normal_(0.0, 0.02, generator=gen)
+        G = torch.empty(e, device=dev).normal_(0.0, 1e-3, generator=gen).to(torch.bfloat16)
+        ts.append((P, G, torch.empty(e, device=dev), torch.empty(e, device=dev)))
+    plan = AdamWPlan(ADAMW_NUMELS, states=[(m, v) for _, _, m, v in ts])
+    for t in range(1, warmup + 1):
+        plan.step(ts, step=t, lr=4.2e-4, weight_decay=0.1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(warmup + 1, warmup + steps + 1):
+        plan.step(ts, step=t, lr=4.2e-4, weight_decay=0.1)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    plan.close()
+    total = sum(ADAMW_NUMELS)
+    gbs = total * ADAMW_BYTES_PER_ELEM / (ms * 1e-3) / 1e9
+    peaks, kind = load_peaks()
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"kernel": "adamw_kernel (fused multi-tensor AdamW)", "bound": "hbm",
+            "workload": "synthetic non-matrix parameters: embedding and LM head [65536, 2048] and 16 RMSNorm "
+                        "gains [2048], bf16 gradients, fp32 P/m/v",
+            "elements": total, "ms_per_step": ms, "achieved": gbs, "unit": "GB/s", "peak": peak,
+            "peak_source": f"hbm_gbs ({kind})", "frac": gbs / peak, "bytes_per_elem": ADAMW_BYTES_PER_ELEM}
+
+
 # ---------------------------------------------------------------------- oracle (CPU) legs
 
 def cpu_sample(wl, budget_s: float, seed: int = 0):
@@ -262,6 +303,7 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", default="moe")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the PyTorch eager comparison point")
+    ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
     ap.add_argument("--scale", default="max_dim", choices=["max_dim", "hidden", "update_norm"],
                     help="update scale of Sec. 3.1: Eq. 4 (default), Eq. 5 with H = 2048, Eq. 6")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -402,6 +444,13 @@ def main(argv=None) -> int:
                    "ns_ms_per_step": t_eager, "tflops_algorithmic": nz_flops / (t_eager * 1e-3) / 1e12,
                    "tflops_dense_equivalent": dense_flops / (t_eager * 1e-3) / 1e12}
 
+    adamw = None
+    if not args.no_adamw:
+        plan.close()
+        del Wbuf, Gbuf, Mbuf, Ws, Gs, Ms, params
+        torch.cuda.empty_cache()
+        adamw = bench_adamw(dev)
+
     cpu = None
     if world == 1 and args.cpu_budget > 0:
         f, s, d = cpu_sample(wl, args.cpu_budget)
@@ -437,6 +486,7 @@ def main(argv=None) -> int:
                         "bytes_per_elem": K1_BYTES_PER_ELEM},
         "cpu_baseline": cpu,
         "context_torch_eager_ns": context,
+        "adamw_companion": adamw,
         "e2e": e2e,
         "gpu_launches": int(round(per_step_launches * args.steps)),
         "clocks": clk.summary(),

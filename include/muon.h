@@ -196,6 +196,60 @@ MUON_API muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_out
                                                   int32_t in_dtype, int32_t ns_steps, const float abc[3],
                                                   void* stream);
 
+/* ------------------------------------------------------------------------
+ * AdamW companion for the parameters that are not matrices.  The pages
+ * update RMSNorm gains, the embedding and the LM head with AdamW, sharing the
+ * learning rate and weight decay with Muon (Sec. 2.2, "Matching update RMS of
+ * AdamW"; decay on the RMSNorm gains, Appendix D).  The algorithm is AdamW as
+ * the pages cite it (Loshchilov and Hutter 2019), per element:
+ *   m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2
+ *   P <- P - lr ( m / (1 - beta1^t) / (sqrt(v / (1 - beta2^t)) + eps) + wd P )
+ * with wd = weight_decay for tensors with decay = 1 and 0 otherwise.  One
+ * fused launch streams every tensor of the plan (fp32 arithmetic, about
+ * 26 bytes of HBM traffic per element with a bf16 gradient).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  float*      P;        /* fp32 parameter [numel], updated in place                      */
+  const void* G;        /* gradient [numel], dtype g_dtype, read only                    */
+  float*      m;        /* fp32 first moment [numel], updated in place                   */
+  float*      v;        /* fp32 second moment [numel], updated in place                  */
+  int64_t     numel;    /* 1 <= numel <= 2^31 - 1                                        */
+  int32_t     g_dtype;  /* muon_dtype_t                                                   */
+  int32_t     decay;    /* 1: decoupled weight decay on this tensor, 0: none             */
+} muon_adamw_param_t;
+
+typedef struct {
+  float   lr;            /* eta_t, shared with Muon                                        */
+  float   beta1, beta2;  /* moment decay rates, each in [0, 1) (not given by the pages)    */
+  float   eps;           /* > 0                                                            */
+  float   weight_decay;  /* lambda, shared with Muon                                       */
+  int32_t step;          /* t >= 1 of this update, for the bias corrections                */
+} muon_adamw_hparams_t;
+
+typedef struct muon_adamw_plan_s* muon_adamw_plan_t;
+
+/* lr 4.2e-4, beta1 0.9, beta2 0.95, eps 1e-8, weight_decay 0.1, step 1.
+ * Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
+MUON_API muon_status_t muon_adamw_hparams_default(muon_adamw_hparams_t* hp);
+
+/* Plan for a fixed list of n >= 1 tensors (only numel and g_dtype are kept;
+ * MUON_INIT_ZERO_MOMENTUM zeroes every m and v on `stream`, the usual
+ * m_0 = v_0 = 0).  Errors: INVALID_ARG, NO_MEMORY, CUDA, UNSUPPORTED (not an
+ * sm_100 device). */
+MUON_API muon_status_t muon_adamw_init(muon_adamw_plan_t* out, const muon_adamw_param_t* params, int32_t n,
+                                       uint32_t flags, void* stream);
+
+/* One AdamW step over every tensor, asynchronous on `stream`.  params must
+ * match the plan (count, numel, g_dtype); P, m and v of all tensors and every
+ * G must not overlap.  Validated before anything is enqueued: INVALID_ARG
+ * (bad pointer, hyper-parameter or step), SHAPE_MISMATCH, ALIAS; launch
+ * failures give MUON_ERR_CUDA. */
+MUON_API muon_status_t muon_adamw_step(muon_adamw_plan_t plan, const muon_adamw_param_t* params, int32_t n,
+                                       const muon_adamw_hparams_t* hp, void* stream);
+
+/* Waits for the plan's last stream and frees it; NULL is ignored. */
+MUON_API void muon_adamw_destroy(muon_adamw_plan_t plan);
+
 #ifdef __cplusplus
 }
 #endif

@@ -35,7 +35,8 @@ PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
 
 EXPORTED = ("muon_hparams_default", "muon_init", "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
             "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read",
-            "muon_orthogonalize_noalloc")
+            "muon_orthogonalize_noalloc", "muon_adamw_hparams_default", "muon_adamw_init", "muon_adamw_step",
+            "muon_adamw_destroy")
 
 
 class muon_param_t(ctypes.Structure):
@@ -49,6 +50,16 @@ class muon_hparams_t(ctypes.Structure):
                 ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float), ("b", ctypes.c_float),
                 ("c", ctypes.c_float), ("rms_scale", ctypes.c_float), ("nesterov", ctypes.c_int32),
                 ("ns_precision", ctypes.c_int32), ("scale_mode", ctypes.c_int32), ("hidden_dim", ctypes.c_float)]
+
+
+class muon_adamw_param_t(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_void_p), ("G", ctypes.c_void_p), ("m", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("numel", ctypes.c_int64), ("g_dtype", ctypes.c_int32), ("decay", ctypes.c_int32)]
+
+
+class muon_adamw_hparams_t(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32)]
 
 
 class MuonError(RuntimeError):
@@ -95,6 +106,16 @@ def load() -> ctypes.CDLL:
     lib.muon_orthogonalize_noalloc.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.POINTER(ctypes.c_float), P]
     lib.muon_orthogonalize_noalloc.restype = ctypes.c_int
+    lib.muon_adamw_hparams_default.argtypes = [ctypes.POINTER(muon_adamw_hparams_t)]
+    lib.muon_adamw_hparams_default.restype = ctypes.c_int
+    lib.muon_adamw_init.argtypes = [ctypes.POINTER(P), ctypes.POINTER(muon_adamw_param_t), ctypes.c_int32,
+                                    ctypes.c_uint32, P]
+    lib.muon_adamw_init.restype = ctypes.c_int
+    lib.muon_adamw_step.argtypes = [P, ctypes.POINTER(muon_adamw_param_t), ctypes.c_int32,
+                                    ctypes.POINTER(muon_adamw_hparams_t), P]
+    lib.muon_adamw_step.restype = ctypes.c_int
+    lib.muon_adamw_destroy.argtypes = [P]
+    lib.muon_adamw_destroy.restype = None
     _lib = lib
     return lib
 
@@ -164,3 +185,24 @@ def muon_profile_read(plan):
     calls = ctypes.c_int32()
     check(load().muon_profile_read(plan, ms, cnt, ctypes.byref(calls)), "muon_profile_read")
     return list(ms), list(cnt), int(calls.value)
+
+
+def muon_adamw_hparams_default() -> muon_adamw_hparams_t:
+    hp = muon_adamw_hparams_t()
+    check(load().muon_adamw_hparams_default(ctypes.byref(hp)), "muon_adamw_hparams_default")
+    return hp
+
+
+def muon_adamw_init(params, n: int, flags: int, stream: int) -> ctypes.c_void_p:
+    plan = ctypes.c_void_p()
+    check(load().muon_adamw_init(ctypes.byref(plan), params, int(n), int(flags), ctypes.c_void_p(stream)),
+          "muon_adamw_init")
+    return plan
+
+
+def muon_adamw_step(plan, params, n: int, hp: muon_adamw_hparams_t, stream: int) -> None:
+    check(load().muon_adamw_step(plan, params, int(n), ctypes.byref(hp), ctypes.c_void_p(stream)), "muon_adamw_step")
+
+
+def muon_adamw_destroy(plan) -> None:
+    load().muon_adamw_destroy(plan)

@@ -6,9 +6,13 @@ pointers, shapes and the current CUDA stream to the C ABI.
     plan = MuonPlan([W.shape for W in weights], zero_momentum_of=[M...])
     plan.step(list(zip(weights, grads, moms)), lr=4.2e-4, weight_decay=0.1)
 
-Matrices only: the hybrid split of "Muon is Scalable for LLM Training"
-(Sec. 2.2) sends 1-D parameters, embeddings and the LM head to AdamW, which is
-the caller's business.
+The hybrid split of "Muon is Scalable for LLM Training" (Sec. 2.2) sends the
+parameters that are not matrices (RMSNorm gains, embedding, LM head) to
+AdamW with the same learning rate and weight decay; ``AdamWPlan`` does that
+step for them.
+
+    adam = AdamWPlan([g.numel() for g in gains], states=[(m, v) ...])
+    adam.step(list(zip(gains, grads, ms, vs)), step=t, lr=4.2e-4, weight_decay=0.1)
 """
 
 from __future__ import annotations
@@ -150,6 +154,64 @@ class MuonPlan:
     def close(self) -> None:
         if getattr(self, "_plan", None):
             L.muon_destroy(self._plan)
+            self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class AdamWPlan:
+    """A libmuon AdamW plan for a fixed list of tensors (sizes and gradient
+    dtypes) on the current device."""
+
+    def __init__(self, numels, *, g_dtypes=None, states=None, stream=None):
+        self.numels = [int(v) for v in numels]
+        self.n = len(self.numels)
+        self.g_dtypes = list(g_dtypes) if g_dtypes is not None else [torch.bfloat16] * self.n
+        arr = (L.muon_adamw_param_t * self.n)()
+        flags = 0
+        if states is not None:
+            flags |= L.MUON_INIT_ZERO_MOMENTUM
+            for i, (m, v) in enumerate(states):
+                _check_tensor(m, torch.float32, f"m[{i}]")
+                _check_tensor(v, torch.float32, f"v[{i}]")
+                arr[i].m, arr[i].v = m.data_ptr(), v.data_ptr()
+        for i, e in enumerate(self.numels):
+            arr[i].numel = e
+            arr[i].g_dtype = _GDT[self.g_dtypes[i]]
+            arr[i].decay = 1
+        self._plan = L.muon_adamw_init(arr, self.n, flags, _stream_handle(stream))
+        self._params = (L.muon_adamw_param_t * self.n)()
+
+    def step(self, tensors, *, step: int, lr: float, weight_decay: float, betas=(0.9, 0.95), eps: float = 1e-8,
+             decay=None, stream=None) -> None:
+        """One AdamW step: tensors = [(P, G, m, v), ...] in plan order; `decay`
+        (list of bools, default all True) selects the tensors that get weight
+        decay."""
+        if len(tensors) != self.n:
+            raise ValueError("one (P, G, m, v) per planned tensor")
+        for i, (P, G, m, v) in enumerate(tensors):
+            e = self.numels[i]
+            _check_tensor(P, torch.float32, f"P[{i}]")
+            _check_tensor(G, self.g_dtypes[i], f"G[{i}]")
+            _check_tensor(m, torch.float32, f"m[{i}]")
+            _check_tensor(v, torch.float32, f"v[{i}]")
+            if not (P.numel() == G.numel() == m.numel() == v.numel() == e):
+                raise ValueError(f"tensor {i} does not have {e} elements")
+            a = self._params[i]
+            a.P, a.G, a.m, a.v = P.data_ptr(), G.data_ptr(), m.data_ptr(), v.data_ptr()
+            a.numel = e
+            a.g_dtype = _GDT[self.g_dtypes[i]]
+            a.decay = 1 if (decay is None or decay[i]) else 0
+        hp = L.muon_adamw_hparams_t(lr, betas[0], betas[1], eps, weight_decay, int(step))
+        L.muon_adamw_step(self._plan, self._params, self.n, hp, _stream_handle(stream))
+
+    def close(self) -> None:
+        if getattr(self, "_plan", None):
+            L.muon_adamw_destroy(self._plan)
             self._plan = None
 
     def __del__(self):
