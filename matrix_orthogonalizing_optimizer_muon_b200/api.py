@@ -66,29 +66,39 @@ class MuonPlan:
         self._plan = L.muon_init(arr, self.n, flags, _stream_handle(stream))
         self._params = (L.muon_param_t * self.n)()
         self._key = None
+        self._bound = {}   # recent bindings: key -> descriptor array
         self._x = (ctypes.c_void_p * self.n)()
         self._o = (ctypes.c_void_p * self.n)()
 
     # ------------------------------------------------------------ the step
     def bind(self, params):
-        """Fill the descriptor array from [(W, G, M), ...]; reused by step()
-        while the same tensors are passed again."""
+        """Fill the descriptor array from [(W, G, M), ...].  The last few
+        distinct bindings are kept, so alternating between buffer sets (double
+        buffered gradients) costs no re-validation."""
         if len(params) != self.n:
             raise ValueError(f"expected {self.n} (W, G, M) triples, got {len(params)}")
         key = tuple((W.data_ptr(), G.data_ptr(), M.data_ptr(), G.dtype) for W, G, M in params)
         if key == self._key:
             return
+        cached = self._bound.get(key)
+        if cached is not None:
+            self._params, self._key = cached, key
+            return
+        arr = (L.muon_param_t * self.n)()
         for i, (W, G, M) in enumerate(params):
             shp = self.shapes[i]
             _check_tensor(W, torch.float32, f"W[{i}]", shp)
             _check_tensor(G, (torch.bfloat16, torch.float32), f"G[{i}]", shp)
             _check_tensor(M, torch.float32, f"M[{i}]", shp)
-            d = self._params[i]
+            d = arr[i]
             d.W, d.G, d.M = W.data_ptr(), G.data_ptr(), M.data_ptr()
             d.rows, d.cols = shp
             d.g_dtype = _GDT[G.dtype]
             d.reserved = 0
-        self._key = key
+        if len(self._bound) >= 4:
+            self._bound.pop(next(iter(self._bound)))
+        self._bound[key] = arr
+        self._params, self._key = arr, key
 
     def step(self, params=None, *, lr: float, weight_decay: float, momentum: float = 0.95, ns_steps: int = 5,
              coeffs=DEFAULT_COEFFS, rms_scale: float = 0.2, nesterov: bool = True, precision: str = "bf16",

@@ -126,7 +126,6 @@ struct muon_plan_s {
   size_t dbytes = 0;
   Workspace ws{};
   MatInfo* mats_d = nullptr;
-  MatPtrs* ptrs_d = nullptr;
   TileDesc* sym_d = nullptr;
   TileDesc* full_d = nullptr;
   TileDesc* sym32_d = nullptr;
@@ -135,12 +134,24 @@ struct muon_plan_s {
   ChunkDesc* chunks_d = nullptr;
   int nchunks = 0;
   void* tmaps_d = nullptr;
-  // per-call pointer table cache
-  std::vector<MatPtrs> ptr_cache;
-  bool ptr_cache_valid = false;
-  MatPtrs* ptr_pinned = nullptr;
-  cudaEvent_t ptr_event = nullptr;
-  bool ptr_event_pending = false;
+  // Per-call pointer tables, kept resident on the device: a call whose
+  // pointers match a kept table uses it with no copy.  A caller that
+  // alternates between buffer sets (double-buffered gradients) thus issues no
+  // host-to-device copy per step; such a small copy would otherwise queue on
+  // the copy engine behind the caller's own large input copies.
+  struct PtrSlot {
+    MatPtrs* dev = nullptr;     // device table
+    MatPtrs* pinned = nullptr;  // staging of its last upload
+    cudaEvent_t ev = nullptr;   // that upload has been read
+    bool pending = false;
+    bool valid = false;
+    uint64_t last_use = 0;
+    std::vector<MatPtrs> host;  // what the device table holds
+  };
+  static constexpr int kPtrSlots = 4;
+  PtrSlot slots[kPtrSlots];
+  MatPtrs* ptrs_d = nullptr;    // the table of the current call
+  uint64_t use_clock = 0;
   cudaStream_t last_stream = nullptr;
   // profiling
   bool prof = false;
@@ -169,22 +180,33 @@ bool any_overlap(std::vector<Interval>& v) {
   return false;
 }
 
-// Upload the per-call pointer table if it differs from the last one.
+// Make pl->ptrs_d a device table holding `t`: a kept table if one matches,
+// else the least recently used slot, refilled by an asynchronous copy on `st`
+// (stream order protects kernels of earlier calls still reading it).
 muon_status_t upload_ptrs(muon_plan_s* pl, const std::vector<MatPtrs>& t, cudaStream_t st) {
-  if (pl->ptr_cache_valid && std::memcmp(t.data(), pl->ptr_cache.data(), t.size() * sizeof(MatPtrs)) == 0)
-    return MUON_OK;
-  if (pl->ptr_event_pending) {
-    if (cudaEventSynchronize(pl->ptr_event) != cudaSuccess) return MUON_ERR_CUDA;
-    pl->ptr_event_pending = false;
+  const size_t bytes = t.size() * sizeof(MatPtrs);
+  muon_plan_s::PtrSlot* victim = nullptr;
+  for (auto& sl : pl->slots) {
+    if (sl.valid && std::memcmp(t.data(), sl.host.data(), bytes) == 0) {
+      sl.last_use = ++pl->use_clock;
+      pl->ptrs_d = sl.dev;
+      return MUON_OK;
+    }
+    if (victim == nullptr || !sl.valid || (victim->valid && sl.last_use < victim->last_use)) victim = &sl;
   }
-  std::memcpy(pl->ptr_pinned, t.data(), t.size() * sizeof(MatPtrs));
-  if (cudaMemcpyAsync(pl->ptrs_d, pl->ptr_pinned, t.size() * sizeof(MatPtrs), cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
+  if (victim->pending) {  // its staging buffer may still be read by the previous upload
+    if (cudaEventSynchronize(victim->ev) != cudaSuccess) return MUON_ERR_CUDA;
+    victim->pending = false;
+  }
+  std::memcpy(victim->pinned, t.data(), bytes);
+  if (cudaMemcpyAsync(victim->dev, victim->pinned, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MUON_ERR_CUDA;
-  if (cudaEventRecord(pl->ptr_event, st) != cudaSuccess) return MUON_ERR_CUDA;
-  pl->ptr_event_pending = true;
-  pl->ptr_cache = t;
-  pl->ptr_cache_valid = true;
+  if (cudaEventRecord(victim->ev, st) != cudaSuccess) return MUON_ERR_CUDA;
+  victim->pending = true;
+  victim->host = t;
+  victim->valid = true;
+  victim->last_use = ++pl->use_clock;
+  pl->ptrs_d = victim->dev;
   return MUON_OK;
 }
 
@@ -293,8 +315,10 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
 void free_plan(muon_plan_s* pl) {
   if (pl == nullptr) return;
   if (pl->dmem) cudaFree(pl->dmem);
-  if (pl->ptr_pinned) cudaFreeHost(pl->ptr_pinned);
-  if (pl->ptr_event) cudaEventDestroy(pl->ptr_event);
+  for (auto& sl : pl->slots) {
+    if (sl.pinned) cudaFreeHost(sl.pinned);
+    if (sl.ev) cudaEventDestroy(sl.ev);
+  }
   for (cudaEvent_t ev : pl->events) cudaEventDestroy(ev);
   delete pl;
 }
@@ -449,7 +473,7 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   const size_t o_status = take(sizeof(unsigned));
   const size_t o_unorm = take(n * sizeof(float));
   const size_t o_mats = take(n * sizeof(MatInfo));
-  const size_t o_ptrs = take(n * sizeof(MatPtrs));
+  const size_t o_ptrs = take(muon_plan_s::kPtrSlots * n * sizeof(MatPtrs));
   const size_t o_sym = take(std::max<size_t>(1, sym.size()) * sizeof(TileDesc));
   const size_t o_full = take(std::max<size_t>(1, full.size()) * sizeof(TileDesc));
   const size_t o_sym32 = take(std::max<size_t>(1, sym32.size()) * sizeof(TileDesc));
@@ -482,7 +506,8 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   ws.status = reinterpret_cast<unsigned*>(b + o_status);
   ws.unorm = reinterpret_cast<float*>(b + o_unorm);
   pl->mats_d = reinterpret_cast<MatInfo*>(b + o_mats);
-  pl->ptrs_d = reinterpret_cast<MatPtrs*>(b + o_ptrs);
+  for (int k = 0; k < muon_plan_s::kPtrSlots; ++k) pl->slots[k].dev = reinterpret_cast<MatPtrs*>(b + o_ptrs) + k * n;
+  pl->ptrs_d = pl->slots[0].dev;
   pl->sym_d = reinterpret_cast<TileDesc*>(b + o_sym);
   pl->full_d = reinterpret_cast<TileDesc*>(b + o_full);
   pl->sym32_d = reinterpret_cast<TileDesc*>(b + o_sym32);
@@ -518,9 +543,11 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   ok = ok && cudaMemset(ws.norm_count, 0, n * sizeof(unsigned)) == cudaSuccess;
   ok = ok && cudaMemset(ws.status, 0, sizeof(unsigned)) == cudaSuccess;
   ok = ok && cudaMemset(ws.s, 0, n * sizeof(float)) == cudaSuccess;
-  ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&pl->ptr_pinned), n * sizeof(MatPtrs), cudaHostAllocDefault) ==
-                 cudaSuccess;
-  ok = ok && cudaEventCreateWithFlags(&pl->ptr_event, cudaEventDisableTiming) == cudaSuccess;
+  for (auto& sl : pl->slots) {
+    ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&sl.pinned), n * sizeof(MatPtrs), cudaHostAllocDefault) ==
+                   cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&sl.ev, cudaEventDisableTiming) == cudaSuccess;
+  }
   if (!ok) {
     cudaGetLastError();
     free_plan(pl);

@@ -136,3 +136,25 @@ def test_workspace_and_profile_accounting():
     assert prof["launches"]["gram"] == 5 and prof["launches"]["poly"] == 5 and prof["launches"]["x_update"] == 5
     assert prof["launches"]["momentum_normalise"] == 1
     assert all(v >= 0 for v in prof["ms"].values())
+
+
+def test_rotating_buffer_sets_use_their_own_pointers():
+    # the plan keeps a few device pointer tables; six distinct (W, G, M) sets
+    # in rotation (more sets than tables) must each see exactly their own
+    # step, bit for bit the same as a fresh plan on that set alone
+    sets = [make(100 + k) for k in range(6)]
+    fresh = [make(100 + k) for k in range(6)]
+    plan = MuonPlan(SHAPES)
+    for _ in range(2):
+        for Ws, Gs, Ms in sets:
+            plan.step(list(zip(Ws, Gs, Ms)), lr=LR, weight_decay=WD, momentum=MU, coeffs=ABC32)
+    for Ws, Gs, Ms in fresh:
+        p = MuonPlan(SHAPES)
+        for _ in range(2):
+            p.step(list(zip(Ws, Gs, Ms)), lr=LR, weight_decay=WD, momentum=MU, coeffs=ABC32)
+        p.close()
+    torch.cuda.synchronize()
+    for (W1, _, M1), (W2, _, M2) in zip(sets, fresh):
+        for a, b in zip(W1 + M1, W2 + M2):
+            assert torch.equal(a, b)
+    plan.close()
