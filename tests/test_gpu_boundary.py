@@ -158,3 +158,33 @@ def test_rotating_buffer_sets_use_their_own_pointers():
         for a, b in zip(W1 + M1, W2 + M2):
             assert torch.equal(a, b)
     plan.close()
+
+
+def test_step_replays_from_a_cuda_graph():
+    # After one eager call with the same tensors (which uploads the pointer
+    # table), a step enqueues kernels only, so it can be captured once and
+    # replayed; the replays must equal eager steps bit for bit.
+    Ws, Gs, Ms = make(8)
+    We, Ge, Me = make(8)
+    hp = dict(lr=LR, weight_decay=WD, momentum=MU, coeffs=ABC32)
+    eager = MuonPlan(SHAPES)
+    for _ in range(4):
+        eager.step(list(zip(We, Ge, Me)), **hp)
+    plan = MuonPlan(SHAPES)
+    plan.step(list(zip(Ws, Gs, Ms)), **hp)          # step 1, eager
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            plan.step(list(zip(Ws, Gs, Ms)), **hp)  # captured, not run
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):                               # steps 2..4
+        graph.replay()
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    for a, b in zip(Ws + Ms, We + Me):
+        assert torch.equal(a, b)
+    del graph
+    plan.close()
+    eager.close()
