@@ -69,8 +69,8 @@ typedef enum { MUON_NS_BF16 = 0, MUON_NS_FP32 = 1 } muon_ns_precision_t;
  *   MUON_SCALE_HIDDEN      rms_scale * sqrt(hidden_dim)        Eq. 5, "Baseline": one H for all
  *   MUON_SCALE_UPDATE_NORM rms_scale / RMS(O), 0 when O = 0    Eq. 6, "Update Norm": every
  *                          matrix's update has RMS exactly rms_scale.  Needs RMS(O) before any
- *                          weight changes, so the step adds a reduction pass and an apply pass
- *                          over the iterate instead of the update fused into the last product. */
+ *                          weight changes, so the step adds one reduction pass over the last
+ *                          iterate before the update pass. */
 typedef enum { MUON_SCALE_MAX_DIM = 0, MUON_SCALE_HIDDEN = 1, MUON_SCALE_UPDATE_NORM = 2 } muon_scale_mode_t;
 
 /* muon_init flags */
@@ -109,7 +109,8 @@ typedef struct muon_plan_s* muon_plan_t;
 /* Fill `hp` with the pages' values: lr 4.2e-4 (Sec. 3.3 peak), weight_decay 0.1
  * (Sec. 3.3), momentum 0.95, ns_steps 5 (Sec. 2.2), (a, b, c) =
  * (3.4445, -4.7750, 2.0315) (Sec. 2.1), rms_scale 0.2 (Eq. 4), nesterov 1,
- * ns_precision MUON_NS_BF16, scale_mode MUON_SCALE_MAX_DIM, hidden_dim 0.  Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
+ * ns_precision MUON_NS_BF16, scale_mode MUON_SCALE_MAX_DIM, hidden_dim 0.
+ * Errors: MUON_ERR_INVALID_ARG if hp is NULL. */
 MUON_API muon_status_t muon_hparams_default(muon_hparams_t* hp);
 
 /* Build a plan for `n` matrices with the shapes in params[0..n).  The plan
@@ -126,11 +127,16 @@ MUON_API muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, i
 /* One Muon step over all n matrices of the plan (n and every shape must equal
  * the plan's):  M <- mu M + G;  Y = mu M + G (or M);  O = Newton-Schulz(Y) with
  * N = hp->ns_steps in the wide orientation (a matrix with rows > cols is
- * treated as its transpose; no data is transposed);  W <- W - lr (rms_scale
- * sqrt(max(rows, cols)) O + weight_decay W).  A matrix whose Y is exactly 0
- * gets O = 0 (pure weight decay).  If update_rms is not NULL it receives, on
+ * treated as its transpose; no data is transposed);  W <- W - lr (scale O +
+ * weight_decay W) with scale rms_scale sqrt(max(rows, cols)) (Eq. 4), or as
+ * hp->scale_mode selects.  A matrix whose Y is exactly 0 gets O = 0 (pure
+ * weight decay).  If update_rms is not NULL it receives, on
  * the device, n floats sqrt(mean(O^2)) in descriptor order.
  * W, G, M of all descriptors must be pairwise disjoint.
+ * The plan keeps the device copies of the last few distinct pointer tables,
+ * so alternating between buffer sets (double-buffered gradients) issues no
+ * copy once each set has been seen; after such a warm-up call a step
+ * enqueues kernels only and can be captured in a CUDA graph.
  * Errors: INVALID_ARG, SHAPE_MISMATCH, ALIAS, UNSUPPORTED, CUDA.  Non-finite
  * norms and device-side timeouts are reported later by muon_get_status. */
 MUON_API muon_status_t muon_step(muon_plan_t plan, const muon_param_t* params, int32_t n, const muon_hparams_t* hp,
@@ -164,8 +170,8 @@ MUON_API const char* muon_status_string(muon_status_t s);
 /* Phase timing, for measurement.  When enabled, every step/orthogonalize call
  * records CUDA events on its stream at each phase boundary.  Phases:
  * 0 momentum/normalise, 1 Gram (X X^T), 2 polynomial (b A + c A^2),
- * 3 X update (a X + B X, includes the fused weight update of the last
- * iteration), 4 stand-alone update and RMS finalisation. */
+ * 3 X update (a X + B X), 4 the update pass over the last iterate (weight
+ * update or O output), the Eq. 6 reduction and the RMS finalisation. */
 #define MUON_NUM_PHASES 5
 MUON_API muon_status_t muon_profile_enable(muon_plan_t plan, int32_t enable);
 

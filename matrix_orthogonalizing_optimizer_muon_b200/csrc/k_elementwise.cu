@@ -19,7 +19,7 @@
 // update_norm: RMS(O) per matrix and the Eq. 6 factor rms_scale / RMS(O)
 //     (Sec. 3.1, "Update Norm"), chunk partials in fp64 reduced in chunk
 //     order by the last CTA of each matrix.
-// rms_finalize: sqrt(mean(O^2)) per matrix from per-tile partial sums
+// rms_finalize: sqrt(mean(O^2)) per matrix from the update pass's per-chunk partial sums
 //     (Sec. 2.3, Algorithm 1, returned value).
 #include "muon_internal.cuh"
 

@@ -3,14 +3,16 @@
 // muon_init turns the list of parameter shapes into a plan: one device
 // allocation that holds the Newton-Schulz workspace, the per-matrix
 // descriptors, the tile schedules of every GEMM phase, the chunk schedule of
-// the elementwise kernels and one TMA descriptor per operand buffer.  A step
-// is then a fixed sequence of launches on the caller's stream:
+// the elementwise kernels and the TMA descriptors of every buffer.  A step is
+// then a fixed sequence of launches on the caller's stream:
 //   k1 (momentum, Nesterov input, Frobenius norm, bf16 split)
-//   N x [Gram, polynomial, X update]   (tensor cores; the last X update
-//                                       applies the weight update)
+//   N x [Gram, polynomial, X update]   (tensor cores)
+//   [Eq. 6 only: RMS(O) reduction]
+//   the update pass (weight update, or O for muon_orthogonalize)
 //   optional update-RMS finalisation.
-// No host synchronisation happens in muon_step; per-call device pointers are
-// uploaded only when they differ from the previous call's.
+// muon_step does not wait for the device except, rarely, to reuse the pinned
+// staging of a pointer table; per-call device pointer tables are kept on the
+// device (a few of them) and uploaded only when a call brings a new one.
 #include "muon.h"
 #include "muon_internal.cuh"
 

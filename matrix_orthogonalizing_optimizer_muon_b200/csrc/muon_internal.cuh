@@ -61,7 +61,8 @@ constexpr uint32_t kStatusNonFinite = 2u;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 enum Phase : int { kPhaseGram = 0, kPhasePoly = 1, kPhaseUpdate = 2 };
-enum FinalMode : int { kFinalNone = 0, kFinalWeight = 1, kFinalOut = 2 };
+// what the update pass writes: the weight update (muon_step) or O itself (muon_orthogonalize)
+enum FinalMode : int { kFinalWeight = 1, kFinalOut = 2 };
 enum K1Mode : int { kK1Momentum = 0, kK1Copy = 1 };
 // scaling of the update O (Sec. 3.1): Eq. 4, Eq. 5, Eq. 6
 enum ScaleMode : int { kScaleMaxDim = 0, kScaleHidden = 1, kScaleUpdateNorm = 2 };
