@@ -188,3 +188,22 @@ def test_step_replays_from_a_cuda_graph():
     del graph
     plan.close()
     eager.close()
+
+
+def test_zero_input_after_nonzero_gives_exact_zero_output():
+    # the Newton-Schulz launches skip a zero matrix, so its iterate buffers
+    # still hold the previous call's matrix; O must nevertheless be exactly 0
+    plan = MuonPlan(SHAPES)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(31)
+    xs = [torch.randn(s, device="cuda", generator=g).to(torch.bfloat16) for s in SHAPES]
+    outs = [torch.empty(s, device="cuda") for s in SHAPES]
+    plan.orthogonalize(xs, outs, ns_steps=5, coeffs=ABC32)
+    torch.cuda.synchronize()
+    assert all(bool(o.abs().max() > 0) for o in outs)
+    for x in xs:
+        x.zero_()
+    plan.orthogonalize(xs, outs, ns_steps=5, coeffs=ABC32)
+    torch.cuda.synchronize()
+    assert all(torch.equal(o, torch.zeros_like(o)) for o in outs)
+    plan.close()

@@ -90,3 +90,17 @@ def test_limits_and_argument_errors():
     assert lib.muon_orthogonalize_noalloc(xp, op, 0, 4, 0, 5, abc, s) == L.MUON_ERR_INVALID_ARG
     assert lib.muon_orthogonalize_noalloc(xp, op, 4, 4, 7, 5, abc, s) == L.MUON_ERR_INVALID_ARG
     assert lib.muon_orthogonalize_noalloc(xp, xp, 4, 4, 0, 5, abc, s) == L.MUON_ERR_ALIAS
+
+
+def test_zero_input_after_nonzero_gives_exact_zero_output():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    x = torch.randn(300, 520, device="cuda", generator=g).to(torch.bfloat16)
+    o = torch.empty(x.shape, device="cuda")
+    noalloc(x, o)
+    torch.cuda.synchronize()
+    assert bool(o.abs().max() > 0)
+    x.zero_()
+    noalloc(x, o)
+    torch.cuda.synchronize()
+    assert torch.equal(o, torch.zeros_like(o))
