@@ -18,11 +18,11 @@
 // stage takes about two stage-times of MMA to arrive), so the ring is as deep
 // as shared memory allows: 6 stages for the Gram and polynomial phases, 4 for
 // the X update, whose epilogue also stages its hi/lo inputs.  Per CTA:
-//   warps 0, 10 TMA producers for the even and the odd stages: up to four
-//               lanes issue one box each per stage in a single instruction
-//               (a 64 x 128 K-major box, or 64 x 64 boxes for MN-major
-//               operands and narrow K-major ones); both CTAs' loads complete
-//               on the leader's "full" barrier.
+//   warps 0, 10 TMA producers taking alternate stage fills: up to four lanes
+//               issue one box each per stage in a single instruction (a
+//               64 x 128 K-major box, or 64 x 64 boxes for MN-major operands
+//               and narrow K-major ones); both CTAs' loads complete on the
+//               leader's "full" barrier.
 //   warp 1      TMEM allocator (both CTAs) and MMA issuer (leader only); two
 //               256-column accumulators so the epilogue of one tile overlaps
 //               the main loop of the next.
@@ -61,10 +61,14 @@ constexpr int kEpiBlockBytes = 32 * 32 * 2;               // 2 KiB
 constexpr int kEpiWarpBytes = 2 * kEpiBlockBytes;         // 4 KiB
 constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;      // 32 KiB
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
-constexpr int kWarpProducer2 = kWarpEpi0 + kEpiWarps;  // second producer warp (odd stages)
-constexpr int kThreads = 32 * (kWarpProducer2 + 1);
-static_assert(MUON_TC_STAGES_SYM % 2 == 0 && MUON_TC_STAGES_UPD % 2 == 0,
-              "the two producer warps own the even and the odd stages");
+// Producer warps: warp 0 and the warps after the epilogue; fill f of the
+// stage ring goes to producer f mod kProducers.
+#ifndef MUON_TC_PRODUCERS
+#define MUON_TC_PRODUCERS 2
+#endif
+constexpr int kProducers = MUON_TC_PRODUCERS;
+constexpr int kWarpProducer2 = kWarpEpi0 + kEpiWarps;  // first of the extra producer warps
+constexpr int kThreads = 32 * (kWarpProducer2 + kProducers - 1);
 
 // X-update inputs: per warp a ring of 2 buffers, each a 32 x 32 hi block and
 // lo block (4 KiB), filled by cp.async two chunks ahead.
@@ -471,13 +475,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   unsigned* status = g.ws.status;
 
-  if (warp == kWarpProducer || warp == kWarpProducer2) {
+  if (warp == kWarpProducer || warp >= kWarpProducer2) {
     // ------------------------------------------------------------ TMA producers (both CTAs)
-    // Two warps take alternate stages, so two stage fills are being issued at
-    // any time (one thread issues about one TMA instruction per few hundred
-    // ns).  Within a warp, lane l < nbox_a loads A box l and the next lanes the
+    // The producer warps take the fills in turn, so several stage fills are
+    // being issued at any time (one thread issues about one TMA instruction
+    // per few hundred ns; a second warp measured about 2% faster, a third
+    // no better).  Within a warp, lane l < nbox_a loads A box l and the next lanes the
     // B boxes, all in one instruction; lane 0 owns the barriers.
-    const int pp = (warp == kWarpProducer) ? 0 : 1;
+    const int pp = (warp == kWarpProducer) ? 0 : warp - kWarpProducer2 + 1;
     long fills = 0;  // fills of both producers, in order
     for (int t = pair; t < g.ntiles; t += npairs) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
@@ -491,7 +496,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 1) prefetch_tensormap(c.b.tmap);
       bool ok = true;
       for (int kb = 0; kb < c.nk; ++kb, ++fills) {
-        if ((fills & 1) != pp) continue;
+        if (fills % kProducers != pp) continue;
         const int stage = static_cast<int>(fills % nst);
         const uint32_t phase = static_cast<uint32_t>((fills / nst) & 1);
         int ready = 0;
@@ -521,12 +526,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) break;
     }
     // Drain (leader): both CTAs' loads complete on the leader's barriers,
-    // so the most recent fill of each of this warp's stages must have landed
-    // before exit.
+    // so each of this warp's fills among the last nst (the latest of its
+    // stage) must have landed before exit.
     if (leader && lane == 0) {
-      for (int s = pp; s < nst; s += 2) {
-        const long cnt = fills / nst + ((s < fills % nst) ? 1 : 0);
-        if (cnt > 0 && !wait_bounded(full_bar(s), static_cast<uint32_t>((cnt - 1) & 1), nullptr))
+      for (long f = fills > nst ? fills - nst : 0; f < fills; ++f) {
+        if (f % kProducers != pp) continue;
+        if (!wait_bounded(full_bar(static_cast<int>(f % nst)), static_cast<uint32_t>((f / nst) & 1), nullptr))
           atomicOr(status, kStatusTimeout);
       }
     }
