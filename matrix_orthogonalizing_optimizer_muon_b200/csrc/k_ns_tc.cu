@@ -479,11 +479,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producers (both CTAs)
     // The producer warps take the fills in turn, so several stage fills are
     // being issued at any time (one thread issues about one TMA instruction
-    // per few hundred ns; a second warp measured about 2% faster, a third
-    // no better).  Within a warp, lane l < nbox_a loads A box l and the next lanes the
-    // B boxes, all in one instruction; lane 0 owns the barriers.
+    // per few hundred ns; a second warp measured about 2% faster, a third no
+    // better).  Within a warp, lane l < nbox_a loads A box l and the next
+    // lanes the B boxes, all in one instruction; lane 0 owns the barriers.
     const int pp = (warp == kWarpProducer) ? 0 : warp - kWarpProducer2 + 1;
-    long fills = 0;  // fills of both producers, in order
+    long fills = 0;  // fills of all producers, in order
     for (int t = pair; t < g.ntiles; t += npairs) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
       const TileCfg c = decode_tile(g, t);
