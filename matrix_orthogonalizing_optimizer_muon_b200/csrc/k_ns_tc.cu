@@ -641,9 +641,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int ld_in = upd ? mi.ld : mi.lda;
       const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
       const bool poly = (g.phase == kPhasePoly);
-      // a chunk needs work unless it is a block strictly above the diagonal
-      // of a symmetric output (its mirror writes it)
-      auto needed = [&](int ch) { return !(sym && (c.col0 + ch * kEpiBoxCols > i_lo + 31)); };
+      // A chunk needs work unless it is a block strictly above the diagonal
+      // of a symmetric output that the mirror of a lower block writes.  A
+      // transposed tile (col0 > row0) lies wholly above the diagonal and
+      // writes every block with its mirror.
+      const int j_lim = (sym && c.col0 <= c.row0) ? i_lo + 31 : INT_MAX;
+      auto needed = [&](int ch) { return c.col0 + ch * kEpiBoxCols <= j_lim; };
       auto block_inside = [&](int ch) {
         return i_lo + 31 < rows_in && c.col0 + ch * kEpiBoxCols + 32 <= cols_in;
       };
@@ -742,8 +745,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __align__(16) __nv_bfloat16 h[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
-          if (inside && j0 + 31 < i_lo) {
-            // strictly lower block: stage it and its transpose, store both
+          const bool above = j0 > i_lo + 31;  // only in a transposed tile
+          if (inside && (above || j0 + 31 < i_lo)) {
+            // off-diagonal block: stage it and its transpose, store both
             staging_free();
             write_row32(blk0, lane, h);
 #pragma unroll
@@ -758,8 +762,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 32; ++q) {
               const int j = j0 + q;
               if (i < mi.m && j < mi.m) {
-                if (j <= i) row[j] = h[q];
-                if (j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
+                if (above || j <= i) row[j] = h[q];
+                if (above || j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
               }
             }
           }

@@ -431,11 +431,7 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   }
   for (int i : order) {
     const MatInfo& mi = pl->mats[i];
-    for (int r0 = 0; r0 < mi.m; r0 += kTileM)
-      for (int c0 = 0; c0 < mi.m && c0 <= r0 + kTileM - 1; c0 += kBN) {
-        const int need = std::min({kBN, mi.m - c0, r0 + kTileM - c0});
-        sym.push_back(make_int4(i, r0, c0, need));
-      }
+    for_each_sym_tile(mi.m, [&](int r0, int c0, int need) { sym.push_back(make_int4(i, r0, c0, need)); });
     for (int r0 = 0; r0 < mi.rows; r0 += kTileM)
       for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
     if (pl->fp32_ws) {

@@ -91,9 +91,27 @@ struct MatPtrs {
 };
 
 // Tile of a GEMM phase: .x matrix, .y row0, .z col0, .w n_need (columns that
-// hold useful output, <= kBN).  Symmetric phases list only tiles that touch
-// the lower triangle.
+// hold useful output, <= kBN).  Symmetric phases list each tile of the lower
+// triangle once; see for_each_sym_tile.
 using TileDesc = int4;
+
+// Tiles of a symmetric m x m product (X X^T, A A) on the kTileM x kBN grid,
+// lower triangle only.  A ragged last row block (fewer than kTileM rows)
+// would leave part of every M = 256 tile in its row empty, so its
+// off-diagonal tiles are listed transposed: rows of the full block c0 and
+// columns of the ragged block.  col0 > row0 marks such a tile; every 32 x 32
+// block of it lies above the diagonal and is stored with its mirror.
+template <class F>
+inline void for_each_sym_tile(int m, F&& emit) {
+  static_assert(kTileM == kBN, "square tile grid");
+  for (int r0 = 0; r0 < m; r0 += kTileM) {
+    const int rv = m - r0 < kTileM ? m - r0 : kTileM;
+    for (int c0 = 0; c0 <= r0; c0 += kBN) {
+      if (c0 < r0 && rv < kTileM) emit(c0, r0, rv);
+      else emit(r0, c0, m - c0 < kBN ? m - c0 : kBN);
+    }
+  }
+}
 
 // Momentum/normalise chunk: .x matrix, .y first row, .z number of rows, .w slot
 using ChunkDesc = int4;

@@ -135,11 +135,12 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   mi.nchunks = nch;
   TileDesc sym[kNaMaxTiles], full[kNaMaxTiles];
   int nsym = 0, nfull = 0;
-  for (int r0 = 0; r0 < mi.m; r0 += kTileM)
-    for (int c0 = 0; c0 < mi.m && c0 <= r0 + kTileM - 1; c0 += kBN) {
-      if (nsym == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
-      sym[nsym++] = make_int4(0, r0, c0, std::min({kBN, mi.m - c0, r0 + kTileM - c0}));
-    }
+  bool sym_fits = true;
+  for_each_sym_tile(mi.m, [&](int r0, int c0, int need) {
+    if (nsym == kNaMaxTiles) sym_fits = false;
+    else sym[nsym++] = make_int4(0, r0, c0, need);
+  });
+  if (!sym_fits) return MUON_ERR_UNSUPPORTED;
   for (int r0 = 0; r0 < R; r0 += kTileM)
     for (int c0 = 0; c0 < C; c0 += kBN) {
       if (nfull == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
