@@ -185,6 +185,53 @@ def bench_adamw(dev, steps: int = 20, warmup: int = 3):
             "peak_source": f"hbm_gbs ({kind})", "frac": gbs / peak, "bytes_per_elem": ADAMW_BYTES_PER_ELEM}
 
 
+# fp64 CUDA-core peak, derived: 148 SMs x 64 FP64 FMA per clock x 2 FLOP x 1.965 GHz
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+
+
+def entropy_update_flops(shapes, sweeps) -> float:
+    """FLOPs of jacobi_update_kernel over a call: per matrix and sweep, nb - 1
+    rounds of (nb/2)(nb/2 + 1)/2 super-blocks, each two 64 x 64 x 64 products."""
+    total = 0.0
+    for (r, c), sw in zip(shapes, sweeps):
+        nb = -(-min(r, c) // 32)
+        nb += nb % 2
+        pairs = nb // 2
+        total += sw * (nb - 1) * pairs * (pairs + 1) / 2 * 4 * 64 ** 3
+    return total
+
+
+def bench_entropy(Ws, calls: int = 2):
+    """Time the SVD-entropy diagnostic (Sec. 3.4) on the workload's weight
+    matrices; returns the bench line's `svd_entropy` object."""
+    import torch
+    from matrix_orthogonalizing_optimizer_muon_b200.api import EntropyPlan
+    shapes = [tuple(W.shape) for W in Ws]
+    plan = EntropyPlan(shapes)
+    H = plan.compute(Ws)  # warm-up
+    torch.cuda.synchronize()
+    plan.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        plan.compute(Ws, H=H)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / calls
+    phases = plan.profile_read()
+    st, sweeps = plan.status()
+    plan.close()
+    flops = entropy_update_flops(shapes, sweeps)
+    achieved = flops / (phases["jacobi"] * 1e-3) / 1e12
+    return {"what": "SVD entropy (Sec. 3.4) of every weight matrix after the timed steps: fp64 Gram, "
+                    "two-sided block Jacobi, entropy; one call covers all matrices",
+            "matrices": len(Ws), "ms_per_call": ms, "phases_ms": phases, "status": st,
+            "sweeps": [min(sweeps), max(sweeps)], "kernel": "jacobi_update_kernel (fp64 CUDA cores)",
+            "bound": "alu", "achieved": achieved, "unit": "TFLOP/s (fp64)", "peak": FP64_PEAK_TFLOPS,
+            "peak_source": "derived: 148 SMs x 64 FP64 FMA/clk x 2 x 1.965 GHz", "frac": achieved / FP64_PEAK_TFLOPS,
+            "achieved_basis": "update-kernel FLOPs over the whole Jacobi phase (solves and checks included)"}
+
+
 # ---------------------------------------------------------------------- oracle (CPU) legs
 
 def cpu_sample(wl, budget_s: float, seed: int = 0):
@@ -304,6 +351,7 @@ def main(argv=None) -> int:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the PyTorch eager comparison point")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW companion measurement")
+    ap.add_argument("--no-entropy", action="store_true", help="skip the SVD-entropy diagnostic measurement")
     ap.add_argument("--scale", default="max_dim", choices=["max_dim", "hidden", "update_norm"],
                     help="update scale of Sec. 3.1: Eq. 4 (default), Eq. 5 with H = 2048, Eq. 6")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -475,6 +523,10 @@ def main(argv=None) -> int:
                    "ns_ms_per_step": t_eager, "tflops_algorithmic": nz_flops / (t_eager * 1e-3) / 1e12,
                    "tflops_dense_equivalent": dense_flops / (t_eager * 1e-3) / 1e12}
 
+    entropy = None
+    if not args.no_entropy:
+        entropy = bench_entropy(Ws)
+
     adamw = None
     if not args.no_adamw:
         plan.close()
@@ -518,6 +570,7 @@ def main(argv=None) -> int:
         "cpu_baseline": cpu,
         "context_torch_eager_ns": context,
         "adamw_companion": adamw,
+        "svd_entropy": entropy,
         "e2e": e2e,
         "gpu_launches": int(round(per_step_launches * args.steps)),
         "clocks": clk.summary(),

@@ -49,7 +49,8 @@ typedef enum {
   MUON_ERR_CUDA = 5,           /* a CUDA call or launch failed */
   MUON_ERR_NONFINITE = 6,      /* (muon_get_status) a Frobenius norm was NaN or Inf */
   MUON_ERR_TIMEOUT = 7,        /* (muon_get_status) a device-side wait gave up; results of that call are invalid */
-  MUON_ERR_ALIAS = 8           /* W, G, M (or X_in, O_out) buffers overlap */
+  MUON_ERR_ALIAS = 8,          /* W, G, M (or X_in, O_out) buffers overlap */
+  MUON_ERR_NOT_CONVERGED = 9   /* (muon_entropy_get_status) an eigenvalue iteration hit its sweep limit */
 } muon_status_t;
 
 typedef enum { MUON_DT_BF16 = 0, MUON_DT_FP32 = 1 } muon_dtype_t;
@@ -255,6 +256,62 @@ MUON_API muon_status_t muon_adamw_step(muon_adamw_plan_t plan, const muon_adamw_
 
 /* Waits for the plan's last stream and frees it; NULL is ignored. */
 MUON_API void muon_adamw_destroy(muon_adamw_plan_t plan);
+
+/* ------------------------------------------------------------------------
+ * SVD-entropy diagnostic ("Muon is Scalable for LLM Training", Sec. 3.4,
+ * the SVD-entropy equation and Fig. 4).  For a weight matrix with singular
+ * values sigma_1 .. sigma_n, n = min(rows, cols):
+ *   H = -(1 / log n) sum_i p_i log p_i,   p_i = sigma_i^2 / sum_j sigma_j^2
+ * with 0 log 0 = 0.  H is NaN for a zero matrix, for n = 1 (both 0 / 0) and
+ * for a matrix with non-finite entries.
+ * sigma_i^2 are the eigenvalues of the fp32 Gram matrix of the wide
+ * orientation, found by two-sided block Jacobi in fp64 (32-row blocks, at
+ * most 24 sweeps, stopped once the off-diagonal Frobenius norm is below 1e-8
+ * of the whole); the entropy sums run in fp64 too.
+ * ------------------------------------------------------------------------ */
+typedef struct muon_entropy_plan_s* muon_entropy_plan_t;
+
+/* Plan for n >= 1 fp32 matrices: shapes[2 i] = rows, shapes[2 i + 1] = cols,
+ * each >= 1 with rows * cols < 2^31.  min(rows, cols) <= 8192, else
+ * MUON_ERR_UNSUPPORTED.  Allocates the fp64 Gram workspace (about 8 m^2 bytes
+ * per matrix, m = min(rows, cols)) and the rotation store.  Errors:
+ * INVALID_ARG, UNSUPPORTED, NO_MEMORY, CUDA. */
+MUON_API muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64_t* shapes, int32_t n, void* stream);
+
+/* Entropy of every planned matrix, asynchronous on `stream`.
+ * W[i]: device pointer to matrix i, fp32 row-major [rows, cols], read only
+ *   (W is a host array of n device pointers).
+ * H_out: device fp32 [n], H of each matrix.
+ * sigma_out: NULL, or device fp32 [muon_entropy_num_singular_values(plan)]:
+ *   the singular values of matrix i, descending, follow those of matrices
+ *   0 .. i-1.
+ * The outputs must not overlap the inputs or each other.  Everything is
+ * validated before anything is enqueued: INVALID_ARG, SHAPE_MISMATCH,
+ * ALIAS; launch failures give MUON_ERR_CUDA.  Results are bitwise
+ * reproducible. */
+MUON_API muon_status_t muon_entropy_compute(muon_entropy_plan_t plan, const float* const* W, int32_t n, float* H_out,
+                                            float* sigma_out, void* stream);
+
+/* Total number of singular values of the plan (sum of min(rows, cols)); -1 for NULL. */
+MUON_API int64_t muon_entropy_num_singular_values(muon_entropy_plan_t plan);
+
+/* Synchronises the plan's last stream, then returns and clears the sticky
+ * status of the calls since the previous read: MUON_OK, MUON_ERR_NONFINITE
+ * (a matrix had non-finite entries; its H is NaN) or MUON_ERR_NOT_CONVERGED
+ * (a matrix used all 24 sweeps; its H comes from the last iterate).
+ * sweeps_out: NULL or a host int32 array [n] that receives, for the last
+ * call, the sweeps each matrix needed (0: not converged or non-finite).
+ * CUDA errors: MUON_ERR_CUDA. */
+MUON_API muon_status_t muon_entropy_get_status(muon_entropy_plan_t plan, int32_t* sweeps_out);
+
+/* Per-phase timing of the next calls with CUDA events when enable != 0.
+ * ms_out: NULL, or a host double array [3] that receives the Gram, Jacobi
+ * and entropy phase times of the last profiled call (waits for its events;
+ * MUON_ERR_INVALID_ARG if no call was profiled). */
+MUON_API muon_status_t muon_entropy_profile(muon_entropy_plan_t plan, int32_t enable, double* ms_out);
+
+/* Waits for the plan's last stream and frees it; NULL is ignored. */
+MUON_API void muon_entropy_destroy(muon_entropy_plan_t plan);
 
 #ifdef __cplusplus
 }

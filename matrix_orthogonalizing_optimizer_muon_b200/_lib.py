@@ -22,6 +22,7 @@ MUON_ERR_CUDA = 5
 MUON_ERR_NONFINITE = 6
 MUON_ERR_TIMEOUT = 7
 MUON_ERR_ALIAS = 8
+MUON_ERR_NOT_CONVERGED = 9
 
 MUON_DT_BF16 = 0
 MUON_DT_FP32 = 1
@@ -36,7 +37,8 @@ PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
 EXPORTED = ("muon_hparams_default", "muon_init", "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
             "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read",
             "muon_orthogonalize_noalloc", "muon_adamw_hparams_default", "muon_adamw_init", "muon_adamw_step",
-            "muon_adamw_destroy")
+            "muon_adamw_destroy", "muon_entropy_init", "muon_entropy_compute", "muon_entropy_num_singular_values",
+            "muon_entropy_get_status", "muon_entropy_profile", "muon_entropy_destroy")
 
 
 class muon_param_t(ctypes.Structure):
@@ -116,6 +118,18 @@ def load() -> ctypes.CDLL:
     lib.muon_adamw_step.restype = ctypes.c_int
     lib.muon_adamw_destroy.argtypes = [P]
     lib.muon_adamw_destroy.restype = None
+    lib.muon_entropy_init.argtypes = [ctypes.POINTER(P), ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, P]
+    lib.muon_entropy_init.restype = ctypes.c_int
+    lib.muon_entropy_compute.argtypes = [P, ctypes.POINTER(P), ctypes.c_int32, P, P, P]
+    lib.muon_entropy_compute.restype = ctypes.c_int
+    lib.muon_entropy_num_singular_values.argtypes = [P]
+    lib.muon_entropy_num_singular_values.restype = ctypes.c_int64
+    lib.muon_entropy_get_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+    lib.muon_entropy_get_status.restype = ctypes.c_int
+    lib.muon_entropy_profile.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]
+    lib.muon_entropy_profile.restype = ctypes.c_int
+    lib.muon_entropy_destroy.argtypes = [P]
+    lib.muon_entropy_destroy.restype = None
     _lib = lib
     return lib
 
@@ -206,3 +220,37 @@ def muon_adamw_step(plan, params, n: int, hp: muon_adamw_hparams_t, stream: int)
 
 def muon_adamw_destroy(plan) -> None:
     load().muon_adamw_destroy(plan)
+
+
+def muon_entropy_init(shapes, stream: int) -> ctypes.c_void_p:
+    flat = (ctypes.c_int64 * (2 * len(shapes)))(*[int(v) for s in shapes for v in s])
+    plan = ctypes.c_void_p()
+    check(load().muon_entropy_init(ctypes.byref(plan), flat, len(shapes), ctypes.c_void_p(stream)),
+          "muon_entropy_init")
+    return plan
+
+
+def muon_entropy_compute(plan, w_ptrs, n: int, h_ptr: int, sigma_ptr: int | None, stream: int) -> None:
+    check(load().muon_entropy_compute(plan, w_ptrs, int(n), ctypes.c_void_p(h_ptr), ctypes.c_void_p(sigma_ptr or 0),
+                                      ctypes.c_void_p(stream)), "muon_entropy_compute")
+
+
+def muon_entropy_num_singular_values(plan) -> int:
+    return int(load().muon_entropy_num_singular_values(plan))
+
+
+def muon_entropy_get_status(plan, n: int):
+    """(status code, sweeps per matrix) -- synchronising read-and-clear."""
+    sweeps = (ctypes.c_int32 * n)()
+    st = int(load().muon_entropy_get_status(plan, sweeps))
+    return st, list(sweeps)
+
+
+def muon_entropy_profile(plan, enable: bool, read: bool = False):
+    ms = (ctypes.c_double * 3)()
+    check(load().muon_entropy_profile(plan, 1 if enable else 0, ms if read else None), "muon_entropy_profile")
+    return list(ms) if read else None
+
+
+def muon_entropy_destroy(plan) -> None:
+    load().muon_entropy_destroy(plan)

@@ -13,6 +13,12 @@ step for them.
 
     adam = AdamWPlan([g.numel() for g in gains], states=[(m, v) ...])
     adam.step(list(zip(gains, grads, ms, vs)), step=t, lr=4.2e-4, weight_decay=0.1)
+
+Sec. 3.4 compares optimisers by the SVD entropy of the weight matrices;
+``EntropyPlan`` computes it on the GPU.
+
+    ent = EntropyPlan([W.shape for W in weights])
+    H = ent.compute(weights)            # fp32 [n] on the device
 """
 
 from __future__ import annotations
@@ -222,6 +228,63 @@ class AdamWPlan:
     def close(self) -> None:
         if getattr(self, "_plan", None):
             L.muon_adamw_destroy(self._plan)
+            self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class EntropyPlan:
+    """A libmuon SVD-entropy plan for a fixed list of fp32 matrix shapes on the
+    current device (Sec. 3.4): H = -(1/log n) sum p_i log p_i with
+    p_i = sigma_i^2 / sum sigma_j^2 over the n = min(rows, cols) singular values."""
+
+    _PHASES = ("gram", "jacobi", "entropy")
+
+    def __init__(self, shapes, *, stream=None):
+        self.shapes = [tuple(int(v) for v in s) for s in shapes]
+        if any(len(s) != 2 for s in self.shapes):
+            raise ValueError("entropy plans take 2-D shapes only")
+        self.n = len(self.shapes)
+        self._plan = L.muon_entropy_init(self.shapes, _stream_handle(stream))
+        self.num_singular_values = L.muon_entropy_num_singular_values(self._plan)
+        self._w = (ctypes.c_void_p * self.n)()
+
+    def compute(self, weights, H=None, sigma=None, *, stream=None) -> torch.Tensor:
+        """Entropy of each matrix into H (fp32 [n] on the device, allocated if
+        None).  sigma, if given (fp32 [num_singular_values]), receives each
+        matrix's singular values, descending, matrix after matrix."""
+        if len(weights) != self.n:
+            raise ValueError(f"expected {self.n} matrices, got {len(weights)}")
+        for i, W in enumerate(weights):
+            _check_tensor(W, torch.float32, f"W[{i}]", self.shapes[i])
+            self._w[i] = W.data_ptr()
+        if H is None:
+            H = torch.empty(self.n, dtype=torch.float32, device=weights[0].device)
+        _check_tensor(H, torch.float32, "H", (self.n,))
+        sp = None
+        if sigma is not None:
+            _check_tensor(sigma, torch.float32, "sigma", (self.num_singular_values,))
+            sp = sigma.data_ptr()
+        L.muon_entropy_compute(self._plan, self._w, self.n, H.data_ptr(), sp, _stream_handle(stream))
+        return H
+
+    def status(self):
+        """(status code, sweeps per matrix of the last call); synchronising."""
+        return L.muon_entropy_get_status(self._plan, self.n)
+
+    def profile(self, enable: bool = True) -> None:
+        L.muon_entropy_profile(self._plan, enable)
+
+    def profile_read(self) -> dict:
+        return dict(zip(self._PHASES, L.muon_entropy_profile(self._plan, True, read=True)))
+
+    def close(self) -> None:
+        if getattr(self, "_plan", None):
+            L.muon_entropy_destroy(self._plan)
             self._plan = None
 
     def __del__(self):

@@ -340,6 +340,7 @@ const char* muon_status_string(muon_status_t s) {
     case MUON_ERR_NONFINITE: return "non-finite Frobenius norm";
     case MUON_ERR_TIMEOUT: return "device-side wait timed out";
     case MUON_ERR_ALIAS: return "buffers overlap";
+    case MUON_ERR_NOT_CONVERGED: return "eigenvalue iteration did not converge";
   }
   return "unknown status";
 }

@@ -46,8 +46,8 @@ def test_no_other_exported_functions(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 9):
-        assert L.status_string(code)
+    for code in range(0, 10):
+        assert L.status_string(code) != "unknown status"
     assert L.status_string(0) == "ok"
     assert L.status_string(123) == "unknown status"
 
@@ -109,6 +109,25 @@ def test_null_plan_calls(lib):
     abc = (ctypes.c_float * 3)(1, 0, 0)
     assert lib.muon_orthogonalize(None, None, None, 1, 0, 5, abc, 0, None) == L.MUON_ERR_INVALID_ARG
     assert lib.muon_profile_enable(None, 1) == L.MUON_ERR_INVALID_ARG
+
+
+def test_entropy_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
+    plan = ctypes.c_void_p()
+    shapes = (ctypes.c_int64 * 4)(16, 24, 8, 8)
+    assert lib.muon_entropy_init(None, shapes, 2, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_entropy_init(ctypes.byref(plan), None, 2, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_entropy_init(ctypes.byref(plan), shapes, 0, None) == L.MUON_ERR_INVALID_ARG
+    for bad in ((0, 5), (5, 0), (-1, 4), (1 << 20, 1 << 12)):
+        arr = (ctypes.c_int64 * 2)(*bad)
+        assert lib.muon_entropy_init(ctypes.byref(plan), arr, 1, None) == L.MUON_ERR_INVALID_ARG, bad
+    big = (ctypes.c_int64 * 2)(8193, 8200)
+    assert lib.muon_entropy_init(ctypes.byref(plan), big, 1, None) == L.MUON_ERR_UNSUPPORTED
+    assert plan.value is None
+    assert lib.muon_entropy_compute(None, None, 1, None, None, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_entropy_get_status(None, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_entropy_profile(None, 1, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_entropy_num_singular_values(None) == -1
+    lib.muon_entropy_destroy(None)
 
 
 def test_build_flags_target_sm100a():

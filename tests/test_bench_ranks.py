@@ -84,3 +84,13 @@ def test_reference_arm_line_on_rank_zero(monkeypatch):
               "vs_baseline", "dtype", "data", "config"):
         assert k in line
     assert "workload" in line["config"]
+
+
+def test_entropy_update_flop_count():
+    # (64, 64): nb = 2 blocks, one round of one super-block per sweep, two 64^3 products
+    assert bench.entropy_update_flops([(64, 64)], [3]) == 3 * 4 * 64 ** 3
+    # min(1408, 2048) = 1408: 44 blocks, 43 rounds of 22 * 23 / 2 super-blocks
+    assert bench.entropy_update_flops([(2048, 1408)], [1]) == 43 * 253 * 4 * 64 ** 3
+    # 33 rows round up to 2 blocks; a matrix that took no sweep adds nothing
+    assert bench.entropy_update_flops([(33, 70), (500, 9)], [2, 0]) == 2 * 4 * 64 ** 3
+    assert abs(bench.FP64_PEAK_TFLOPS - 37.23) < 0.01
