@@ -215,7 +215,10 @@ __device__ __forceinline__ void small_gemm(const double* A, const double* B, dou
 // 64 indices: 63 rounds of 32 disjoint rotations per sweep.  For a pair with
 // alpha = S_aa, beta = S_bb, gamma = S_ab the rotation J = [c s; -s c] zeroes
 // S_ab in J^T S J when t = s / c is the smaller root of t^2 + 2 tau t - 1 = 0,
-// tau = (beta - alpha) / (2 gamma) (the symmetric 2 x 2 Schur decomposition).
+// tau = (beta - alpha) / (2 gamma) (the symmetric 2 x 2 Schur decomposition);
+// with d = beta - alpha that root is t = 2 gamma sgn(d) / (|d| + sqrt(d^2 + 4 gamma^2)).
+// A round applies its rotations to the rows of S, then to the columns of S
+// and V; each warp works on one pair and 32 consecutive rows or columns.
 __global__ void __launch_bounds__(kEThreads) jacobi_solve_kernel(const int2* __restrict__ pairs, int npairs,
                                                                  const EntMat* __restrict__ mats, const double* __restrict__ G,
                                                                  double* __restrict__ Vst, const EntCtl ctl, int round) {
@@ -243,58 +246,45 @@ __global__ void __launch_bounds__(kEThreads) jacobi_solve_kernel(const int2* __r
     for (int sweep = 0; sweep < kInnerSweeps; ++sweep) {
       int rotated = 0;
       for (int rr = 0; rr < kEs - 1; ++rr) {
+        int rot = 0;
         if (t < kEb) {
           const int2 ab = tournament(kEs, rr, t);
           const double alpha = S[ab.x * kEsLd + ab.x], beta = S[ab.y * kEsLd + ab.y], gamma = S[ab.x * kEsLd + ab.y];
           double c = 1.0, s = 0.0;
           if (fabs(gamma) > kInnerTol * fmax(fabs(alpha), fabs(beta))) {
-            const double tau = (beta - alpha) / (2.0 * gamma);
-            const double tt = copysign(1.0, tau) / (fabs(tau) + sqrt(fma(tau, tau, 1.0)));
-            c = 1.0 / sqrt(fma(tt, tt, 1.0));
+            const double d = beta - alpha;
+            const double tt = (d >= 0.0 ? 2.0 * gamma : -2.0 * gamma) / (fabs(d) + sqrt(fma(d, d, 4.0 * gamma * gamma)));
+            c = rsqrt(fma(tt, tt, 1.0));
             s = tt * c;
-            rotated = 1;
+            rot = 1;
           }
           ra[t] = ab.x;
           rb[t] = ab.y;
           rc[t] = c;
           rs[t] = s;
         }
-        __syncthreads();
-        // S <- J^T S J one 2 x 2 block (rows of pair k1, columns of pair k2)
-        // at a time; blocks with k1 > k2 are the mirror of (k2, k1)
-        for (int e = t; e < kEb * kEb; e += kEThreads) {
-          const int k1 = e >> 5, k2 = e & 31;
-          if (k1 > k2) continue;
-          const double c1 = rc[k1], s1 = rs[k1], c2 = rc[k2], s2 = rs[k2];
-          if (s1 == 0.0 && s2 == 0.0) continue;
-          const int a1 = ra[k1], b1 = rb[k1], a2 = ra[k2], b2 = rb[k2];
-          const double m00 = S[a1 * kEsLd + a2], m01 = S[a1 * kEsLd + b2];
-          const double m10 = S[b1 * kEsLd + a2], m11 = S[b1 * kEsLd + b2];
-          const double n00 = m00 * c2 - m01 * s2, n01 = m00 * s2 + m01 * c2;
-          const double n10 = m10 * c2 - m11 * s2, n11 = m10 * s2 + m11 * c2;
-          const double o00 = c1 * n00 - s1 * n10, o01 = c1 * n01 - s1 * n11;
-          const double o10 = s1 * n00 + c1 * n10, o11 = s1 * n01 + c1 * n11;
-          S[a1 * kEsLd + a2] = o00;
-          S[b1 * kEsLd + b2] = o11;
-          if (k1 == k2) {
-            // the rotated pair's own block: exactly diagonal in exact arithmetic
-            S[a1 * kEsLd + b1] = 0.0;
-            S[b1 * kEsLd + a1] = 0.0;
-          } else {
-            S[a1 * kEsLd + b2] = o01;
-            S[b1 * kEsLd + a2] = o10;
-            S[a2 * kEsLd + a1] = o00;
-            S[b2 * kEsLd + a1] = o01;
-            S[a2 * kEsLd + b1] = o10;
-            S[b2 * kEsLd + b1] = o11;
-          }
-        }
-        // V <- V J
-        for (int e = t; e < kEs * kEb; e += kEThreads) {
-          const int i = e >> 5, k = e & 31;
+        if (!__syncthreads_or(rot)) continue;  // nothing to rotate in this round
+        rotated = 1;
+        // rows: S <- J^T S (pair k, column j; a warp takes one pair, 32 columns)
+        for (int e = t; e < kEb * kEs; e += kEThreads) {
+          const int k = e >> 6, j = e & 63;
           const double c = rc[k], s = rs[k];
           if (s == 0.0) continue;
           const int a = ra[k], b = rb[k];
+          const double sa = S[a * kEsLd + j], sb = S[b * kEsLd + j];
+          S[a * kEsLd + j] = c * sa - s * sb;
+          S[b * kEsLd + j] = s * sa + c * sb;
+        }
+        __syncthreads();
+        // columns: S <- S J and V <- V J (pair k, row i; a warp takes one pair, 32 rows)
+        for (int e = t; e < kEb * kEs; e += kEThreads) {
+          const int k = e >> 6, i = e & 63;
+          const double c = rc[k], s = rs[k];
+          if (s == 0.0) continue;
+          const int a = ra[k], b = rb[k];
+          const double sa = S[i * kEsLd + a], sb = S[i * kEsLd + b];
+          S[i * kEsLd + a] = c * sa - s * sb;
+          S[i * kEsLd + b] = s * sa + c * sb;
           const double va = V[i * kEsLd + a], vb = V[i * kEsLd + b];
           V[i * kEsLd + a] = c * va - s * vb;
           V[i * kEsLd + b] = s * va + c * vb;
