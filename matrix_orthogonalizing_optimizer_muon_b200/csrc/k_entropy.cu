@@ -14,12 +14,11 @@
 //      multiple of 64.  Products of fp32 entries are exact in fp64.
 //   2. Two-sided block Jacobi on G.  The 32-row blocks are paired by a
 //      round-robin tournament, nb - 1 rounds per sweep.  In a round, every
-//      pair's 64 x 64 subproblem [G_PP G_PQ; G_QP G_QQ] is diagonalised in
-//      shared memory by one sweep of cyclic Jacobi (jacobi_solve_kernel),
-//      which keeps the
+//      pair's 64 x 64 subproblem [G_PP G_PQ; G_QP G_QQ] gets one sweep of
+//      cyclic Jacobi in shared memory (jacobi_solve_kernel), which keeps the
 //      accumulated rotation V (re-orthonormalised by one polar Newton-Schulz
-//      step at the end); then G <- J^T G J for the block-diagonal J of
-//      all pairs, one 64 x 64 super-block per CTA iteration
+//      step at the end); then G <- J^T G J for the block-diagonal J of all
+//      pairs, one 64 x 64 super-block per CTA iteration
 //      (jacobi_update_kernel: two small GEMMs, V_u^T T V_v).
 //   3. After each sweep, off_norm_kernel and converge_kernel compare the
 //      off-diagonal Frobenius norm with ||G||_F (fp64, fixed order).  A
@@ -58,7 +57,7 @@ constexpr int kGramK = 32;
 constexpr int kMaxSweeps = 24;
 // One cyclic sweep per subproblem and round: solving the 64 x 64 problems to
 // convergence (up to 10 sweeps) saved at most one outer sweep in fp64
-// simulations of 704 x 704 Gram matrices (Gaussian: 11 against 10; four
+// simulations of 704 x 704 Gram matrices (Gaussian: 11 against 10; three
 // decades of singular values: 17 against 17) for five times the inner work.
 constexpr int kInnerSweeps = 1;
 constexpr int kMaxDim = 8192;        // min(rows, cols) limit (the sort stages 8192 values)
