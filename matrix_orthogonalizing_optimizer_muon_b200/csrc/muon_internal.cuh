@@ -15,6 +15,7 @@
 // X update is Y B, so every buffer keeps the parameter's layout.
 #pragma once
 
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>

@@ -1,0 +1,26 @@
+"""The symmetric-product tile enumerator of the tensor-core path, checked on
+the host: the real header function, compiled with g++ against
+csrc/muon_internal.cuh (no GPU).  See tests/host/sym_tiles_check.cpp for
+the properties."""
+
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CUDA_INC = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+
+
+@pytest.mark.skipif(shutil.which("g++") is None or not os.path.isdir(CUDA_INC), reason="needs g++ and CUDA headers")
+def test_sym_tile_list_covers_the_lower_triangle_once(tmp_path):
+    exe = tmp_path / "sym_tiles_check"
+    cmd = ["g++", "-std=c++17", "-O2", "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(ROOT, "matrix_orthogonalizing_optimizer_muon_b200", "csrc"), "-I", CUDA_INC,
+           os.path.join(ROOT, "tests", "host", "sym_tiles_check.cpp"), "-o", str(exe)]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stdout
+    # 1408 = 5 full row blocks + 128 rows: 15 + 5 transposed + 1 diagonal tiles
+    assert out.stdout.strip() == "ok 21"
