@@ -120,17 +120,6 @@ __global__ void __launch_bounds__(kAdamThreads) adamw_kernel(const AdamChunk* __
 
 bool is_finite(float x) { return std::isfinite(x); }
 
-struct Span {
-  uintptr_t lo, hi;
-};
-
-bool any_overlap(std::vector<Span>& v) {
-  std::sort(v.begin(), v.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
-  for (size_t i = 1; i < v.size(); ++i)
-    if (v[i].lo < v[i - 1].hi) return true;
-  return false;
-}
-
 }  // namespace
 }  // namespace muon
 
@@ -249,7 +238,7 @@ extern "C" muon_status_t muon_adamw_step(muon_adamw_plan_t pl, const muon_adamw_
       !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || hp->step < 1)
     return MUON_ERR_INVALID_ARG;
   std::vector<AdamPtrs> t(n);
-  std::vector<Span> spans;
+  std::vector<ByteRange> spans;
   spans.reserve(4 * static_cast<size_t>(n));
   for (int i = 0; i < n; ++i) {
     const muon_adamw_param_t& p = params[i];

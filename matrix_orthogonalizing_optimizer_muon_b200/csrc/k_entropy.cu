@@ -539,18 +539,6 @@ __global__ void __launch_bounds__(kSortThreads) entropy_kernel(const EntMat* __r
   for (int i = t; i < mi.m; i += kSortThreads) out[i] = sv[i];
 }
 
-// ---------------------------------------------------------------- host side
-struct Span {
-  uintptr_t lo, hi;
-};
-
-bool spans_overlap(std::vector<Span>& v) {
-  std::sort(v.begin(), v.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
-  for (size_t i = 1; i < v.size(); ++i)
-    if (v[i].lo < v[i - 1].hi) return true;
-  return false;
-}
-
 }  // namespace
 }  // namespace muon
 
@@ -729,7 +717,7 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
                                               float* sigma_out, void* stream) {
   if (pl == nullptr || W == nullptr || H_out == nullptr) return MUON_ERR_INVALID_ARG;
   if (n != pl->n) return MUON_ERR_SHAPE_MISMATCH;
-  std::vector<Span> spans;
+  std::vector<ByteRange> spans;
   spans.reserve(n + 2);
   std::vector<const float*> t(n);
   for (int i = 0; i < n; ++i) {
@@ -739,9 +727,9 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
     t[i] = W[i];
   }
   // the inputs may overlap one another (they are only read); the outputs may not touch them
-  std::sort(spans.begin(), spans.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
+  std::sort(spans.begin(), spans.end(), [](const ByteRange& a, const ByteRange& b) { return a.lo < b.lo; });
   auto hits_inputs = [&](uintptr_t lo, uintptr_t hi) {
-    for (const Span& s : spans)
+    for (const ByteRange& s : spans)
       if (lo < s.hi && s.lo < hi) return true;
     return false;
   };
@@ -752,8 +740,8 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
     const uintptr_t s = reinterpret_cast<uintptr_t>(sigma_out);
     if (s % sizeof(float) != 0) return MUON_ERR_INVALID_ARG;
     if (hits_inputs(s, s + pl->total_sv * sizeof(float))) return MUON_ERR_ALIAS;
-    std::vector<Span> outs{{h, h + n * sizeof(float)}, {s, s + pl->total_sv * sizeof(float)}};
-    if (spans_overlap(outs)) return MUON_ERR_ALIAS;
+    std::vector<ByteRange> outs{{h, h + n * sizeof(float)}, {s, s + pl->total_sv * sizeof(float)}};
+    if (any_overlap(outs)) return MUON_ERR_ALIAS;
   }
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != pl->device) return MUON_ERR_INVALID_ARG;

@@ -171,17 +171,6 @@ muon_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MUON_OK : MUO
 
 bool finite(float v) { return std::isfinite(v); }
 
-struct Interval {
-  uintptr_t lo, hi;
-};
-
-bool any_overlap(std::vector<Interval>& v) {
-  std::sort(v.begin(), v.end(), [](const Interval& a, const Interval& b) { return a.lo < b.lo; });
-  for (size_t i = 1; i < v.size(); ++i)
-    if (v[i].lo < v[i - 1].hi) return true;
-  return false;
-}
-
 // Make pl->ptrs_d a device table holding `t`: a kept table if one matches,
 // else the least recently used slot, refilled by an asynchronous copy on `st`
 // (stream order protects kernels of earlier calls still reading it).
@@ -584,7 +573,7 @@ muon_status_t muon_step(muon_plan_t pl, const muon_param_t* params, int32_t n, c
   if (hp->ns_precision != MUON_NS_BF16 && hp->ns_precision != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
   if (hp->ns_precision == MUON_NS_FP32 && !pl->fp32_ws) return MUON_ERR_UNSUPPORTED;
   std::vector<MatPtrs> t(n);
-  std::vector<Interval> iv;
+  std::vector<ByteRange> iv;
   iv.reserve(3 * static_cast<size_t>(n) + 1);
   for (int i = 0; i < n; ++i) {
     const muon_param_t& p = params[i];
@@ -631,7 +620,7 @@ muon_status_t muon_orthogonalize(muon_plan_t pl, const void* const* X_in, float*
   if (ns_precision != MUON_NS_BF16 && ns_precision != MUON_NS_FP32) return MUON_ERR_INVALID_ARG;
   if (ns_precision == MUON_NS_FP32 && !pl->fp32_ws) return MUON_ERR_UNSUPPORTED;
   std::vector<MatPtrs> t(n);
-  std::vector<Interval> iv;
+  std::vector<ByteRange> iv;
   iv.reserve(2 * static_cast<size_t>(n));
   for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];

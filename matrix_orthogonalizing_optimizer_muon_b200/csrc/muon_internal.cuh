@@ -15,8 +15,10 @@
 // X update is Y B, so every buffer keeps the parameter's layout.
 #pragma once
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <vector>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -90,6 +92,19 @@ struct MatPtrs {
   int32_t g_dtype;      // 0 bf16, 1 fp32
   int32_t vec_ok;       // all three pointers 16-byte aligned and C % 8 == 0
 };
+
+// Host: a byte range [lo, hi) of a caller buffer, for the aliasing checks
+struct ByteRange {
+  uintptr_t lo, hi;
+};
+
+// Host: true if any two ranges of v intersect (sorts v)
+inline bool any_overlap(std::vector<ByteRange>& v) {
+  std::sort(v.begin(), v.end(), [](const ByteRange& a, const ByteRange& b) { return a.lo < b.lo; });
+  for (size_t i = 1; i < v.size(); ++i)
+    if (v[i].lo < v[i - 1].hi) return true;
+  return false;
+}
 
 // Tile of a GEMM phase: .x matrix, .y row0, .z col0, .w n_need (columns that
 // hold useful output, <= kBN).  Symmetric phases list each tile of the lower
