@@ -97,3 +97,58 @@ def test_owner_assignment_is_balanced_and_deterministic():
         assert a == assign_owners(list(shapes), world)
         load = [sum(ns_work(s) for s, r in zip(shapes, a) if r == k) for k in range(world)]
         assert max(load) - min(load) <= max(ns_work(s) for s in shapes)
+
+
+SHAPES3 = [(24, 40), (8, 64)]
+
+
+def exact_grads(rank, step):
+    # small integer multiples of 2^-12: every partial sum over ranks is exact in
+    # fp32, whatever order the all-reduce adds them in
+    g = torch.Generator().manual_seed(500 * rank + step)
+    return [torch.randint(-512, 513, s, generator=g).float() * 2.0 ** -12 for s in SHAPES3]
+
+
+def _worker3(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        opt = DistributedMuon(SHAPES3, local_step=oracle_local_step, device="cpu")
+        g = torch.Generator().manual_seed(3)
+        Ws = [torch.randn(s, generator=g) * 0.02 for s in SHAPES3]
+        rms = None
+        for t in range(STEPS):
+            rms = opt.step(list(zip(Ws, exact_grads(rank, t))), lr=LR, weight_decay=WD, momentum=MU).clone()
+        out.put((rank, [W.numpy().copy() for W in Ws], rms.numpy().copy(), sorted(opt.M), opt.owner))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_ranks_with_an_idle_owner():
+    # two matrices on three ranks: one rank owns nothing, but still joins every
+    # collective and ends with the same weights
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker3, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=300) for _ in range(world)), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    g = torch.Generator().manual_seed(3)
+    Ws = [torch.randn(s, generator=g) * 0.02 for s in SHAPES3]
+    Ms = [torch.zeros(s) for s in SHAPES3]
+    for t in range(STEPS):
+        Gsum = [sum(gs) for gs in zip(*(exact_grads(r, t) for r in range(world)))]
+        ref_rms = oracle_local_step(list(zip(Ws, Gsum, Ms)), lr=LR, weight_decay=WD, momentum=MU)
+    owners = res[0][4]
+    assert len(set(owners)) == 2                       # one of the three ranks is idle
+    for rank, W_out, rms, owned, owner in res:
+        assert owner == owners
+        for a, b in zip(W_out, Ws):
+            assert np.array_equal(a, b.numpy())
+        assert np.array_equal(rms, ref_rms.numpy())
+        assert owned == [i for i, r in enumerate(owner) if r == rank]
