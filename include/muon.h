@@ -266,7 +266,7 @@ MUON_API void muon_adamw_destroy(muon_adamw_plan_t plan);
  * for a matrix with non-finite entries.
  * sigma_i^2 are the eigenvalues of the fp32 Gram matrix of the wide
  * orientation, found by two-sided block Jacobi in fp64 (32-row blocks, at
- * most 24 sweeps, stopped once the off-diagonal Frobenius norm is below 1e-8
+ * most 24 sweeps, stopped once the off-diagonal Frobenius norm is below 1e-6
  * of the whole); the entropy sums run in fp64 too.
  * ------------------------------------------------------------------------ */
 typedef struct muon_entropy_plan_s* muon_entropy_plan_t;

@@ -66,10 +66,11 @@ constexpr int kSortThreads = 1024;
 // a skipped entry moves an eigenvalue by at most S_ab^2 / |S_aa - S_bb|, or by
 // |S_ab| itself for a near-degenerate pair.
 constexpr double kInnerTol = 1e-13;
-// A matrix is done when off(G) <= kOffTol ||G||_F (Frobenius norms); the
-// rest moves the eigenvalues by second-order amounts (about 1e-11 of the
-// largest in the same simulations).
-constexpr double kOffTol = 1e-8;
+// A matrix is done when off(G) <= kOffTol ||G||_F (Frobenius norms).  The
+// rest moves the eigenvalues by second-order amounts: in the same
+// simulations at most 3e-9 of the largest eigenvalue, and H by 1e-10, far
+// below the rounding of the fp32 outputs.
+constexpr double kOffTol = 1e-6;
 constexpr size_t kSolveSmem = 2 * kEs * kEsLd * sizeof(double);
 constexpr size_t kUpdSmem = 3 * kEs * (kEs + 2) * sizeof(double);
 
