@@ -11,6 +11,9 @@
  *   - Sec. 2.2, Eq. 3 and Eq. 4 (= Sec. 3.1, Eq. 7): the decoupled, shape-scaled
  *     update W_t = W_{t-1} - eta (rms_scale sqrt(max(A,B)) O_t + lambda W_{t-1});
  *   - Sec. 2.3, Algorithm 1, last line: the logged update RMS sqrt(mean(u^2)).
+ * Also: the other update scales of Sec. 3.1 (Eq. 5, Eq. 6), the AdamW step
+ * of the parameters that are not matrices (Sec. 2.2), and the SVD-entropy
+ * diagnostic of Sec. 3.4.
  *
  * Conventions for every entry point:
  *   - All tensors are dense, row-major, contiguous, and live in device memory
@@ -18,7 +21,7 @@
  *     (descriptor lists, coefficient triples) are read before the call returns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; no entry point synchronizes
- *     the host except muon_get_status and muon_profile_read, which say so.
+ *     the host except the status and profile reads, which say so.
  *   - Arguments are validated on the host before anything is enqueued; an
  *     error return means nothing was launched and no tensor was modified.
  *   - A plan is not thread-safe: calls on one plan must be serialized by the
