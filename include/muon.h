@@ -20,8 +20,11 @@
  *     of the device that is current when the plan is created.  "Host" arrays
  *     (descriptor lists, coefficient triples) are read before the call returns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
- *     stream).  Work is enqueued asynchronously; no entry point synchronizes
- *     the host except the status and profile reads, which say so.
+ *     stream).  Work is enqueued asynchronously.  The status and profile
+ *     reads synchronize the host, and say so.  A step or compute call whose
+ *     device pointers differ from every table the plan keeps may first wait
+ *     for the host-to-device copy of an older table to finish, because that
+ *     copy reads the pinned buffer the new table is written to.
  *   - Arguments are validated on the host before anything is enqueued; an
  *     error return means nothing was launched and no tensor was modified.
  *   - A plan is not thread-safe: calls on one plan must be serialized by the
