@@ -80,14 +80,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 25):
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
         self.proc = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -105,7 +106,12 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
+        """Median SM clock under load (samples with power above 400 W, the
+        idle GPU draws about 200 W), the maximum clock, the throttle reasons
+        seen in any sample, and how many samples showed each."""
         sm, mx, reasons = [], [], set()
+        counts = {}
+        loaded = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in getattr(self, "lines", []):
             f = [x.strip() for x in ln.split(",")]
@@ -116,13 +122,20 @@ class ClockSampler:
                 mx.append(float(f[2]))
             except ValueError:
                 continue
+            try:
+                if float(f[3]) > 400.0:
+                    loaded.append(float(f[1]))
+            except ValueError:
+                pass
             for name, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
+                    counts[name] = counts.get(name, 0) + 1
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(loaded), "reason_samples": counts,
+                "sm_mhz_min": min(loaded or sm), "interval_ms": self.interval_ms}
 
 
 # ---------------------------------------------------------------------- replicas
@@ -306,6 +319,123 @@ def torch_eager_ns_ms(Gs, zero, steps: int, abc, reps: int = 3) -> float:
     return e0.elapsed_time(e1) / reps
 
 
+def library_ceiling(wl, dev, steps: int = 5, reps: int = 3):
+    """Same-box context point, not part of the product: the three products of
+    the quintic iteration as cuBLAS batched GEMMs (torch.bmm / baddbmm in
+    bf16, dense, no symmetry) over the workload's non-zero matrices, grouped
+    by shape in the wide orientation, on random inputs of the same shapes.
+    Returns per-phase dense TFLOP/s and the whole iteration's rate in the
+    algorithmic (symmetry-aware) count used for the kernel."""
+    import torch
+    groups = {}
+    for i, (_, r, c) in enumerate(wl.shapes):
+        if i not in wl.zero_grad:
+            m, n = min(r, c), max(r, c)
+            groups[(m, n)] = groups.get((m, n), 0) + 1
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    bufs = []
+    for (m, n), cnt in groups.items():
+        X = (torch.randn(cnt, m, n, device=dev, generator=gen) / math.sqrt(m * n)).to(torch.bfloat16)
+        bufs.append((X, torch.empty(cnt, m, m, device=dev, dtype=torch.bfloat16),
+                     torch.empty(cnt, m, m, device=dev, dtype=torch.bfloat16), torch.empty_like(X)))
+    a, b, c = 3.4445, -4.7750, 2.0315
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ms = [0.0, 0.0, 0.0]
+
+    def one_pass(record):
+        for _ in range(steps):
+            if record:
+                ev[0].record()
+            for X, A, _, _ in bufs:
+                torch.bmm(X, X.transpose(1, 2), out=A)
+            if record:
+                ev[1].record()
+            for _, A, B, _ in bufs:
+                torch.baddbmm(A, A, A, beta=b, alpha=c, out=B)
+            if record:
+                ev[2].record()
+            for X, _, B, Y in bufs:
+                torch.baddbmm(X, B, X, beta=a, alpha=1.0, out=Y)
+            if record:
+                ev[3].record()
+                torch.cuda.synchronize()
+                for k in range(3):
+                    ms[k] += ev[k].elapsed_time(ev[k + 1])
+
+    one_pass(False)
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        one_pass(True)
+    ms = [v / reps for v in ms]
+    dense = [0.0, 0.0, 0.0]
+    alg = 0.0
+    for (m, n), cnt in groups.items():
+        dense[0] += cnt * steps * 2.0 * m * m * n
+        dense[1] += cnt * steps * 2.0 * m * m * m
+        dense[2] += cnt * steps * 2.0 * m * m * n
+        alg += cnt * ns_flops(m, n, steps)
+    del bufs
+    torch.cuda.empty_cache()
+    return {"what": "cuBLAS batched bf16 GEMMs (torch.bmm/baddbmm, dense, no symmetry) of the Gram, polynomial and "
+                    "X-update products over the same non-zero matrices, 5 iterations; context only",
+            "ms_per_step": sum(ms), "phase_ms": dict(zip(("gram", "poly", "x_update"), ms)),
+            "phase_tflops_dense": {k: d / (t * 1e-3) / 1e12 for k, d, t in zip(("gram", "poly", "x_update"), dense, ms)},
+            "tflops_algorithmic": alg / (sum(ms) * 1e-3) / 1e12}
+
+
+def hybrid_mixed8(dev, steps: int = 5, warmup: int = 3):
+    """Time the full optimizer step of the 1624-matrix mixed model: Muon over
+    every matrix and AdamW over its 16 RMSNorm gains (Sec. 2.2 and Appendix D),
+    one HybridStep per step on resident synthetic inputs."""
+    import torch
+    from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
+    from matrix_orthogonalizing_optimizer_muon_b200.api import HybridStep
+    wl = wlm.mixed8()
+    shapes = [(r, c) for _, r, c in wl.shapes]
+    sizes = [r * c for r, c in shapes]
+    total = sum(sizes)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    Wbuf = torch.empty(total, device=dev).normal_(0.0, 0.02, generator=gen)
+    Gbuf = torch.empty(total, device=dev).normal_(0.0, 1e-3, generator=gen).to(torch.bfloat16)
+    Mbuf = torch.empty(total, device=dev)
+    mats, off = [], 0
+    for (r, c), e in zip(shapes, sizes):
+        mats.append((Wbuf[off:off + e].view(r, c), Gbuf[off:off + e].view(r, c), Mbuf[off:off + e].view(r, c)))
+        off += e
+    for i in wl.zero_grad:
+        mats[i][1].zero_()
+    k, gsz = wl.excluded_gains, wl.gain_size
+    vecs = [(torch.ones(gsz, device=dev), torch.full((gsz,), 1e-3, device=dev, dtype=torch.bfloat16),
+             torch.empty(gsz, device=dev), torch.empty(gsz, device=dev)) for _ in range(k)]
+    opt = HybridStep(shapes, [gsz] * k, momenta=[m for _, _, m in mats], adam_states=[(m, v) for _, _, m, v in vecs])
+    ws = opt.muon.workspace_bytes
+    for t in range(1, warmup + 1):
+        opt.step(mats, vecs, t=t, lr=4.2e-4, weight_decay=0.1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    opt.muon.profile(True)
+    opt.muon.profile_read()
+    e0.record()
+    for t in range(warmup + 1, warmup + steps + 1):
+        opt.step(mats, vecs, t=t, lr=4.2e-4, weight_decay=0.1)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    prof = opt.muon.profile_read()
+    st = opt.status()
+    opt.close()
+    nz = sum(ns_flops(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
+    gemm_ms = sum(prof["ms"][x] for x in ("gram", "poly", "x_update")) / max(prof["calls"], 1)
+    del mats, vecs, Wbuf, Gbuf, Mbuf
+    torch.cuda.empty_cache()
+    return {"what": "full optimizer step of the 8-layer mixed MoE: Muon over 1624 matrices + AdamW over 16 decayed "
+                    "RMSNorm gains (HybridStep), shared lr and weight decay",
+            "ms_per_step": ms, "steps": steps, "status": st, "muon_workspace_gb": ws / 1e9,
+            "ns_ms_per_step": gemm_ms, "ns_tflops": nz / (gemm_ms * 1e-3) / 1e12}
+
+
 def run_reference(args, wl, rank: int):
     if rank != 0:
         return
@@ -323,20 +453,25 @@ def run_reference(args, wl, rank: int):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(wl),
+            "data": "synthetic", "config": workload_config(wl, args.scale),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                              "host_cpus": os.cpu_count(), "blas": blas_vendor()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def workload_config(wl):
+SCALE_TEXT = {"max_dim": "Eq. 4: 0.2 sqrt(max(A,B))", "hidden": "Eq. 5: 0.2 sqrt(H), H = 2048",
+              "update_norm": "Eq. 6: 0.2 / RMS(O)"}
+
+
+def workload_config(wl, scale: str = "max_dim"):
     nz = [s for i, s in enumerate(wl.shapes) if i not in wl.zero_grad]
     return {"workload": f"{wl.name}: {wl.n} matrices ({len(nz)} with non-zero gradient)",
             "matrices": wl.n, "elements": wl.elements, "ns_steps": 5,
             "shapes": sorted({(r, c) for _, r, c in wl.shapes}),
             "inputs": "synthetic: W ~ N(0, 0.02^2) fp32, G ~ N(0, 1e-6) bf16, M_0 = 0",
-            "l2": "inputs larger than L2 (no flush needed)", "parallelism": "replicas (no exchange)"}
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": "replicas (no exchange)",
+            "update_scale": SCALE_TEXT[scale]}
 
 
 # ---------------------------------------------------------------------- GPU arm
@@ -356,12 +491,25 @@ def main(argv=None) -> int:
                     help="update scale of Sec. 3.1: Eq. 4 (default), Eq. 5 with H = 2048, Eq. 6")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--limit", type=int, default=0, help="keep only the first N matrices (small profiling case)")
+    ap.add_argument("--shape", default=None,
+                    help="RxC: time one matrix of this shape (with --workload ns_sweep, one of the sweep shapes)")
+    ap.add_argument("--max-workspace-gb", type=float, default=0.0,
+                    help="cap the plan's device memory (muon_init_ex); 0 = uncapped")
+    ap.add_argument("--no-hybrid", action="store_true",
+                    help="skip the hybrid Muon + AdamW step of the 1624-matrix mixed model")
+    ap.add_argument("--no-ceiling", action="store_true",
+                    help="skip the library batched-GEMM context point of the three product shapes")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
 
     from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
     wl = wlm.get(args.workload)
+    if args.shape:
+        r, c = (int(v) for v in args.shape.lower().split("x"))
+        wl.shapes = [(f"m{r}x{c}", r, c)]
+        wl.zero_grad = set()
+        wl.name += f"[{r}x{c}]"
     if args.limit > 0:
         wl.shapes = wl.shapes[:args.limit]
         wl.zero_grad = {i for i in wl.zero_grad if i < args.limit}
@@ -400,7 +548,8 @@ def main(argv=None) -> int:
         off += e
     for i in wl.zero_grad:
         Gs[i].zero_()
-    plan = MuonPlan(shapes, momenta=Ms)
+    cap = int(args.max_workspace_gb * 1e9)
+    plan = MuonPlan(shapes, momenta=Ms, max_workspace_bytes=cap or None)
     params = list(zip(Ws, Gs, Ms))
     plan.bind(params)
     rms = torch.zeros(wl.n, device=dev)
@@ -491,7 +640,7 @@ def main(argv=None) -> int:
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": Gbuf.numel() * 2, "d2h_bytes_per_step": wl.n * 4,
                "path": "MuonPlan.step (C ABI muon_step) with each step's G copied from pinned host memory "
                        "(double-buffered: the copy of step k+1 overlaps step k) and the update RMS copied back "
-                       "each step"}
+                       "each step; W and M, the optimizer state, stay resident in HBM as in training"}
         del Gbufs, views, pbufs
         plan.bind(params)
     st = plan.status()
@@ -523,16 +672,24 @@ def main(argv=None) -> int:
                    "ns_ms_per_step": t_eager, "tflops_algorithmic": nz_flops / (t_eager * 1e-3) / 1e12,
                    "tflops_dense_equivalent": dense_flops / (t_eager * 1e-3) / 1e12}
 
+    ceiling = None
+    if not args.no_ceiling:
+        ceiling = library_ceiling(wl, dev)
+
     entropy = None
     if not args.no_entropy:
         entropy = bench_entropy(Ws)
 
     adamw = None
-    if not args.no_adamw:
+    hybrid = None
+    if not (args.no_adamw and args.no_hybrid):
         plan.close()
         del Wbuf, Gbuf, Mbuf, Ws, Gs, Ms, params
         torch.cuda.empty_cache()
-        adamw = bench_adamw(dev)
+        if not args.no_adamw:
+            adamw = bench_adamw(dev)
+        if not args.no_hybrid:
+            hybrid = hybrid_mixed8(dev)
 
     cpu = None
     if world == 1 and args.cpu_budget > 0:
@@ -541,9 +698,8 @@ def main(argv=None) -> int:
                "sample": f"{d} whole-matrix fp64 oracle steps of the workload ({s:.1f} s), same FLOP count",
                "host_cpus": os.cpu_count(), "blas": blas_vendor()}
 
-    config = workload_config(wl)
-    config["update_scale"] = {"max_dim": "Eq. 4: 0.2 sqrt(max(A,B))", "hidden": "Eq. 5: 0.2 sqrt(H), H = 2048",
-                              "update_norm": "Eq. 6: 0.2 / RMS(O)"}[args.scale]
+    clocks = clk.summary()
+    config = workload_config(wl, args.scale)
     if args.scale == "update_norm":
         fin_ms = prof["ms"]["finalize"] / calls
         config["update_norm_passes"] = {
@@ -569,11 +725,14 @@ def main(argv=None) -> int:
                         "bytes_per_elem": K1_BYTES_PER_ELEM},
         "cpu_baseline": cpu,
         "context_torch_eager_ns": context,
+        "context_library_batched_gemm": ceiling,
+        "hybrid_step_mixed8": hybrid,
         "adamw_companion": adamw,
         "svd_entropy": entropy,
         "e2e": e2e,
         "gpu_launches": int(round(per_step_launches * args.steps)),
-        "clocks": clk.summary(),
+        "clocks": clocks,
+        "ns_mcycles_per_step": (gemm_ms * clocks["sm_mhz"] / 1e3) if clocks.get("sm_mhz") else None,
     }
     print(json.dumps(line), flush=True)
     plan.close()

@@ -83,6 +83,7 @@ typedef enum { MUON_SCALE_MAX_DIM = 0, MUON_SCALE_HIDDEN = 1, MUON_SCALE_UPDATE_
 /* muon_init flags */
 #define MUON_INIT_ZERO_MOMENTUM 0x1u /* zero every M on `stream` (M_0 = 0, Sec. 2.1) */
 #define MUON_INIT_FP32_NS       0x2u /* also reserve the workspace of the fp32 path */
+#define MUON_INIT_MAX_WORKSPACE 0x4u /* cap the plan's device memory (muon_init_ex only) */
 
 /* One matrix parameter.  Shape [rows, cols]; for muon_init only the shape is
  * kept (pointers may be NULL unless MUON_INIT_ZERO_MOMENTUM is given), for
@@ -126,10 +127,32 @@ MUON_API muon_status_t muon_hparams_default(muon_hparams_t* hp);
  * With MUON_INIT_ZERO_MOMENTUM the M buffers are zeroed on `stream`.
  * The current CUDA device must be an sm_100 part.
  * Errors: INVALID_ARG (out/params NULL, n < 1, shape out of range, reserved != 0,
- * M NULL with ZERO_MOMENTUM), UNSUPPORTED (device is not sm_100), NO_MEMORY, CUDA.
+ * M NULL with ZERO_MOMENTUM, MUON_INIT_MAX_WORKSPACE without a budget: use
+ * muon_init_ex), UNSUPPORTED (device is not sm_100), NO_MEMORY, CUDA.
  * On error *out is set to NULL and nothing is allocated. */
 MUON_API muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags,
                         void* stream);
+
+/* muon_init with a cap on the plan's device memory.  With
+ * MUON_INIT_MAX_WORKSPACE in `flags` (and only then) max_workspace_bytes > 0
+ * bounds muon_workspace_bytes(plan): the matrices are packed, largest
+ * Newton-Schulz work first, into waves whose iterate and Gram/polynomial
+ * buffers are resident one wave at a time, and every call runs the waves one
+ * after another on its stream (momentum and normalisation, the N iterations
+ * and the update pass of one wave, then the next).  Each matrix's arithmetic
+ * does not depend on the wave that holds it, so results are bitwise those of
+ * an uncapped plan; only the launch count grows.  Without the flag
+ * max_workspace_bytes must be 0 and the call equals muon_init (one wave).
+ * For scale: 1624 matrices of an 8-layer, 64+2-expert MoE at hidden 2048
+ * need about 41 GB uncapped; a cap trades that for more, smaller launches.
+ * Errors: as muon_init, plus INVALID_ARG (flag and budget disagree) and
+ * NO_MEMORY (the cap cannot hold the plan's fixed structures and the largest
+ * matrix's buffers). */
+MUON_API muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags,
+                                    size_t max_workspace_bytes, void* stream);
+
+/* Number of waves of the plan (1 unless capped); -1 for NULL. */
+MUON_API int32_t muon_num_waves(muon_plan_t plan);
 
 /* One Muon step over all n matrices of the plan (n and every shape must equal
  * the plan's):  M <- mu M + G;  Y = mu M + G (or M);  O = Newton-Schulz(Y) with
@@ -161,6 +184,19 @@ MUON_API muon_status_t muon_orthogonalize(muon_plan_t plan, const void* const* X
 
 /* Device bytes owned by the plan (workspace, schedules, descriptors). 0 for NULL. */
 MUON_API size_t muon_workspace_bytes(muon_plan_t plan);
+
+/* Failure-detection test hook (host-side injection; nothing faults).  The
+ * first Newton-Schulz launch of the next bf16-path muon_step or
+ * muon_orthogonalize call on this plan makes one thread of every CTA wait on
+ * a barrier that nothing arrives at, for at most wait_ns nanoseconds
+ * (1 .. 10^9), before any operand load or tensor-core instruction is issued.
+ * The wait runs out, the launch records MUON_ERR_TIMEOUT in the plan's status
+ * and does no work, and the call's results are invalid, as after any
+ * device-side timeout; later launches and calls run normally.  This exercises
+ * the bounded device waits' error path: muon_get_status must report
+ * MUON_ERR_TIMEOUT and the context must stay usable.
+ * Errors: INVALID_ARG (NULL plan, wait_ns out of range). */
+MUON_API muon_status_t muon_inject_wait_timeout(muon_plan_t plan, uint32_t wait_ns);
 
 /* Synchronizes the plan's last stream, returns the sticky device status of all
  * calls since the previous muon_get_status (MUON_OK, MUON_ERR_TIMEOUT or
@@ -201,13 +237,52 @@ MUON_API muon_status_t muon_profile_read(muon_plan_t plan, double* phase_ms, int
  * device array of about 10.7 MB that every GPU loading this library holds
  * until the process exits.  The first call on a device resolves that array's
  * address (cudaGetSymbolAddress); make that first call before any stream
- * capture.  Every call shares the array: calls that can overlap on the GPU
- * (different streams, or several host threads) race and must be serialized
- * by the caller.  Non-finite inputs give non-finite outputs; no status is
- * recorded.  Errors: INVALID_ARG, ALIAS, UNSUPPORTED, CUDA. */
+ * capture.  Each call copies its small descriptors (tile lists, TMA
+ * descriptors) from pageable host memory, so it may wait on the host until
+ * the driver has staged them; a call on a stream that is being captured
+ * returns MUON_ERR_UNSUPPORTED and enqueues nothing.  Every call shares the
+ * array: calls that can overlap on the GPU (different streams, or several
+ * host threads) race and must be serialized by the caller.  Non-finite
+ * inputs give non-finite outputs; no status is recorded.
+ * Errors: INVALID_ARG, ALIAS, UNSUPPORTED, CUDA. */
 MUON_API muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_out, int64_t rows, int64_t cols,
                                                   int32_t in_dtype, int32_t ns_steps, const float abc[3],
                                                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packing for data-parallel Muon ("Muon is Scalable for LLM Training",
+ * Sec. 2.3, Algorithm 1): the gradients of many matrices go into one flat
+ * buffer before the reduce-scatter, and the updated weights into and out of
+ * the flat buffers of the all-gather.  A pack plan holds a fixed list of
+ * segments; each run copies all of them in one launch (dst[k] = src[k],
+ * converted between bf16 and fp32 with round-to-nearest-even when the dtypes
+ * differ), so a step issues a constant number of launches whatever its
+ * matrix count.  HBM-bound: source plus destination bytes per element.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* src;       /* device, numel elements of src_dtype                   */
+  void*       dst;       /* device, numel elements of dst_dtype                   */
+  int64_t     numel;     /* 1 <= numel <= 2^40                                    */
+  int32_t     src_dtype; /* muon_dtype_t                                          */
+  int32_t     dst_dtype; /* muon_dtype_t                                          */
+} muon_segment_t;
+
+typedef struct muon_pack_plan_s* muon_pack_plan_t;
+
+/* Plan for n >= 1 segments on the current device (the pointers are kept;
+ * the caller keeps the buffers alive).  Destinations must be pairwise
+ * disjoint and no source may overlap a destination (sources may overlap each
+ * other).  Uploads the segment table with a synchronous copy.
+ * Errors: INVALID_ARG (NULL, bad count, size or dtype), ALIAS, NO_MEMORY, CUDA.
+ * On error *out is NULL. */
+MUON_API muon_status_t muon_pack_init(muon_pack_plan_t* out, const muon_segment_t* segs, int32_t n, void* stream);
+
+/* Copy every segment of the plan, asynchronously on `stream` (one launch).
+ * Errors: INVALID_ARG (NULL plan, or another device is current), CUDA. */
+MUON_API muon_status_t muon_pack_run(muon_pack_plan_t plan, void* stream);
+
+/* Waits for the plan's last stream and frees it; NULL is ignored. */
+MUON_API void muon_pack_destroy(muon_pack_plan_t plan);
 
 /* ------------------------------------------------------------------------
  * AdamW companion for the parameters that are not matrices.  The pages

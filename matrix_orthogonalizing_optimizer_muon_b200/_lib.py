@@ -30,15 +30,18 @@ MUON_NS_BF16 = 0
 MUON_NS_FP32 = 1
 MUON_INIT_ZERO_MOMENTUM = 0x1
 MUON_INIT_FP32_NS = 0x2
+MUON_INIT_MAX_WORKSPACE = 0x4
 MUON_SCALE_MAX_DIM, MUON_SCALE_HIDDEN, MUON_SCALE_UPDATE_NORM = 0, 1, 2
 MUON_NUM_PHASES = 5
 PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
 
-EXPORTED = ("muon_hparams_default", "muon_init", "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
+EXPORTED = ("muon_hparams_default", "muon_init", "muon_init_ex", "muon_num_waves", "muon_inject_wait_timeout",
+            "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
             "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read",
             "muon_orthogonalize_noalloc", "muon_adamw_hparams_default", "muon_adamw_init", "muon_adamw_step",
             "muon_adamw_destroy", "muon_entropy_init", "muon_entropy_compute", "muon_entropy_num_singular_values",
-            "muon_entropy_get_status", "muon_entropy_profile", "muon_entropy_destroy")
+            "muon_entropy_get_status", "muon_entropy_profile", "muon_entropy_destroy", "muon_pack_init",
+            "muon_pack_run", "muon_pack_destroy")
 
 
 class muon_param_t(ctypes.Structure):
@@ -52,6 +55,11 @@ class muon_hparams_t(ctypes.Structure):
                 ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float), ("b", ctypes.c_float),
                 ("c", ctypes.c_float), ("rms_scale", ctypes.c_float), ("nesterov", ctypes.c_int32),
                 ("ns_precision", ctypes.c_int32), ("scale_mode", ctypes.c_int32), ("hidden_dim", ctypes.c_float)]
+
+
+class muon_segment_t(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("numel", ctypes.c_int64),
+                ("src_dtype", ctypes.c_int32), ("dst_dtype", ctypes.c_int32)]
 
 
 class muon_adamw_param_t(ctypes.Structure):
@@ -87,6 +95,19 @@ def load() -> ctypes.CDLL:
     lib.muon_hparams_default.restype = ctypes.c_int
     lib.muon_init.argtypes = [ctypes.POINTER(P), ctypes.POINTER(muon_param_t), ctypes.c_int32, ctypes.c_uint32, P]
     lib.muon_init.restype = ctypes.c_int
+    lib.muon_init_ex.argtypes = [ctypes.POINTER(P), ctypes.POINTER(muon_param_t), ctypes.c_int32, ctypes.c_uint32,
+                                 ctypes.c_size_t, P]
+    lib.muon_init_ex.restype = ctypes.c_int
+    lib.muon_num_waves.argtypes = [P]
+    lib.muon_num_waves.restype = ctypes.c_int32
+    lib.muon_inject_wait_timeout.argtypes = [P, ctypes.c_uint32]
+    lib.muon_inject_wait_timeout.restype = ctypes.c_int
+    lib.muon_pack_init.argtypes = [ctypes.POINTER(P), ctypes.POINTER(muon_segment_t), ctypes.c_int32, P]
+    lib.muon_pack_init.restype = ctypes.c_int
+    lib.muon_pack_run.argtypes = [P, P]
+    lib.muon_pack_run.restype = ctypes.c_int
+    lib.muon_pack_destroy.argtypes = [P]
+    lib.muon_pack_destroy.restype = None
     lib.muon_step.argtypes = [P, ctypes.POINTER(muon_param_t), ctypes.c_int32, ctypes.POINTER(muon_hparams_t), P, P]
     lib.muon_step.restype = ctypes.c_int
     lib.muon_orthogonalize.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int32, ctypes.c_int32,
@@ -155,6 +176,35 @@ def muon_init(params, n: int, flags: int, stream: int) -> ctypes.c_void_p:
     plan = ctypes.c_void_p()
     check(load().muon_init(ctypes.byref(plan), params, int(n), int(flags), ctypes.c_void_p(stream)), "muon_init")
     return plan
+
+
+def muon_init_ex(params, n: int, flags: int, max_workspace_bytes: int, stream: int) -> ctypes.c_void_p:
+    plan = ctypes.c_void_p()
+    check(load().muon_init_ex(ctypes.byref(plan), params, int(n), int(flags), int(max_workspace_bytes),
+                              ctypes.c_void_p(stream)), "muon_init_ex")
+    return plan
+
+
+def muon_num_waves(plan) -> int:
+    return int(load().muon_num_waves(plan))
+
+
+def muon_pack_init(segs, n: int, stream: int) -> ctypes.c_void_p:
+    plan = ctypes.c_void_p()
+    check(load().muon_pack_init(ctypes.byref(plan), segs, int(n), ctypes.c_void_p(stream)), "muon_pack_init")
+    return plan
+
+
+def muon_pack_run(plan, stream: int) -> None:
+    check(load().muon_pack_run(plan, ctypes.c_void_p(stream)), "muon_pack_run")
+
+
+def muon_pack_destroy(plan) -> None:
+    load().muon_pack_destroy(plan)
+
+
+def muon_inject_wait_timeout(plan, wait_ns: int) -> None:
+    check(load().muon_inject_wait_timeout(plan, int(wait_ns)), "muon_inject_wait_timeout")
 
 
 def muon_step(plan, params, n: int, hp: muon_hparams_t, update_rms_ptr: int | None, stream: int) -> None:

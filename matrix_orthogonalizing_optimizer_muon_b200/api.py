@@ -14,6 +14,8 @@ step for them.
     adam = AdamWPlan([g.numel() for g in gains], states=[(m, v) ...])
     adam.step(list(zip(gains, grads, ms, vs)), step=t, lr=4.2e-4, weight_decay=0.1)
 
+``HybridStep`` runs both plans as one optimizer step.
+
 Sec. 3.4 compares optimisers by the SVD entropy of the weight matrices;
 ``EntropyPlan`` computes it on the GPU.
 
@@ -54,7 +56,8 @@ _GDT = {torch.bfloat16: L.MUON_DT_BF16, torch.float32: L.MUON_DT_FP32}
 class MuonPlan:
     """A libmuon plan for a fixed list of matrix shapes on the current device."""
 
-    def __init__(self, shapes, *, momenta=None, fp32_ns: bool = False, stream=None):
+    def __init__(self, shapes, *, momenta=None, fp32_ns: bool = False, max_workspace_bytes: int | None = None,
+                 stream=None):
         shapes = [tuple(int(v) for v in s) for s in shapes]
         if any(len(s) != 2 for s in shapes):
             raise ValueError("Muon plans take 2-D shapes only")
@@ -69,7 +72,11 @@ class MuonPlan:
                 arr[i].M = M.data_ptr()
         for i, (r, c) in enumerate(shapes):
             arr[i].rows, arr[i].cols = r, c
-        self._plan = L.muon_init(arr, self.n, flags, _stream_handle(stream))
+        if max_workspace_bytes:
+            self._plan = L.muon_init_ex(arr, self.n, flags | L.MUON_INIT_MAX_WORKSPACE, int(max_workspace_bytes),
+                                        _stream_handle(stream))
+        else:
+            self._plan = L.muon_init(arr, self.n, flags, _stream_handle(stream))
         self._params = (L.muon_param_t * self.n)()
         self._key = None
         self._bound = {}   # recent bindings: key -> descriptor array
@@ -156,6 +163,11 @@ class MuonPlan:
     def workspace_bytes(self) -> int:
         return L.muon_workspace_bytes(self._plan)
 
+    @property
+    def waves(self) -> int:
+        """How many waves a call runs (1 unless the plan has a workspace cap)."""
+        return L.muon_num_waves(self._plan)
+
     def status(self) -> int:
         """Synchronizing read-and-clear of the device status (an int status code)."""
         return L.muon_get_status(self._plan)
@@ -235,6 +247,81 @@ class AdamWPlan:
             self.close()
         except Exception:
             pass
+
+
+class PackPlan:
+    """One-launch copy of a fixed list of (src, dst) tensor pairs (bf16 or
+    fp32 each; the values are converted when the dtypes differ)."""
+
+    def __init__(self, pairs, *, stream=None):
+        pairs = list(pairs)
+        if not pairs:
+            raise ValueError("a pack plan needs at least one (src, dst) pair")
+        arr = (L.muon_segment_t * len(pairs))()
+        for k, (src, dst) in enumerate(pairs):
+            for t, name in ((src, "src"), (dst, "dst")):
+                _check_tensor(t, (torch.bfloat16, torch.float32), f"{name}[{k}]")
+            if src.numel() != dst.numel():
+                raise ValueError(f"pair {k}: {src.numel()} source and {dst.numel()} destination elements")
+            a = arr[k]
+            a.src, a.dst, a.numel = src.data_ptr(), dst.data_ptr(), src.numel()
+            a.src_dtype, a.dst_dtype = _GDT[src.dtype], _GDT[dst.dtype]
+        self._keep = pairs  # the plan holds raw pointers: keep the tensors alive
+        self._plan = L.muon_pack_init(arr, len(pairs), _stream_handle(stream))
+
+    def run(self, stream=None) -> None:
+        L.muon_pack_run(self._plan, _stream_handle(stream))
+
+    def close(self) -> None:
+        if getattr(self, "_plan", None):
+            L.muon_pack_destroy(self._plan)
+            self._plan = None
+            self._keep = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class HybridStep:
+    """The full optimizer step of "Muon is Scalable for LLM Training"
+    (Sec. 2.2, "Matching update RMS of AdamW"): Muon for every matrix
+    parameter and AdamW for the rest (RMSNorm gains, embedding, LM head), one
+    learning rate and one weight decay for both; the RMSNorm gains keep their
+    weight decay (Appendix D, "Training stability").  Both plans enqueue on
+    the same stream, Muon first; nothing waits on the host.
+
+        opt = HybridStep([W.shape for W in mats], [p.numel() for p in vecs],
+                         momenta=Ms, adam_states=[(m, v), ...])
+        opt.step(list(zip(mats, mat_grads, Ms)), list(zip(vecs, vec_grads, ms, vs)),
+                 t=step, lr=4.2e-4, weight_decay=0.1)
+    """
+
+    def __init__(self, matrix_shapes, vector_numels, *, momenta=None, adam_states=None, vector_g_dtypes=None,
+                 vector_decay=None, max_workspace_bytes: int | None = None, stream=None):
+        self.muon = MuonPlan(matrix_shapes, momenta=momenta, max_workspace_bytes=max_workspace_bytes, stream=stream)
+        self.adamw = AdamWPlan(vector_numels, g_dtypes=vector_g_dtypes, states=adam_states, stream=stream)
+        self.vector_decay = list(vector_decay) if vector_decay is not None else None
+
+    def step(self, matrices, vectors, *, t: int, lr: float, weight_decay: float, momentum: float = 0.95,
+             ns_steps: int = 5, coeffs=DEFAULT_COEFFS, betas=(0.9, 0.95), eps: float = 1e-8,
+             update_rms: torch.Tensor | None = None, stream=None) -> None:
+        """matrices: [(W, G, M), ...] in the Muon plan's order; vectors:
+        [(P, G, m, v), ...] in the AdamW plan's order; t >= 1 is the step
+        count of AdamW's bias corrections."""
+        self.muon.step(matrices, lr=lr, weight_decay=weight_decay, momentum=momentum, ns_steps=ns_steps,
+                       coeffs=coeffs, update_rms=update_rms, stream=stream)
+        self.adamw.step(vectors, step=t, lr=lr, weight_decay=weight_decay, betas=betas, eps=eps,
+                        decay=self.vector_decay, stream=stream)
+
+    def status(self) -> int:
+        return self.muon.status()
+
+    def close(self) -> None:
+        self.muon.close()
+        self.adamw.close()
 
 
 class EntropyPlan:

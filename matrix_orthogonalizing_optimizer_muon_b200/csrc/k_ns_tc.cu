@@ -80,8 +80,8 @@ struct SmemLayout {
   static constexpr int kUpdRing = kStagesUpd * kStageBytes;           // X update only
   static constexpr int kEpi = kStagesSym * kStageBytes;               // staging blocks
   static constexpr int kBar = kEpi + kEpiBytes;
-  // full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr int kNumBars = 2 * kStagesMax + 5;
+  // full[S], empty[S], tfull[2], tempty[2], drain, never (nothing arrives on it)
+  static constexpr int kNumBars = 2 * kStagesMax + 6;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort (int)
   static constexpr int kBytes = kMisc + 16;
 };
@@ -157,17 +157,22 @@ __device__ __forceinline__ unsigned long long global_ns() {
 }
 
 // Wait for the phase with the given parity to complete; false after
-// kWaitLimitNs or as soon as another role of this CTA raised `abort`.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+// limit_ns or as soon as another role of this CTA raised `abort`.
+__device__ __noinline__ bool wait_bounded_ns(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                             unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0u) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) return false;
+      if (global_ns() - t0 > limit_ns) return false;
     }
   }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+  return wait_bounded_ns(bar, parity, abort_flag, kWaitLimitNs);
 }
 
 // TMA load into this CTA's shared memory, completing on a barrier that may
@@ -438,6 +443,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStagesMax + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStagesMax + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * kStagesMax + 4);
+  const uint32_t never_bar = bar0 + 8u * (2 * kStagesMax + 5);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::kMisc + 4);
 
@@ -459,6 +465,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(tempty_bar(b), 2 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -474,6 +481,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   unsigned* status = g.ws.status;
+
+  if (g.test_wait_ns != 0) {
+    // Failure-detection test (the same value in every CTA of the grid): one
+    // thread per CTA waits, with the short limit, on a barrier that nothing
+    // arrives at, then raises the abort flag of both CTAs of its pair and the
+    // timeout status.  This happens before any role starts, so no operand
+    // load or tensor-core instruction is ever issued and every role below
+    // sees the flag and returns at once.
+    if (warp == kWarpEpi0 && lane == 0) {
+      if (!wait_bounded_ns(never_bar, 0u, nullptr, g.test_wait_ns)) {
+        const uint32_t peer_abort = map_to_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+        *abort_flag = 1;
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+        atomicOr(status, kStatusTimeout);
+      }
+    }
+    cluster_sync();
+  }
 
   if (warp == kWarpProducer || warp >= kWarpProducer2) {
     // ------------------------------------------------------------ TMA producers (both CTAs)

@@ -108,9 +108,21 @@ bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0,
 namespace {
 
 struct ProfRec {
-  int first_event;
-  int nlaunch;
-  int phases[3 * kMaxNsSteps + 4];
+  int first_event = 0;
+  int nlaunch = 0;
+  std::vector<int> phases;
+};
+
+// One wave of a plan: the matrices whose Newton-Schulz workspace is resident
+// at the same time, and the ranges of the plan's schedules that cover them.
+// A plan without a workspace cap has one wave holding every matrix.
+struct Wave {
+  int sym_off = 0, n_sym = 0;      // bf16 path, symmetric products
+  int full_off = 0, n_full = 0;    // bf16 path, X update
+  int sym32_off = 0, n_sym32 = 0;  // fp32 path
+  int full32_off = 0, n_full32 = 0;
+  int chunk_off = 0, nchunks = 0;  // elementwise chunks
+  int nmat = 0;
 };
 
 }  // namespace
@@ -135,6 +147,8 @@ struct muon_plan_s {
   int n_sym = 0, n_full = 0, n_sym32 = 0, n_full32 = 0;
   ChunkDesc* chunks_d = nullptr;
   int nchunks = 0;
+  std::vector<Wave> waves;     // run one after another; their workspace is shared
+  uint64_t inject_wait_ns = 0; // failure-detection test: consumed by the next call's first GEMM launch
   void* tmaps_d = nullptr;
   // Per-call pointer tables, kept resident on the device: a call whose
   // pointers match a kept table uses it with no copy.  A caller that
@@ -224,15 +238,20 @@ struct Recorder {
   bool on = false;
   Recorder(muon_plan_s* p, cudaStream_t s, int max_launches) : pl(p), st(s) {
     if (!pl->prof) return;
+    if (max_launches + 1 > static_cast<int>(pl->events.size())) pl->events.resize(max_launches + 1, nullptr);
+    for (auto& ev : pl->events)
+      if (ev == nullptr && cudaEventCreate(&ev) != cudaSuccess) return;
     if (pl->ev_next + max_launches + 1 > static_cast<int>(pl->events.size())) prof_flush(pl);
     rec.first_event = pl->ev_next;
     rec.nlaunch = 0;
+    rec.phases.reserve(max_launches);
     cudaEventRecord(pl->events[pl->ev_next++], st);
     on = true;
   }
   void mark(int phase) {
     if (!on) return;
-    rec.phases[rec.nlaunch++] = phase;
+    rec.phases.push_back(phase);
+    rec.nlaunch++;
     cudaEventRecord(pl->events[pl->ev_next++], st);
   }
   ~Recorder() {
@@ -241,60 +260,71 @@ struct Recorder {
 };
 
 // ------------------------------------------------------------ the launch sequence
+// The launch sequence of one call: for each wave, k1 over its chunks, the
+// Newton-Schulz launches over its tiles and the update pass over its chunks
+// (every matrix's arithmetic is the same whichever wave holds it), then the
+// RMS finalisation over all matrices.
 muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int precision, int final_mode,
                      int k1_mode, float* update_rms, cudaStream_t st) {
-  Recorder rec(pl, st, 3 * ns_steps + 4);
+  const int nwave = static_cast<int>(pl->waves.size());
+  Recorder rec(pl, st, nwave * (3 * ns_steps + 3) + 1);
   const int fp32 = precision == MUON_NS_FP32 ? 1 : 0;
-  cudaError_t e = launch_k1(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, k1_mode, fp32, st);
-  if (e != cudaSuccess) return MUON_ERR_CUDA;
-  rec.mark(0);
-  int cur = 0;
-  for (int it = 0; it < ns_steps; ++it) {
-    for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
-      if (fp32) {
-        Gemm32Args a{};
-        a.tiles = (ph == kPhaseUpdate) ? pl->full32_d : pl->sym32_d;
-        a.ntiles = (ph == kPhaseUpdate) ? pl->n_full32 : pl->n_sym32;
-        a.phase = ph;
-        a.iter = it;
-        a.cur = cur;
-        a.mats = pl->mats_d;
-        a.ptrs = pl->ptrs_d;
-        a.ws = pl->ws;
-        a.sc = sc;
-        e = launch_gemm_f32(a, st);
-      } else {
-        GemmArgs a{};
-        a.tiles = (ph == kPhaseUpdate) ? pl->full_d : pl->sym_d;
-        a.ntiles = (ph == kPhaseUpdate) ? pl->n_full : pl->n_sym;
-        a.phase = ph;
-        a.iter = it;
-        a.cur = cur;
-        a.mats = pl->mats_d;
-        a.ptrs = pl->ptrs_d;
-        a.tmaps = pl->tmaps_d;
-        a.ws = pl->ws;
-        a.sc = sc;
-        e = launch_gemm_tc(a, pl->npairs, st);
-      }
-      if (e != cudaSuccess) return MUON_ERR_CUDA;
-      rec.mark(1 + ph);
-    }
-    cur ^= 1;  // the X update wrote the other buffer
-  }
   // The last iterate is in hi[cur]/lo (x32[cur]); O = s X when N = 0.  Eq. 6
   // needs RMS(O) before any weight changes, so it adds a reduction pass.
   const int mul_s = ns_steps == 0 ? 1 : 0;
   const bool norm_pass = (final_mode == kFinalWeight && sc.scale_mode == kScaleUpdateNorm);
-  if (norm_pass) {
-    e = launch_update_norm(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ws, sc, fp32, cur, mul_s, update_rms, st);
+  cudaError_t e = cudaSuccess;
+  for (const Wave& w : pl->waves) {
+    const ChunkDesc* chunks = pl->chunks_d + w.chunk_off;
+    e = launch_k1(chunks, w.nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, k1_mode, fp32, st);
+    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    rec.mark(0);
+    int cur = 0;
+    for (int it = 0; it < ns_steps; ++it) {
+      for (int ph = kPhaseGram; ph <= kPhaseUpdate; ++ph) {
+        if (fp32) {
+          Gemm32Args a{};
+          a.tiles = (ph == kPhaseUpdate) ? pl->full32_d + w.full32_off : pl->sym32_d + w.sym32_off;
+          a.ntiles = (ph == kPhaseUpdate) ? w.n_full32 : w.n_sym32;
+          a.phase = ph;
+          a.iter = it;
+          a.cur = cur;
+          a.mats = pl->mats_d;
+          a.ptrs = pl->ptrs_d;
+          a.ws = pl->ws;
+          a.sc = sc;
+          e = launch_gemm_f32(a, st);
+        } else {
+          GemmArgs a{};
+          a.tiles = (ph == kPhaseUpdate) ? pl->full_d + w.full_off : pl->sym_d + w.sym_off;
+          a.ntiles = (ph == kPhaseUpdate) ? w.n_full : w.n_sym;
+          a.phase = ph;
+          a.iter = it;
+          a.cur = cur;
+          a.mats = pl->mats_d;
+          a.ptrs = pl->ptrs_d;
+          a.tmaps = pl->tmaps_d;
+          a.ws = pl->ws;
+          a.sc = sc;
+          a.test_wait_ns = pl->inject_wait_ns;
+          pl->inject_wait_ns = 0;
+          e = launch_gemm_tc(a, pl->npairs, st);
+        }
+        if (e != cudaSuccess) return MUON_ERR_CUDA;
+        rec.mark(1 + ph);
+      }
+      cur ^= 1;  // the X update wrote the other buffer
+    }
+    if (norm_pass) {
+      e = launch_update_norm(chunks, w.nchunks, pl->mats_d, pl->ws, sc, fp32, cur, mul_s, update_rms, st);
+      if (e != cudaSuccess) return MUON_ERR_CUDA;
+      rec.mark(4);
+    }
+    e = launch_apply_update(chunks, w.nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, final_mode, fp32, cur, mul_s,
+                            st);
     if (e != cudaSuccess) return MUON_ERR_CUDA;
     rec.mark(4);
   }
-  e = launch_apply_update(pl->chunks_d, pl->nchunks, pl->mats_d, pl->ptrs_d, pl->ws, sc, final_mode, fp32, cur,
-                          mul_s, st);
-  if (e != cudaSuccess) return MUON_ERR_CUDA;
-  rec.mark(4);
   if (update_rms != nullptr && !norm_pass) {
     e = launch_rms_finalize(pl->mats_d, pl->n, pl->ws.rms_part, update_rms, st);
     if (e != cudaSuccess) return MUON_ERR_CUDA;
@@ -310,7 +340,8 @@ void free_plan(muon_plan_s* pl) {
     if (sl.pinned) cudaFreeHost(sl.pinned);
     if (sl.ev) cudaEventDestroy(sl.ev);
   }
-  for (cudaEvent_t ev : pl->events) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : pl->events)
+    if (ev != nullptr) cudaEventDestroy(ev);
   delete pl;
 }
 
@@ -352,10 +383,19 @@ muon_status_t muon_hparams_default(muon_hparams_t* hp) {
 }
 
 muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags, void* stream) {
+  if (out != nullptr) *out = nullptr;
+  if (flags & MUON_INIT_MAX_WORKSPACE) return MUON_ERR_INVALID_ARG;  // the budget needs muon_init_ex
+  return muon_init_ex(out, params, n, flags, 0, stream);
+}
+
+muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t n, uint32_t flags,
+                           size_t max_workspace_bytes, void* stream) {
   if (out == nullptr) return MUON_ERR_INVALID_ARG;
   *out = nullptr;
   if (params == nullptr || n < 1 || n > (1 << 20)) return MUON_ERR_INVALID_ARG;
-  if (flags & ~(MUON_INIT_ZERO_MOMENTUM | MUON_INIT_FP32_NS)) return MUON_ERR_INVALID_ARG;
+  if (flags & ~(MUON_INIT_ZERO_MOMENTUM | MUON_INIT_FP32_NS | MUON_INIT_MAX_WORKSPACE)) return MUON_ERR_INVALID_ARG;
+  const bool capped = (flags & MUON_INIT_MAX_WORKSPACE) != 0;
+  if (capped != (max_workspace_bytes != 0)) return MUON_ERR_INVALID_ARG;
   for (int i = 0; i < n; ++i) {
     const muon_param_t& p = params[i];
     if (p.rows < 1 || p.cols < 1 || p.rows > kMaxDim || p.cols > kMaxDim || p.reserved != 0)
@@ -386,19 +426,8 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   pl->fp32_ws = (flags & MUON_INIT_FP32_NS) != 0;
   pl->mats.resize(n);
 
-  // ---- per-matrix layout and schedules
-  std::vector<TileDesc> sym, full, sym32, full32;
-  std::vector<ChunkDesc> chunks;
-  size_t total_x = 0, total_a = 0;
-  // LPT order of matrices for the GEMM schedules (largest Newton-Schulz work first)
-  std::vector<int> order(n);
-  for (int i = 0; i < n; ++i) order[i] = i;
-  auto work = [&](int i) {
-    const double m = static_cast<double>(std::min(params[i].rows, params[i].cols));
-    const double nn = static_cast<double>(std::max(params[i].rows, params[i].cols));
-    return m * m * nn + m * m * m;
-  };
-  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return work(x) > work(y); });
+  // ---- per-matrix shapes and workspace sizes (elements of the [R, ld] and [m, lda] arrays)
+  std::vector<size_t> xel(n), ael(n);
   for (int i = 0; i < n; ++i) {
     MatInfo& mi = pl->mats[i];
     const int R = static_cast<int>(params[i].rows), C = static_cast<int>(params[i].cols);
@@ -409,33 +438,169 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
     mi.tall = R > C ? 1 : 0;
     mi.ld = static_cast<int>(round_up(C, 8));
     mi.lda = static_cast<int>(round_up(mi.m, 8));
-    mi.off_x = static_cast<int64_t>(total_x);
-    total_x += round_up(static_cast<size_t>(R) * mi.ld, 128);
-    mi.off_a = static_cast<int64_t>(total_a);
-    total_a += round_up(static_cast<size_t>(mi.m) * mi.lda, 128);
-    const int rows_per_chunk = std::max(1, kChunkElems / C);
-    mi.chunk_base = static_cast<int>(chunks.size());
-    for (int r = 0; r < R; r += rows_per_chunk)
-      chunks.push_back(make_int4(i, r, std::min(rows_per_chunk, R - r), static_cast<int>(chunks.size())));
-    mi.nchunks = static_cast<int>(chunks.size()) - mi.chunk_base;
+    xel[i] = round_up(static_cast<size_t>(R) * mi.ld, 128);
+    ael[i] = round_up(static_cast<size_t>(mi.m) * mi.lda, 128);
   }
-  for (int i : order) {
+  // bytes per element of the iterate arrays (hi0, hi1, lo; + x32[2]) and of the
+  // symmetric arrays (A, B; + a32, b32)
+  const size_t bx = pl->fp32_ws ? 6 + 8 : 6, ba = pl->fp32_ws ? 4 + 8 : 4;
+  // LPT order of matrices (largest Newton-Schulz work first): the order of the
+  // GEMM schedules and of the wave packing
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  auto work = [&](int i) {
+    const double m = static_cast<double>(pl->mats[i].m), nn = static_cast<double>(pl->mats[i].n);
+    return m * m * nn + m * m * m;
+  };
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return work(x) > work(y); });
+
+  // ---- the small device structures every plan holds, whatever its waves
+  std::vector<TileDesc> sym, full, sym32, full32;
+  std::vector<ChunkDesc> chunks;
+  std::vector<int> wave_of(n, 0);
+  auto fixed_bytes = [&](size_t ntile_sym, size_t ntile_full, size_t ntile_sym32, size_t ntile_full32,
+                         size_t nchunk) {
+    size_t b = 0;
+    auto add = [&](size_t v) { b += round_up(v, 256); };
+    add(n * sizeof(float));                          // s
+    add(nchunk * sizeof(double));                    // norm partials
+    add(n * sizeof(unsigned));                       // arrival counters
+    add(nchunk * sizeof(float));                     // update partials
+    add(sizeof(unsigned));                           // status
+    add(n * sizeof(float));                          // Eq. 6 factors
+    add(n * sizeof(MatInfo));
+    add(muon_plan_s::kPtrSlots * n * sizeof(MatPtrs));
+    add(std::max<size_t>(1, ntile_sym) * sizeof(TileDesc));
+    add(std::max<size_t>(1, ntile_full) * sizeof(TileDesc));
+    add(std::max<size_t>(1, ntile_sym32) * sizeof(TileDesc));
+    add(std::max<size_t>(1, ntile_full32) * sizeof(TileDesc));
+    add(nchunk * sizeof(ChunkDesc));
+    add(static_cast<size_t>(n) * kMapsPerMat * sizeof(CUtensorMap));
+    return b;
+  };
+  // tile and chunk counts do not depend on the waves
+  size_t cnt_sym = 0, cnt_full = 0, cnt_sym32 = 0, cnt_full32 = 0, cnt_chunk = 0;
+  for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];
-    for_each_sym_tile(mi.m, [&](int r0, int c0, int need) { sym.push_back(make_int4(i, r0, c0, need)); });
-    for (int r0 = 0; r0 < mi.rows; r0 += kTileM)
-      for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
+    for_each_sym_tile(mi.m, [&](int, int, int) { ++cnt_sym; });
+    cnt_full += static_cast<size_t>((mi.rows + kTileM - 1) / kTileM) * ((mi.cols + kBN - 1) / kBN);
     if (pl->fp32_ws) {
-      for (int r0 = 0; r0 < mi.m; r0 += kT32)
-        for (int c0 = 0; c0 < mi.m; c0 += kT32) sym32.push_back(make_int4(i, r0, c0, 0));
-      for (int r0 = 0; r0 < mi.rows; r0 += kT32)
-        for (int c0 = 0; c0 < mi.cols; c0 += kT32) full32.push_back(make_int4(i, r0, c0, 0));
+      cnt_sym32 += static_cast<size_t>((mi.m + kT32 - 1) / kT32) * ((mi.m + kT32 - 1) / kT32);
+      cnt_full32 += static_cast<size_t>((mi.rows + kT32 - 1) / kT32) * ((mi.cols + kT32 - 1) / kT32);
     }
+    const int rows_per_chunk = std::max(1, kChunkElems / mi.cols);
+    cnt_chunk += (mi.rows + rows_per_chunk - 1) / rows_per_chunk;
+  }
+  const size_t fixed = fixed_bytes(cnt_sym, cnt_full, cnt_sym32, cnt_full32, cnt_chunk);
+
+  // ---- waves: with a workspace cap, matrices are packed first-fit in LPT
+  // order into waves whose iterate and symmetric arrays fit what the cap
+  // leaves after the fixed structures.  The arrays are shared by all waves and
+  // sized by the largest wave of each kind, so the packing is repeated with a
+  // tighter capacity until the total fits.
+  size_t X_total = 0, A_total = 0;
+  int nwave = 1;
+  if (!capped) {
+    for (int i = 0; i < n; ++i) {
+      X_total += xel[i];
+      A_total += ael[i];
+    }
+  } else {
+    const size_t slack = 6 * 256;  // alignment of the iterate and symmetric arrays
+    if (max_workspace_bytes <= fixed + slack) {
+      free_plan(pl);
+      return MUON_ERR_NO_MEMORY;
+    }
+    size_t cap = max_workspace_bytes - fixed - slack;
+    size_t biggest = 0;
+    for (int i = 0; i < n; ++i) biggest = std::max(biggest, bx * xel[i] + ba * ael[i]);
+    bool fits = false;
+    for (int attempt = 0; attempt < 64 && cap >= biggest; ++attempt) {
+      std::vector<size_t> wx, wa;
+      for (int i : order) {
+        const size_t need = bx * xel[i] + ba * ael[i];
+        int w = 0;
+        while (w < static_cast<int>(wx.size()) && bx * wx[w] + ba * wa[w] + need > cap) ++w;
+        if (w == static_cast<int>(wx.size())) {
+          wx.push_back(0);
+          wa.push_back(0);
+        }
+        wx[w] += xel[i];
+        wa[w] += ael[i];
+        wave_of[i] = w;
+      }
+      X_total = *std::max_element(wx.begin(), wx.end());
+      A_total = *std::max_element(wa.begin(), wa.end());
+      nwave = static_cast<int>(wx.size());
+      const size_t total = bx * X_total + ba * A_total;
+      if (total <= max_workspace_bytes - fixed - slack) {
+        fits = true;
+        break;
+      }
+      const size_t over = total - (max_workspace_bytes - fixed - slack);
+      cap = cap > over ? cap - over : 0;
+    }
+    if (!fits) {
+      free_plan(pl);
+      return MUON_ERR_NO_MEMORY;
+    }
+  }
+
+  // ---- per-wave offsets, chunk lists and tile schedules (LPT order inside a wave)
+  pl->waves.assign(nwave, Wave{});
+  {
+    std::vector<size_t> xoff(nwave, 0), aoff(nwave, 0);
+    for (int i = 0; i < n; ++i) {  // descriptor order inside a wave
+      MatInfo& mi = pl->mats[i];
+      const int w = wave_of[i];
+      mi.off_x = static_cast<int64_t>(xoff[w]);
+      mi.off_a = static_cast<int64_t>(aoff[w]);
+      xoff[w] += xel[i];
+      aoff[w] += ael[i];
+      pl->waves[w].nmat += 1;
+    }
+  }
+  for (int w = 0; w < nwave; ++w) {
+    Wave& wv = pl->waves[w];
+    wv.chunk_off = static_cast<int>(chunks.size());
+    for (int i = 0; i < n; ++i) {  // descriptor order inside a wave
+      if (wave_of[i] != w) continue;
+      MatInfo& mi = pl->mats[i];
+      const int rows_per_chunk = std::max(1, kChunkElems / mi.cols);
+      mi.chunk_base = static_cast<int>(chunks.size());
+      for (int r = 0; r < mi.rows; r += rows_per_chunk)
+        chunks.push_back(make_int4(i, r, std::min(rows_per_chunk, mi.rows - r), static_cast<int>(chunks.size())));
+      mi.nchunks = static_cast<int>(chunks.size()) - mi.chunk_base;
+    }
+    wv.nchunks = static_cast<int>(chunks.size()) - wv.chunk_off;
+    wv.sym_off = static_cast<int>(sym.size());
+    wv.full_off = static_cast<int>(full.size());
+    wv.sym32_off = static_cast<int>(sym32.size());
+    wv.full32_off = static_cast<int>(full32.size());
+    for (int i : order) {
+      if (wave_of[i] != w) continue;
+      const MatInfo& mi = pl->mats[i];
+      for_each_sym_tile(mi.m, [&](int r0, int c0, int need) { sym.push_back(make_int4(i, r0, c0, need)); });
+      for (int r0 = 0; r0 < mi.rows; r0 += kTileM)
+        for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
+      if (pl->fp32_ws) {
+        for (int r0 = 0; r0 < mi.m; r0 += kT32)
+          for (int c0 = 0; c0 < mi.m; c0 += kT32) sym32.push_back(make_int4(i, r0, c0, 0));
+        for (int r0 = 0; r0 < mi.rows; r0 += kT32)
+          for (int c0 = 0; c0 < mi.cols; c0 += kT32) full32.push_back(make_int4(i, r0, c0, 0));
+      }
+    }
+    wv.n_sym = static_cast<int>(sym.size()) - wv.sym_off;
+    wv.n_full = static_cast<int>(full.size()) - wv.full_off;
+    wv.n_sym32 = static_cast<int>(sym32.size()) - wv.sym32_off;
+    wv.n_full32 = static_cast<int>(full32.size()) - wv.full32_off;
   }
   pl->n_sym = static_cast<int>(sym.size());
   pl->n_full = static_cast<int>(full.size());
   pl->n_sym32 = static_cast<int>(sym32.size());
   pl->n_full32 = static_cast<int>(full32.size());
   pl->nchunks = static_cast<int>(chunks.size());
+  const size_t total_x = X_total, total_a = A_total;
 
   // ---- carve one device allocation
   size_t off = 0;
@@ -469,6 +634,10 @@ muon_status_t muon_init(muon_plan_t* out, const muon_param_t* params, int32_t n,
   const size_t o_chunks = take(chunks.size() * sizeof(ChunkDesc));
   const size_t o_tmaps = take(static_cast<size_t>(n) * kMapsPerMat * sizeof(CUtensorMap));
   pl->dbytes = off;
+  if (capped && pl->dbytes > max_workspace_bytes) {  // the packing above accounts for every byte
+    free_plan(pl);
+    return MUON_ERR_NO_MEMORY;
+  }
   if (cudaMalloc(&pl->dmem, pl->dbytes) != cudaSuccess) {
     cudaGetLastError();
     free_plan(pl);
@@ -646,6 +815,14 @@ muon_status_t muon_orthogonalize(muon_plan_t pl, const void* const* X_in, float*
 }
 
 size_t muon_workspace_bytes(muon_plan_t pl) { return pl == nullptr ? 0 : pl->dbytes; }
+
+muon_status_t muon_inject_wait_timeout(muon_plan_t pl, uint32_t wait_ns) {
+  if (pl == nullptr || wait_ns < 1 || wait_ns > 1000000000u) return MUON_ERR_INVALID_ARG;
+  pl->inject_wait_ns = wait_ns;
+  return MUON_OK;
+}
+
+int32_t muon_num_waves(muon_plan_t pl) { return pl == nullptr ? -1 : static_cast<int32_t>(pl->waves.size()); }
 
 muon_status_t muon_get_status(muon_plan_t pl) {
   if (pl == nullptr) return MUON_ERR_INVALID_ARG;

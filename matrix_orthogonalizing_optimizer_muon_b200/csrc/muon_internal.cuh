@@ -175,6 +175,7 @@ struct GemmArgs {
   const void* tmaps;    // CUtensorMap[kMapsPerMat * nmat], see MapIndex
   Workspace ws;
   StepScalars sc;
+  unsigned long long test_wait_ns;  // 0; > 0 only for the failure-detection test (see muon_inject_wait_timeout)
 };
 
 // Arguments of the fp32 SIMT GEMM kernel.

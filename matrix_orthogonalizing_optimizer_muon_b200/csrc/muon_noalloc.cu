@@ -9,15 +9,19 @@
 // Gram and polynomial matrices, norms, schedules, TMA descriptors) lives in
 // one file-scope device array of fixed size, which every GPU that loads the
 // library holds until the process exits.  The caller passes the input and the
-// output; the per-call descriptors are copied in from the host stack.
+// output; the per-call descriptors are copied in from the host stack, so the
+// call returns only once the driver has staged those (pageable) copies, and a
+// stream that is being captured is refused.
 #include "muon.h"
 #include "muon_internal.cuh"
 
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 using namespace muon;
 
@@ -60,28 +64,39 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 struct DeviceState {
   unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
   int npairs = 0;
-  bool ready = false;
+  bool sm100 = false;             // compute capability 10.0
+  std::atomic<bool> ready{false};
 };
 DeviceState g_state[64];
+std::mutex g_setup_mutex;  // first calls from several host threads set a device up once
 
 // Once per device, with that device current: resolve the scratch array's
-// device address (in host code the symbol's name is only a host-side stand-in).
+// device address (in host code the symbol's name is only a host-side stand-in)
+// and read the device's compute capability and persistent grid size.
 muon_status_t setup_device(int dev) {
   DeviceState& st = g_state[dev];
-  if (st.ready) return MUON_OK;
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+  if (st.ready.load(std::memory_order_acquire)) return MUON_OK;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (st.ready.load(std::memory_order_relaxed)) return MUON_OK;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
-  st.base = static_cast<unsigned char*>(p);
-  st.npairs = gemm_tc_max_pairs();
-  if (st.npairs < 1) {
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
-    st.npairs = std::max(1, prop.multiProcessorCount / 2);
+  st.sm100 = (major == 10 && minor == 0);
+  if (st.sm100) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return MUON_ERR_CUDA;
+    }
+    st.base = static_cast<unsigned char*>(p);
+    st.npairs = gemm_tc_max_pairs();
+    if (st.npairs < 1) st.npairs = std::max(1, sms / 2);
   }
-  st.ready = true;
+  st.ready.store(true, std::memory_order_release);
   return MUON_OK;
 }
 
@@ -103,13 +118,20 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MUON_ERR_CUDA;
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MUON_ERR_CUDA;
-  if (prop.major != 10 || prop.minor != 0) return MUON_ERR_UNSUPPORTED;
   muon_status_t su = setup_device(dev);
   if (su != MUON_OK) return su;
+  if (!g_state[dev].sm100) return MUON_ERR_UNSUPPORTED;
   unsigned char* base = g_state[dev].base;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The descriptors below are copied from this call's stack frame; a stream
+  // capture would record copies that read that frame again at replay, long
+  // after it is gone.  Refuse a capturing stream before enqueuing anything.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  if (cap != cudaStreamCaptureStatusNone) return MUON_ERR_UNSUPPORTED;
 
   // ---- one matrix: descriptors built on the host stack
   const int R = static_cast<int>(rows), C = static_cast<int>(cols);

@@ -99,6 +99,44 @@ def test_init_rejects_bad_arguments_before_any_cuda_call(lib):
     assert plan.value is None
 
 
+def test_init_ex_flag_and_budget_must_agree(lib):
+    plan = ctypes.c_void_p()
+    arr = (L.muon_param_t * 1)()
+    arr[0].rows, arr[0].cols = 4, 4
+    # the cap flag needs a budget, a budget needs the flag, muon_init takes no cap
+    assert lib.muon_init_ex(ctypes.byref(plan), arr, 1, L.MUON_INIT_MAX_WORKSPACE, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init_ex(ctypes.byref(plan), arr, 1, 0, 1 << 30, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init(ctypes.byref(plan), arr, 1, L.MUON_INIT_MAX_WORKSPACE, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_init_ex(None, arr, 1, 0, 0, None) == L.MUON_ERR_INVALID_ARG
+    assert plan.value is None
+    assert lib.muon_num_waves(None) == -1
+    m = __import__("re").search(r"MUON_INIT_MAX_WORKSPACE\s+(0x[0-9a-fA-F]+)u",
+                                open(os.path.join(ROOT, "include", "muon.h")).read())
+    assert m and int(m.group(1), 16) == L.MUON_INIT_MAX_WORKSPACE
+
+
+def test_pack_init_rejects_bad_segments_before_any_cuda_call(lib):
+    plan = ctypes.c_void_p()
+    segs = (L.muon_segment_t * 2)()
+    segs[0].src, segs[0].dst, segs[0].numel = 0x10000, 0x20000, 100
+    segs[1].src, segs[1].dst, segs[1].numel = 0x30000, 0x40000, 100
+    assert lib.muon_pack_init(None, segs, 2, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_pack_init(ctypes.byref(plan), None, 2, None) == L.MUON_ERR_INVALID_ARG
+    assert lib.muon_pack_init(ctypes.byref(plan), segs, 0, None) == L.MUON_ERR_INVALID_ARG
+    segs[1].dst_dtype = 5
+    assert lib.muon_pack_init(ctypes.byref(plan), segs, 2, None) == L.MUON_ERR_INVALID_ARG
+    segs[1].dst_dtype = L.MUON_DT_FP32
+    segs[1].dst = 0x20000 + 100          # inside the first destination (100 bf16 = 200 bytes)
+    assert lib.muon_pack_init(ctypes.byref(plan), segs, 2, None) == L.MUON_ERR_ALIAS
+    segs[1].dst = 0x10000 + 8            # over the first source
+    assert lib.muon_pack_init(ctypes.byref(plan), segs, 2, None) == L.MUON_ERR_ALIAS
+    segs[1].numel = 0
+    assert lib.muon_pack_init(ctypes.byref(plan), segs, 2, None) == L.MUON_ERR_INVALID_ARG
+    assert plan.value is None
+    assert lib.muon_pack_run(None, None) == L.MUON_ERR_INVALID_ARG
+    lib.muon_pack_destroy(None)
+
+
 def test_null_plan_calls(lib):
     hp = L.muon_hparams_default()
     arr = (L.muon_param_t * 1)()

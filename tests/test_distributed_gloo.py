@@ -14,7 +14,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle.muon_oracle as orc
-from matrix_orthogonalizing_optimizer_muon_b200.distributed import DistributedMuon, assign_owners, ns_work
+from matrix_orthogonalizing_optimizer_muon_b200.distributed import DistributedMuon, assign_owners, assign_waves, ns_work
 
 SHAPES = [(24, 40), (40, 24), (16, 16), (8, 64), (33, 17)]
 LR, WD, MU = 0.05, 0.1, 0.95
@@ -49,11 +49,11 @@ def weights():
     return [torch.randn(s, generator=g) * 0.02 for s in SHAPES]
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, waves=2):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        opt = DistributedMuon(SHAPES, local_step=oracle_local_step, device="cpu")
+        opt = DistributedMuon(SHAPES, local_step=oracle_local_step, device="cpu", waves=waves)
         Ws = weights()
         rms = None
         for t in range(STEPS):
@@ -63,12 +63,13 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_ranks_match_a_single_process_step_on_the_summed_gradient():
+@pytest.mark.parametrize("waves", [1, 2, 3])
+def test_two_ranks_match_a_single_process_step_on_the_summed_gradient(waves):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, waves)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted((q.get(timeout=300) for _ in range(world)), key=lambda x: x[0])
@@ -97,6 +98,21 @@ def test_owner_assignment_is_balanced_and_deterministic():
         assert a == assign_owners(list(shapes), world)
         load = [sum(ns_work(s) for s, r in zip(shapes, a) if r == k) for k in range(world)]
         assert max(load) - min(load) <= max(ns_work(s) for s in shapes)
+
+
+def test_waves_split_each_rank_evenly_and_deterministically():
+    shapes = [(2048, 1408)] * 9 + [(1408, 2048)] * 6 + [(512, 512)] * 4 + [(2048, 64)] * 3
+    for world in (1, 2, 4):
+        owner = assign_owners(shapes, world)
+        for waves in (1, 2, 3):
+            w = assign_waves(shapes, owner, world, waves)
+            assert w == assign_waves(list(shapes), list(owner), world, waves)
+            assert all(0 <= k < waves for k in w)
+            for r in range(world):
+                load = [sum(ns_work(s) for s, o, k in zip(shapes, owner, w) if o == r and k == j) for j in range(waves)]
+                mine = [ns_work(s) for s, o in zip(shapes, owner) if o == r]
+                if mine:
+                    assert max(load) - min(load) <= max(mine)
 
 
 SHAPES3 = [(24, 40), (8, 64)]

@@ -13,6 +13,8 @@ import oracle.adamw_oracle as ado
 from matrix_orthogonalizing_optimizer_muon_b200 import _lib as L
 from matrix_orthogonalizing_optimizer_muon_b200.api import AdamWPlan
 
+from _gpu import check_adamw
+
 pytestmark = pytest.mark.gpu
 
 # ragged sizes across the 65536-element chunks; one fp32 gradient; decay off on two
@@ -44,21 +46,8 @@ def _tensors(seed, misaligned=False):
 
 
 def _check(P0, m0, v0, G, P1, m1, v1, step, decay):
-    b1, b2 = F32(BETAS[0]), F32(BETAS[1])
-    r = ado.adamw_step(P0, G, m0, v0, step=step, lr=F32(LR), weight_decay=F32(WD), betas=(b1, b2), eps=F32(EPS),
-                       decay=decay)
-    # fp32 arithmetic: each moment is one product and one fused multiply-add
-    tol_m = 3 * U * (np.abs(r.m) + (1 - b1) * np.abs(G)) + 1e-38
-    tol_v = 3 * U * (np.abs(r.v) + (1 - b2) * G * G) + 1e-38
-    assert np.all(np.abs(m1 - r.m) <= tol_m)
-    assert np.all(np.abs(v1 - r.v) <= tol_v)
-    bc1, bc2 = 1 - b1 ** step, 1 - b2 ** step
-    den = np.sqrt(r.v / bc2) + F32(EPS)
-    tol_u = tol_m / bc1 / den + np.abs(r.update) * (0.5 * tol_v / np.maximum(r.v, 1e-300) + 8 * U)
-    wd = F32(WD) if decay else 0.0
-    tol_p = 2 * U * np.abs(r.P) + F32(LR) * (tol_u + 2 * U * (np.abs(r.update) + wd * np.abs(P0)))
-    err = np.abs(P1 - r.P)
-    assert np.all(err <= tol_p), float(np.max(err / tol_p))
+    check_adamw(P0, m0, v0, G, P1, m1, v1, step=step, lr=F32(LR), wd=F32(WD), betas=(F32(BETAS[0]), F32(BETAS[1])),
+                eps=F32(EPS), decay=decay)
 
 
 @pytest.mark.parametrize("misaligned", [False, True])

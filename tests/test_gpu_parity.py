@@ -15,8 +15,9 @@ import oracle.muon_oracle as orc
 from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
 from matrix_orthogonalizing_optimizer_muon_b200.api import MuonPlan
 
-from _gpu import (ABC32, LR, MU, TOL_O_BF16, TOL_O_FP32, WD, bf16_cuda, check_step, f32, host64, random_bf16,
-                  rel_f)
+from _gpu import (ABC32, LR, MU, TOL_O_BF16, TOL_O_FP32, WD, assert_step_errors, bf16_cuda, check_step, f32, host32,
+                  host64, random_bf16, rel_f)
+from _oracle_pool import OraclePool
 
 pytestmark = pytest.mark.gpu
 
@@ -136,33 +137,32 @@ def test_zero_gradient_matrix_is_pure_decay():
     assert float(rms[1]) > 0
 
 
-def _moe_sample():
-    wl = wlm.moe_experts()
-    zero = sorted(wl.zero_grad)
-    rng = np.random.default_rng(4)
-    nonzero = [i for i in range(wl.n) if i not in wl.zero_grad]
-    picks = sorted(set(rng.choice(nonzero, size=6, replace=False).tolist()) | {zero[0], 0, wl.n - 1})
-    return wl, picks
-
-
-def test_moe_expert_batch_full_size_sampled():
+def test_moe_expert_batch_full_size_every_matrix():
     """The 64+2-expert batch (198 matrices, one grouped call, the launch
-    configuration the benchmark times); momentum checked everywhere, W on a
-    seeded sample of matrices including an unrouted one."""
-    wl, picks = _moe_sample()
+    configuration the benchmark times): W, M, O and the update RMS of every
+    matrix, the 18 unrouted ones included, against the oracle."""
+    wl = wlm.moe_experts()
     shapes = [(r, c) for _, r, c in wl.shapes]
     Ws = [torch.from_numpy(wlm.weight(wl, i)).cuda() for i in range(wl.n)]
     Gs = [bf16_cuda(wlm.grad_bf16(wl, i, 0)) for i in range(wl.n)]
     Ms = [torch.empty(s, device="cuda") for s in shapes]
     plan = MuonPlan(shapes, momenta=Ms)
     rms = torch.zeros(wl.n, device="cuda")
-    W_prev = {i: host64(Ws[i]) for i in picks}
     plan.step(list(zip(Ws, Gs, Ms)), lr=LR, weight_decay=WD, momentum=MU, coeffs=ABC32, update_rms=rms)
     torch.cuda.synchronize()
     assert plan.status() == 0
-    for i in range(wl.n):
-        G64 = host64(Gs[i])
-        assert rel_f(host64(Ms[i]), G64) <= 1e-6 if G64.any() else not host64(Ms[i]).any()
-    for i in picks:
-        check_step(W_prev[i], np.zeros(shapes[i]), host64(Gs[i]), host64(Ws[i]), host64(Ms[i]), float(rms[i]),
-                   lr=LR, wd=WD, mu=MU)
+    rms_h = rms.cpu().numpy()
+    with OraclePool() as pool:
+        for i in range(wl.n):
+            pool.submit_step(i, wlm.weight(wl, i), np.zeros(shapes[i], np.float32),
+                             wlm.bf16_bits_to_f32(wlm.grad_bf16(wl, i, 0)), host32(Ws[i]), host32(Ms[i]),
+                             float(rms_h[i]), lr=LR, wd=WD, mu=MU, coeffs=ABC32)
+        res = pool.drain()
+    assert sorted(r["key"] for r in res) == list(range(wl.n))
+    for r in res:
+        assert_step_errors(r)
+    nz = [r for r in res if r["key"] not in wl.zero_grad]
+    worst = {"O": max(r["O"] for r in nz), "dW/bound": max(r["dW"] / r["dW_bound"] for r in res),
+             "M": max(r["M"] for r in res), "rms": max(r["rms"] for r in nz)}
+    print("moe worst", worst)
+    plan.close()
