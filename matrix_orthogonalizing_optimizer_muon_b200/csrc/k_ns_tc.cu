@@ -4,11 +4,14 @@
 // for LLM Training", Sec. 2.1, Eq. 2, factored as A = X X^T, B = b A + c A^2,
 // X' = a X + B X) for every matrix of the plan:
 //   kPhaseGram   A  = scale * X X^T         (wide)   or Y^T Y (tall)  [m, m]
-//   kPhasePoly   B  = b A + c A A            (A symmetric, so A A = A A^T)
-//   kPhaseUpdate X' = alpha (a X + B X)      (wide)   or Y' = alpha (a Y + Y B) (tall)
-// with scale = s^2 and alpha = s on iteration 0 (s = 1/||Y||_F folds the
-// normalisation X_0 = Y/||Y||_F into the first products), 1 afterwards.  The
-// weight update of Eq. 4 is a separate elementwise pass over the last iterate.
+//   kPhasePoly   B' = b A + c A A + a I      (A symmetric, so A A = A A^T)
+//   kPhaseUpdate X' = alpha (B' hi + a lo)   (wide)   or Y' = alpha (hi B' + a lo) (tall)
+// with X = hi + lo the bf16 pair of the iterate, so that X' = alpha (a X + B hi):
+// the a X term of Eq. 2 rides on the product, and the epilogue adds only the
+// a lo part.  scale = s^2 and alpha = s on iteration 0 (s = 1/||Y||_F folds
+// the normalisation X_0 = Y/||Y||_F into the first products), 1 afterwards.
+// The weight update of Eq. 4 is a separate elementwise pass over the last
+// iterate.
 //
 // Structure: persistent 2-CTA clusters (one CTA per SM).  A pair owns a
 // 256 x 256 output tile; tcgen05.mma.cta_group::2 (M = 256, N <= 256, K = 16,
@@ -16,8 +19,8 @@
 // from each CTA's shared memory, so each SM streams 32 KiB per 64-deep K
 // stage for 8.4 MFLOP of the pair.  The operand stream is latency bound (a
 // stage takes about two stage-times of MMA to arrive), so the ring is as deep
-// as shared memory allows: 6 stages for the Gram and polynomial phases, 4 for
-// the X update, whose epilogue also stages its hi/lo inputs.  Per CTA:
+// as shared memory allows: 6 stages for the Gram and polynomial phases, 5 for
+// the X update, whose epilogue also stages its lo inputs.  Per CTA:
 //   warps 0, 10 TMA producers taking alternate stage fills: up to four lanes
 //               issue one box each per stage in a single instruction (a
 //               64 x 128 K-major box, or 64 x 64 boxes for MN-major operands
@@ -31,7 +34,7 @@
 //               and the fused arithmetic.  Results go through a warp-private
 //               swizzled staging block to TMA bulk stores, so the load/store
 //               units and the L1 path stay free for the inputs (the X
-//               update's hi/lo via a per-warp cp.async ring).
+//               update's lo blocks via a per-warp cp.async ring).
 #include "muon_internal.cuh"
 
 #include <cuda.h>
@@ -43,7 +46,7 @@ namespace {
 #define MUON_TC_STAGES_SYM 6
 #endif
 #ifndef MUON_TC_STAGES_UPD
-#define MUON_TC_STAGES_UPD 4
+#define MUON_TC_STAGES_UPD 5
 #endif
 constexpr int kStagesSym = MUON_TC_STAGES_SYM;  // stages of the Gram and polynomial phases
 constexpr int kStagesUpd = MUON_TC_STAGES_UPD;  // stages of the X-update phase
@@ -63,6 +66,9 @@ constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;      // 32 KiB
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
 // Producer warps: warp 0 and the warps after the epilogue; fill f of the
 // stage ring goes to producer f mod kProducers.
+#ifndef MUON_TC_PF_DIST
+#define MUON_TC_PF_DIST 0
+#endif
 #ifndef MUON_TC_PRODUCERS
 #define MUON_TC_PRODUCERS 2
 #endif
@@ -70,10 +76,12 @@ constexpr int kProducers = MUON_TC_PRODUCERS;
 constexpr int kWarpProducer2 = kWarpEpi0 + kEpiWarps;  // first of the extra producer warps
 constexpr int kThreads = 32 * (kWarpProducer2 + kProducers - 1);
 
-// X-update inputs: per warp a ring of 2 buffers, each a 32 x 32 hi block and
-// lo block (4 KiB), filled by cp.async two chunks ahead.
+// X-update input: per warp a ring of 2 buffers, each the 32 x 32 lo block
+// (2 KiB) of the iterate, filled by cp.async two chunks ahead.  The a X term
+// needs no hi block: the polynomial phase writes B' = B + a I, so the
+// product B' hi already holds a hi and the epilogue adds a lo.
 constexpr int kUpdBufs = 2;
-constexpr int kUpdBufBytes = 2 * kEpiBlockBytes;
+constexpr int kUpdBufBytes = kEpiBlockBytes;
 
 struct SmemLayout {
   static constexpr int kStages = 0;                                   // stage s at s * kStageBytes
@@ -183,6 +191,12 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* tmap, in
       "%3}], [%4];" ::"r"(dst),
       "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
+}
+
+// L2 prefetch of one box (no shared memory, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_l2(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+               : "memory");
 }
 
 // Bring a tensor map into the TMA descriptor cache ahead of its first use.
@@ -305,30 +319,38 @@ __device__ __forceinline__ Operand make_operand(const GemmArgs& g, int p, int ma
   return o;
 }
 
-__device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) {
-  const TileDesc d = g.tiles[t];
+// What a role needs to know of a tile before it can work on it: the tile
+// entry, its matrix's m, n and orientation, and whether the matrix is skipped
+// (Y = 0) in this call.  Loaded ahead (see HeadPipe) so that the dependent
+// global loads do not stall the producer or the MMA issuer between tiles.
+struct TileHead {
+  TileDesc d;
+  int m, n, tall;
+  float s;
+};
+
+__device__ __forceinline__ TileCfg make_cfg(const GemmArgs& g, const TileHead& h) {
   TileCfg c;
-  c.p = d.x;
-  c.row0 = d.y;
-  c.col0 = d.z;
-  c.n_need = d.w;
+  c.p = h.d.x;
+  c.row0 = h.d.y;
+  c.col0 = h.d.z;
+  c.n_need = h.d.w;
   c.n_mma = (c.n_need + 31) & ~31;
   c.half = c.n_mma >> 1;
   c.nch = (c.n_need + kEpiBoxCols - 1) / kEpiBoxCols;
-  const MatInfo& mi = g.mats[c.p];
   const int hi = kMapHi0 + g.cur;
   int K;
   if (g.phase == kPhaseGram) {
-    K = mi.n;
-    c.a = make_operand(g, c.p, hi, mi.tall, kHalfM);
-    c.b = make_operand(g, c.p, hi, mi.tall, c.half);
+    K = h.n;
+    c.a = make_operand(g, c.p, hi, h.tall, kHalfM);
+    c.b = make_operand(g, c.p, hi, h.tall, c.half);
   } else if (g.phase == kPhasePoly) {
-    K = mi.m;
+    K = h.m;
     c.a = make_operand(g, c.p, kMapA, 0, kHalfM);
     c.b = make_operand(g, c.p, kMapA, 0, c.half);
   } else {
-    K = mi.m;
-    if (mi.tall) {
+    K = h.m;
+    if (h.tall) {
       c.a = make_operand(g, c.p, hi, 0, kHalfM);
       c.b = make_operand(g, c.p, kMapB, 0, c.half);
     } else {
@@ -337,9 +359,47 @@ __device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) {
     }
   }
   c.nk = (K + kBK - 1) / kBK;
-  c.skip = (g.ws.s[c.p] == 0.0f) ? 1 : 0;
+  c.skip = (h.s == 0.0f) ? 1 : 0;
   return c;
 }
+
+__device__ __forceinline__ TileHead load_head(const GemmArgs& g, const TileDesc& d) {
+  TileHead h;
+  h.d = d;
+  const MatInfo* mi = g.mats + d.x;
+  h.m = mi->m;
+  h.n = mi->n;
+  h.tall = mi->tall;
+  h.s = g.ws.s[d.x];
+  return h;
+}
+
+__device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) { return make_cfg(g, load_head(g, g.tiles[t])); }
+
+// Two-deep prefetch of the tiles a pair visits (t, t + npairs, ...): while a
+// role works on tile t, the entry of tile t + 2 npairs and the matrix fields
+// of tile t + npairs are in flight, so advancing is free of load latency.
+struct HeadPipe {
+  TileHead cur, nxt;
+  TileDesc nn;
+  int t, step, ntiles;
+
+  __device__ __forceinline__ void start(const GemmArgs& g, int t0, int stride) {
+    t = t0;
+    step = stride;
+    ntiles = g.ntiles;
+    if (t < ntiles) cur = load_head(g, g.tiles[t]);
+    if (t + step < ntiles) nxt = load_head(g, g.tiles[t + step]);
+    if (t + 2 * step < ntiles) nn = g.tiles[t + 2 * step];
+  }
+  __device__ __forceinline__ bool valid() const { return t < ntiles; }
+  __device__ __forceinline__ void advance(const GemmArgs& g) {
+    t += step;
+    cur = nxt;
+    if (t + step < ntiles) nxt = load_head(g, nn);
+    if (t + 2 * step < ntiles) nn = g.tiles[t + 2 * step];
+  }
+};
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned* status) {
   *abort_flag = 1;
@@ -509,9 +569,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // lanes the B boxes, all in one instruction; lane 0 owns the barriers.
     const int pp = (warp == kWarpProducer) ? 0 : warp - kWarpProducer2 + 1;
     long fills = 0;  // fills of all producers, in order
-    for (int t = pair; t < g.ntiles; t += npairs) {
+    HeadPipe hp;
+    for (hp.start(g, pair, npairs); hp.valid(); hp.advance(g)) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-      const TileCfg c = decode_tile(g, t);
+      const TileCfg c = make_cfg(g, hp.cur);
       if (c.skip) continue;
       const uint32_t bytes =
           static_cast<uint32_t>(2 * (c.a.nbox * c.a.box_bytes + c.b.nbox * c.b.box_bytes));
@@ -546,6 +607,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int mn0 = (is_a ? arow : brow) + h * kBoxInner;
           const uint32_t dst = (is_a ? sa : sb) + h * kBox64Bytes;
           tma_load_pair(dst, o.tmap, o.mn ? mn0 : k0, o.mn ? k0 : mn0 - h * kBoxInner, fb);
+#if MUON_TC_PF_DIST > 0
+          // bring the box MUON_TC_PF_DIST stages ahead into L2, so that its load
+          // later finds it there rather than in HBM
+          if (kb + MUON_TC_PF_DIST < c.nk) {
+            const int kp = k0 + MUON_TC_PF_DIST * kBK;
+            tma_prefetch_l2(o.tmap, o.mn ? mn0 : kp, o.mn ? kp : mn0 - h * kBoxInner);
+          }
+#endif
         }
       }
       if (!ok) break;
@@ -568,8 +637,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int t = pair; t < g.ntiles && !*abort_flag; t += npairs) {
-        const TileCfg c = decode_tile(g, t);
+      HeadPipe hp;
+      for (hp.start(g, pair, npairs); hp.valid() && !*abort_flag; hp.advance(g)) {
+        const TileCfg c = make_cfg(g, hp.cur);
         if (c.skip) continue;
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
           raise_abort(abort_flag, status);
@@ -660,9 +730,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int i = i_lo + lane;
       const bool upd = (g.phase == kPhaseUpdate);
       const bool sym = !upd;
-      // inputs the epilogue reads: A (polynomial) or the hi/lo iterate (X update)
-      const __nv_bfloat16* in0 = upd ? g.ws.hi[g.cur] + mi.off_x : g.ws.A + mi.off_a;
-      const __nv_bfloat16* in1 = g.ws.lo + mi.off_x;
+      // input the epilogue reads: A (polynomial) or the lo part of the iterate (X update)
+      const __nv_bfloat16* in0 = upd ? g.ws.lo + mi.off_x : g.ws.A + mi.off_a;
       const int ld_in = upd ? mi.ld : mi.lda;
       const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
       const bool poly = (g.phase == kPhasePoly);
@@ -681,8 +750,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!poly || !needed(ch) || !block_inside(ch)) return;
         load_block32(in0, ld_in, i_lo, c.col0 + ch * kEpiBoxCols, lane, pf0);
       };
-      // X update: ring of kUpdBufs (hi, lo) buffers fed by cp.async; chunk k
-      // of this warp lives in buffer k % kUpdBufs
+      // X update: ring of kUpdBufs lo buffers fed by cp.async; chunk k of
+      // this warp lives in buffer k % kUpdBufs
       auto upd_buf = [&](int b) -> uint8_t* {
         return smem + SmemLayout::kUpdRing + (ew * kUpdBufs + b) * kUpdBufBytes;
       };
@@ -692,9 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto stage_chunk = [&](int k) {
         const int chh = grp + k * kEpiGroups;
         if (block_inside(chh)) {
-          uint8_t* b = upd_buf(k % kUpdBufs);
-          cp_block32(b, in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
-          cp_block32(b + kEpiBlockBytes, in1, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
+          cp_block32(upd_buf(k % kUpdBufs), in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
         }
         cp_async_commit();  // one group per chunk, empty for ragged chunks
       };
@@ -723,17 +790,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         __syncwarp();
         tmem_ld32(t_row + static_cast<uint32_t>(ch * kEpiBoxCols), v);  // completes at tmem_ld_wait
-        uint4 xa[4], xb[4];  // this thread's row of the inputs, packed bf16
+        uint4 xa[4];  // this thread's row of the input (A, or lo), packed bf16
         if (upd) {
           if (inside) {
             cp_async_wait(issued - k - 1);
             __syncwarp();
             read_row32(upd_buf(k % kUpdBufs), lane, xa);
-            read_row32(upd_buf(k % kUpdBufs) + kEpiBlockBytes, lane, xb);
             __syncwarp();
           } else {
             load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
-            load_row32_masked(in1, ld_in, rows_in, cols_in, i, j0, xb);
           }
           // this buffer is free again: fetch the chunk two ahead into it
           if (issued < kc) {
@@ -759,12 +824,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
         } else if (poly) {
+          // B' = b A + c A A + a I (the a X term of the update rides on B' hi)
 #pragma unroll
-          for (int q = 0; q < 32; ++q) val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q));
+          for (int q = 0; q < 32; ++q)
+            val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q)) + (j0 + q == i ? a_c : 0.0f);
         } else {
+          // X' = alpha (B' hi + a lo) = alpha (a X + B hi)
           const float alpha = (g.iter == 0) ? s : 1.0f;
 #pragma unroll
-          for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q) + bf_at(xb, q), u2f(v[q]));
+          for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q), u2f(v[q]));
         }
         if (sym) {
           __align__(16) __nv_bfloat16 h[32];

@@ -21,7 +21,7 @@ from _gpu import ABC32, LR, MU, WD, check_step, host64
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(256, 128), (300, 520), (520, 300), (1408, 2048), (2048, 1408), (7, 1), (2048, 64)]
+SHAPES = [(256, 128), (300, 520), (520, 300), (1408, 2048), (2048, 1408), (33, 17), (2048, 64)]
 
 
 def _port():
