@@ -293,8 +293,13 @@ struct Operand {
 };
 
 struct TileCfg {
-  int p, row0, col0, n_need, n_mma, half, nk, nch, skip;
+  int p, n_need, n_mma, half, nk, nch, skip, flags;
+  int r0, r1, c0, c1;  // see TcTile
   Operand a, b;
+  __device__ __forceinline__ int arow(uint32_t rank) const { return rank ? r1 : r0; }
+  __device__ __forceinline__ int brow(uint32_t rank) const { return rank ? c1 : c0; }
+  // output column of accumulator column cc
+  __device__ __forceinline__ int col(int cc) const { return cc < half ? c0 + cc : c1 + (cc - half); }
 };
 
 __device__ __forceinline__ const void* tmap_of(const GemmArgs& g, int p, int which) {
@@ -324,18 +329,21 @@ __device__ __forceinline__ Operand make_operand(const GemmArgs& g, int p, int ma
 // (Y = 0) in this call.  Loaded ahead (see HeadPipe) so that the dependent
 // global loads do not stall the producer or the MMA issuer between tiles.
 struct TileHead {
-  TileDesc d;
+  TcTile d;
   int m, n, tall;
   float s;
 };
 
 __device__ __forceinline__ TileCfg make_cfg(const GemmArgs& g, const TileHead& h) {
   TileCfg c;
-  c.p = h.d.x;
-  c.row0 = h.d.y;
-  c.col0 = h.d.z;
-  c.n_need = h.d.w;
-  c.n_mma = (c.n_need + 31) & ~31;
+  c.p = h.d.p;
+  c.r0 = h.d.r0;
+  c.r1 = h.d.r1;
+  c.c0 = h.d.c0;
+  c.c1 = h.d.c1;
+  c.flags = h.d.flags;
+  c.n_need = h.d.n_need;
+  c.n_mma = tile_n_mma(c.n_need);
   c.half = c.n_mma >> 1;
   c.nch = (c.n_need + kEpiBoxCols - 1) / kEpiBoxCols;
   const int hi = kMapHi0 + g.cur;
@@ -363,14 +371,14 @@ __device__ __forceinline__ TileCfg make_cfg(const GemmArgs& g, const TileHead& h
   return c;
 }
 
-__device__ __forceinline__ TileHead load_head(const GemmArgs& g, const TileDesc& d) {
+__device__ __forceinline__ TileHead load_head(const GemmArgs& g, const TcTile& d) {
   TileHead h;
   h.d = d;
-  const MatInfo* mi = g.mats + d.x;
+  const MatInfo* mi = g.mats + d.p;
   h.m = mi->m;
   h.n = mi->n;
   h.tall = mi->tall;
-  h.s = g.ws.s[d.x];
+  h.s = g.ws.s[d.p];
   return h;
 }
 
@@ -381,7 +389,7 @@ __device__ __forceinline__ TileCfg decode_tile(const GemmArgs& g, int t) { retur
 // of tile t + npairs are in flight, so advancing is free of load latency.
 struct HeadPipe {
   TileHead cur, nxt;
-  TileDesc nn;
+  TcTile nn;
   int t, step, ntiles;
 
   __device__ __forceinline__ void start(const GemmArgs& g, int t0, int stride) {
@@ -576,8 +584,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (c.skip) continue;
       const uint32_t bytes =
           static_cast<uint32_t>(2 * (c.a.nbox * c.a.box_bytes + c.b.nbox * c.b.box_bytes));
-      const int arow = c.row0 + static_cast<int>(rank) * kHalfM;
-      const int brow = c.col0 + static_cast<int>(rank) * c.half;
+      const int arow = c.arow(rank);
+      const int brow = c.brow(rank);
       if (lane == 0) prefetch_tensormap(c.a.tmap);
       if (lane == 1) prefetch_tensormap(c.b.tmap);
       bool ok = true;
@@ -726,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const TileCfg c = decode_tile(g, t);
       const MatInfo& mi = g.mats[c.p];
       if (c.skip) continue;  // Y == 0: nothing downstream reads this matrix
-      const int i_lo = c.row0 + static_cast<int>(rank) * kHalfM + quad * 32;  // first row of this warp
+      const int i_lo = c.arow(rank) + quad * 32;  // first row of this warp
       const int i = i_lo + lane;
       const bool upd = (g.phase == kPhaseUpdate);
       const bool sym = !upd;
@@ -735,20 +743,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int ld_in = upd ? mi.ld : mi.lda;
       const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
       const bool poly = (g.phase == kPhasePoly);
-      // A chunk needs work unless it is a block strictly above the diagonal
-      // of a symmetric output that the mirror of a lower block writes.  A
-      // transposed tile (col0 > row0) lies wholly above the diagonal and
-      // writes every block with its mirror.
-      const int j_lim = (sym && c.col0 <= c.row0) ? i_lo + 31 : INT_MAX;
-      auto needed = [&](int ch) { return c.col0 + ch * kEpiBoxCols <= j_lim; };
+      // how chunk ch of this warp is written: always in the X update, by
+      // sym_block_mode in a symmetric product (0 = not at all)
+      auto mode = [&](int ch) { return sym ? sym_block_mode(c.flags, static_cast<int>(rank), i_lo, c.col(ch * kEpiBoxCols)) : 1; };
+      auto needed = [&](int ch) { return mode(ch) != 0; };
       auto block_inside = [&](int ch) {
-        return i_lo + 31 < rows_in && c.col0 + ch * kEpiBoxCols + 32 <= cols_in;
+        return i_lo + 31 < rows_in && c.col(ch * kEpiBoxCols) + 32 <= cols_in;
       };
-      // polynomial: coalesced prefetch of the next A block into registers
+      // polynomial: coalesced prefetch of an A block into registers; pf_ch
+      // is the chunk whose block pf0 holds (a tile may skip chunks and need
+      // later ones, so the next needed chunk is looked up, not assumed)
       uint4 pf0[4];
-      auto prefetch = [&](int ch) {
-        if (!poly || !needed(ch) || !block_inside(ch)) return;
-        load_block32(in0, ld_in, i_lo, c.col0 + ch * kEpiBoxCols, lane, pf0);
+      int pf_ch = -1;
+      auto prefetch_from = [&](int from) {
+        if (!poly) return;
+        for (int nx = from; nx < c.nch; nx += kEpiGroups)
+          if (needed(nx) && block_inside(nx)) {
+            load_block32(in0, ld_in, i_lo, c.col(nx * kEpiBoxCols), lane, pf0);
+            pf_ch = nx;
+            return;
+          }
       };
       // X update: ring of kUpdBufs lo buffers fed by cp.async; chunk k of
       // this warp lives in buffer k % kUpdBufs
@@ -761,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto stage_chunk = [&](int k) {
         const int chh = grp + k * kEpiGroups;
         if (block_inside(chh)) {
-          cp_block32(upd_buf(k % kUpdBufs), in0, ld_in, i_lo, c.col0 + chh * kEpiBoxCols, lane);
+          cp_block32(upd_buf(k % kUpdBufs), in0, ld_in, i_lo, c.col(chh * kEpiBoxCols), lane);
         }
         cp_async_commit();  // one group per chunk, empty for ragged chunks
       };
@@ -769,7 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (upd) {
         for (; issued < kc && issued < kUpdBufs; ++issued) stage_chunk(issued);
       } else {
-        prefetch(ch);
+        prefetch_from(ch);
       }
       // one lane waits and the warp follows its verdict, so the warp stays
       // converged for the .sync.aligned TMEM loads
@@ -784,8 +798,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
       const float s = g.ws.s[c.p];
       for (int k = 0; ch < c.nch; ch += kEpiGroups, ++k) {
-        const int j0 = c.col0 + ch * kEpiBoxCols;
-        if (!needed(ch)) continue;
+        const int j0 = c.col(ch * kEpiBoxCols);
+        const int md = mode(ch);
+        if (md == 0) continue;
         const bool inside = block_inside(ch);
         uint32_t v[32];
         __syncwarp();
@@ -807,6 +822,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         } else if (poly) {
           if (inside) {
+            if (pf_ch != ch) load_block32(in0, ld_in, i_lo, j0, lane, pf0);  // fallback; prefetch_from lands here
             staging_free();
             put_block32(blk0, lane, pf0);
             __syncwarp();
@@ -815,7 +831,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           } else {
             load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
           }
-          if (ch + kEpiGroups < c.nch) prefetch(ch + kEpiGroups);
+          prefetch_from(ch + kEpiGroups);
         }
         tmem_ld_wait();
         float val[32];
@@ -838,8 +854,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __align__(16) __nv_bfloat16 h[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
-          const bool above = j0 > i_lo + 31;  // only in a transposed tile
-          if (inside && (above || j0 + 31 < i_lo)) {
+          if (inside && md == 1) {
             // off-diagonal block: stage it and its transpose, store both
             staging_free();
             write_row32(blk0, lane, h);
@@ -848,15 +863,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
             publish(map, j0, i_lo, map, i_lo, j0);
           } else {
-            // diagonal or ragged block: element-wise with masks
+            // diagonal or ragged block: element-wise with masks (a ragged
+            // block below the diagonal is written whole, with its mirror)
+            const bool whole = (md == 1);
             __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
             __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
               const int j = j0 + q;
               if (i < mi.m && j < mi.m) {
-                if (above || j <= i) row[j] = h[q];
-                if (above || j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
+                if (whole || j <= i) row[j] = h[q];
+                if (whole || j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
               }
             }
           }

@@ -140,8 +140,8 @@ struct muon_plan_s {
   size_t dbytes = 0;
   Workspace ws{};
   MatInfo* mats_d = nullptr;
-  TileDesc* sym_d = nullptr;
-  TileDesc* full_d = nullptr;
+  TcTile* sym_d = nullptr;
+  TcTile* full_d = nullptr;
   TileDesc* sym32_d = nullptr;
   TileDesc* full32_d = nullptr;
   int n_sym = 0, n_full = 0, n_sym32 = 0, n_full32 = 0;
@@ -455,7 +455,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return work(x) > work(y); });
 
   // ---- the small device structures every plan holds, whatever its waves
-  std::vector<TileDesc> sym, full, sym32, full32;
+  std::vector<TcTile> sym, full;
+  std::vector<TileDesc> sym32, full32;
   std::vector<ChunkDesc> chunks;
   std::vector<int> wave_of(n, 0);
   auto fixed_bytes = [&](size_t ntile_sym, size_t ntile_full, size_t ntile_sym32, size_t ntile_full32,
@@ -470,8 +471,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
     add(n * sizeof(float));                          // Eq. 6 factors
     add(n * sizeof(MatInfo));
     add(muon_plan_s::kPtrSlots * n * sizeof(MatPtrs));
-    add(std::max<size_t>(1, ntile_sym) * sizeof(TileDesc));
-    add(std::max<size_t>(1, ntile_full) * sizeof(TileDesc));
+    add(std::max<size_t>(1, ntile_sym) * sizeof(TcTile));
+    add(std::max<size_t>(1, ntile_full) * sizeof(TcTile));
     add(std::max<size_t>(1, ntile_sym32) * sizeof(TileDesc));
     add(std::max<size_t>(1, ntile_full32) * sizeof(TileDesc));
     add(nchunk * sizeof(ChunkDesc));
@@ -482,8 +483,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   size_t cnt_sym = 0, cnt_full = 0, cnt_sym32 = 0, cnt_full32 = 0, cnt_chunk = 0;
   for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];
-    for_each_sym_tile(mi.m, [&](int, int, int) { ++cnt_sym; });
-    cnt_full += static_cast<size_t>((mi.rows + kTileM - 1) / kTileM) * ((mi.cols + kBN - 1) / kBN);
+    for_each_sym_tile(mi.m, [&](const TcTile&) { ++cnt_sym; });
+    for_each_full_tile(mi.rows, mi.cols, [&](const TcTile&) { ++cnt_full; });
     if (pl->fp32_ws) {
       cnt_sym32 += static_cast<size_t>((mi.m + kT32 - 1) / kT32) * ((mi.m + kT32 - 1) / kT32);
       cnt_full32 += static_cast<size_t>((mi.rows + kT32 - 1) / kT32) * ((mi.cols + kT32 - 1) / kT32);
@@ -580,9 +581,14 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
     for (int i : order) {
       if (wave_of[i] != w) continue;
       const MatInfo& mi = pl->mats[i];
-      for_each_sym_tile(mi.m, [&](int r0, int c0, int need) { sym.push_back(make_int4(i, r0, c0, need)); });
-      for (int r0 = 0; r0 < mi.rows; r0 += kTileM)
-        for (int c0 = 0; c0 < mi.cols; c0 += kBN) full.push_back(make_int4(i, r0, c0, std::min(kBN, mi.cols - c0)));
+      for_each_sym_tile(mi.m, [&](TcTile t) {
+        t.p = i;
+        sym.push_back(t);
+      });
+      for_each_full_tile(mi.rows, mi.cols, [&](TcTile t) {
+        t.p = i;
+        full.push_back(t);
+      });
       if (pl->fp32_ws) {
         for (int r0 = 0; r0 < mi.m; r0 += kT32)
           for (int c0 = 0; c0 < mi.m; c0 += kT32) sym32.push_back(make_int4(i, r0, c0, 0));
@@ -627,8 +633,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   const size_t o_unorm = take(n * sizeof(float));
   const size_t o_mats = take(n * sizeof(MatInfo));
   const size_t o_ptrs = take(muon_plan_s::kPtrSlots * n * sizeof(MatPtrs));
-  const size_t o_sym = take(std::max<size_t>(1, sym.size()) * sizeof(TileDesc));
-  const size_t o_full = take(std::max<size_t>(1, full.size()) * sizeof(TileDesc));
+  const size_t o_sym = take(std::max<size_t>(1, sym.size()) * sizeof(TcTile));
+  const size_t o_full = take(std::max<size_t>(1, full.size()) * sizeof(TcTile));
   const size_t o_sym32 = take(std::max<size_t>(1, sym32.size()) * sizeof(TileDesc));
   const size_t o_full32 = take(std::max<size_t>(1, full32.size()) * sizeof(TileDesc));
   const size_t o_chunks = take(chunks.size() * sizeof(ChunkDesc));
@@ -665,8 +671,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   pl->mats_d = reinterpret_cast<MatInfo*>(b + o_mats);
   for (int k = 0; k < muon_plan_s::kPtrSlots; ++k) pl->slots[k].dev = reinterpret_cast<MatPtrs*>(b + o_ptrs) + k * n;
   pl->ptrs_d = pl->slots[0].dev;
-  pl->sym_d = reinterpret_cast<TileDesc*>(b + o_sym);
-  pl->full_d = reinterpret_cast<TileDesc*>(b + o_full);
+  pl->sym_d = reinterpret_cast<TcTile*>(b + o_sym);
+  pl->full_d = reinterpret_cast<TcTile*>(b + o_full);
   pl->sym32_d = reinterpret_cast<TileDesc*>(b + o_sym32);
   pl->full32_d = reinterpret_cast<TileDesc*>(b + o_full32);
   pl->chunks_d = reinterpret_cast<ChunkDesc*>(b + o_chunks);
@@ -685,9 +691,9 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   bool ok = cudaMemcpy(pl->mats_d, pl->mats.data(), n * sizeof(MatInfo), cudaMemcpyHostToDevice) == cudaSuccess;
-  ok = ok && (sym.empty() || cudaMemcpy(pl->sym_d, sym.data(), sym.size() * sizeof(TileDesc),
+  ok = ok && (sym.empty() || cudaMemcpy(pl->sym_d, sym.data(), sym.size() * sizeof(TcTile),
                                         cudaMemcpyHostToDevice) == cudaSuccess);
-  ok = ok && (full.empty() || cudaMemcpy(pl->full_d, full.data(), full.size() * sizeof(TileDesc),
+  ok = ok && (full.empty() || cudaMemcpy(pl->full_d, full.data(), full.size() * sizeof(TcTile),
                                          cudaMemcpyHostToDevice) == cudaSuccess);
   ok = ok && (sym32.empty() || cudaMemcpy(pl->sym32_d, sym32.data(), sym32.size() * sizeof(TileDesc),
                                           cudaMemcpyHostToDevice) == cudaSuccess);

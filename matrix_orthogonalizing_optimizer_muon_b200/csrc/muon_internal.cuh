@@ -106,27 +106,93 @@ inline bool any_overlap(std::vector<ByteRange>& v) {
   return false;
 }
 
-// Tile of a GEMM phase: .x matrix, .y row0, .z col0, .w n_need (columns that
-// hold useful output, <= kBN).  Symmetric phases list each tile of the lower
-// triangle once; see for_each_sym_tile.
+// Tile of the fp32 path's GEMM phases: .x matrix, .y row0, .z col0, .w unused.
 using TileDesc = int4;
 
-// Tiles of a symmetric m x m product (X X^T, A A) on the kTileM x kBN grid,
-// lower triangle only.  A ragged last row block (fewer than kTileM rows)
-// would leave part of every M = 256 tile in its row empty, so its
-// off-diagonal tiles are listed transposed: rows of the full block c0 and
-// columns of the ragged block.  col0 > row0 marks such a tile; every 32 x 32
-// block of it lies above the diagonal and is stored with its mirror.
+// Tile of the tensor-core path: a pair of CTAs computes rows [r0, r0 + 128)
+// (CTA 0) and [r1, r1 + 128) (CTA 1) of the product against N <= 256 output
+// columns; CTA k stages the B operand rows [ck, ck + N/2), and accumulator
+// column c holds output column c0 + c (c < N/2) or c1 + c - N/2.  Rows and
+// columns need not be contiguous: a symmetric product is tiled in 128-row
+// blocks (see for_each_sym_tile).
+struct TcTile {
+  int32_t p;       // matrix
+  int32_t n_need;  // accumulator columns that hold output (1..256)
+  int32_t flags;   // kTileGhost1, kTileDiagOnly
+  int32_t pad_;
+  int32_t r0, r1;  // first output row of CTA 0 / CTA 1
+  int32_t c0, c1;  // first B-operand row (output column) staged by CTA 0 / CTA 1
+};
+constexpr int32_t kTileGhost1 = 1;    // CTA 1 duplicates CTA 0's rows and writes nothing
+constexpr int32_t kTileDiagOnly = 2;  // only the diagonal 128-blocks of the tile are outputs
+
+// How a 32 x 32 block of a symmetric product, rows [i0, i0 + 32) and columns
+// [j0, j0 + 32) (both multiples of 32), computed by CTA `rank` of a tile with
+// `flags`, is written:
+//   0 not at all (a duplicate, or the upper part of a diagonal 128-block);
+//   1 with its mirror (a block strictly below the diagonal);
+//   2 element-wise, (i, j) for j <= i and (j, i) for j < i (on the diagonal).
+// No tile writes a block above the diagonal of its own: the tiling covers
+// each pair of 128-blocks through the lower one.
+__host__ __device__ __forceinline__ int sym_block_mode(int flags, int rank, int i0, int j0) {
+  if (rank == 1 && (flags & kTileGhost1)) return 0;
+  const int ib = i0 >> 7, jb = j0 >> 7;
+  if (ib != jb) return (ib > jb && !(flags & kTileDiagOnly)) ? 1 : 0;
+  if (j0 > i0) return 0;
+  return j0 == i0 ? 2 : 1;
+}
+
+// Columns of a tile's accumulator: a multiple of 32 covering n_need.
+__host__ __device__ __forceinline__ int tile_n_mma(int n_need) { return (n_need + 31) & ~31; }
+
+// Tiles of a symmetric m x m product (X X^T, A A) over 128-row blocks
+// 0 .. nb - 1, nb = ceil(m / 128); every element (i, j), j <= i, is written by
+// exactly one tile (sym_block_mode).  With P = floor(nb / 2) pairs of blocks:
+//   - rows {2i, 2i+1} x columns {2j, 2j+1}, j < i: four blocks below the diagonal;
+//   - nb even: rows {2i, 2i+1} x columns {2i, 2i+1}: two diagonal blocks and
+//     (2i+1, 2i); the block above the diagonal is skipped;
+//   - nb odd, last block L = nb - 1: rows {2i+1, L} x columns {2i, 2i+1}: the
+//     diagonal block 2i+1, (2i+1, 2i) and the two blocks of row L; then the
+//     remaining diagonal blocks 0, 2, .., 2P-2, L two per tile (rows {a, b} x
+//     columns {a, b}, diagonal blocks only), the last one alone if their count
+//     is odd.
+// For m = 1408 (11 blocks) that is 10 + 5 + 3 = 18 tiles of 256 columns,
+// against 21 for square 256-blocks with the ragged block transposed.
 template <class F>
 inline void for_each_sym_tile(int m, F&& emit) {
-  static_assert(kTileM == kBN, "square tile grid");
-  for (int r0 = 0; r0 < m; r0 += kTileM) {
-    const int rv = m - r0 < kTileM ? m - r0 : kTileM;
-    for (int c0 = 0; c0 <= r0; c0 += kBN) {
-      if (c0 < r0 && rv < kTileM) emit(c0, r0, rv);
-      else emit(r0, c0, m - c0 < kBN ? m - c0 : kBN);
-    }
+  const int nb = (m + 127) / 128, P = nb / 2;
+  const bool odd = (nb & 1) != 0;
+  const int L = nb - 1;
+  auto contiguous = [&](int r0, int r1, int c0, int flags) {
+    const int need = m - c0 < 256 ? m - c0 : 256;
+    const int half = tile_n_mma(need) / 2;
+    emit(TcTile{0, need, flags, 0, r0, r1, c0, c0 + half});
+  };
+  for (int i = 0; i < P; ++i) {
+    for (int j = 0; j < i; ++j) contiguous(256 * i, 256 * i + 128, 256 * j, 0);
+    if (odd) emit(TcTile{0, 256, 0, 0, 256 * i + 128, 128 * L, 256 * i, 256 * i + 128});
+    else contiguous(256 * i, 256 * i + 128, 256 * i, 0);
   }
+  if (odd) {
+    std::vector<int> d;
+    for (int i = 0; i < P; ++i) d.push_back(2 * i);
+    d.push_back(L);
+    size_t k = 0;
+    for (; k + 1 < d.size(); k += 2)
+      emit(TcTile{0, 256, kTileDiagOnly, 0, 128 * d[k], 128 * d[k + 1], 128 * d[k], 128 * d[k + 1]});
+    if (k < d.size()) contiguous(128 * d[k], 128 * d[k], 128 * d[k], kTileGhost1 | kTileDiagOnly);
+  }
+}
+
+// Tiles of a full [R, C] product (the X update): rows [r0, r0 + 256) on the
+// pair, columns [c0, c0 + 256) contiguous.
+template <class F>
+inline void for_each_full_tile(int R, int C, F&& emit) {
+  for (int r0 = 0; r0 < R; r0 += 256)
+    for (int c0 = 0; c0 < C; c0 += 256) {
+      const int need = C - c0 < 256 ? C - c0 : 256;
+      emit(TcTile{0, need, 0, 0, r0, r0 + 128, c0, c0 + tile_n_mma(need) / 2});
+    }
 }
 
 // Momentum/normalise chunk: .x matrix, .y first row, .z number of rows, .w slot
@@ -165,7 +231,7 @@ __host__ __device__ __forceinline__ float update_scale_of(const StepScalars& sc,
 // Arguments of the tensor-core GEMM kernel (one launch = one phase of one
 // Newton-Schulz iteration over every matrix of the plan).
 struct GemmArgs {
-  const TileDesc* tiles;
+  const TcTile* tiles;
   int ntiles;
   int phase;            // Phase
   int iter;             // 0-based iteration index (iteration 0 folds in 1/||Y||_F)

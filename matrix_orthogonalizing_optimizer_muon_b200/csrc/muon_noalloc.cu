@@ -53,8 +53,8 @@ constexpr size_t kOffStatus = kOffRms + align256(kNaMaxRms * sizeof(float));
 constexpr size_t kOffMat = kOffStatus + 256;
 constexpr size_t kOffPtrs = kOffMat + align256(sizeof(MatInfo));
 constexpr size_t kOffSym = kOffPtrs + align256(sizeof(MatPtrs));
-constexpr size_t kOffFull = kOffSym + align256(kNaMaxTiles * sizeof(TileDesc));
-constexpr size_t kOffChunks = kOffFull + align256(kNaMaxTiles * sizeof(TileDesc));
+constexpr size_t kOffFull = kOffSym + align256(kNaMaxTiles * sizeof(TcTile));
+constexpr size_t kOffChunks = kOffFull + align256(kNaMaxTiles * sizeof(TcTile));
 constexpr size_t kOffTmaps = kOffChunks + align256(kNaMaxChunks * sizeof(ChunkDesc));
 constexpr size_t kScratchBytes = kOffTmaps + align256(kMapsPerMat * sizeof(CUtensorMap));
 
@@ -155,19 +155,18 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   }
   mi.chunk_base = 0;
   mi.nchunks = nch;
-  TileDesc sym[kNaMaxTiles], full[kNaMaxTiles];
+  TcTile sym[kNaMaxTiles], full[kNaMaxTiles];
   int nsym = 0, nfull = 0;
-  bool sym_fits = true;
-  for_each_sym_tile(mi.m, [&](int r0, int c0, int need) {
-    if (nsym == kNaMaxTiles) sym_fits = false;
-    else sym[nsym++] = make_int4(0, r0, c0, need);
+  bool fits = true;
+  for_each_sym_tile(mi.m, [&](const TcTile& t) {
+    if (nsym == kNaMaxTiles) fits = false;
+    else sym[nsym++] = t;
   });
-  if (!sym_fits) return MUON_ERR_UNSUPPORTED;
-  for (int r0 = 0; r0 < R; r0 += kTileM)
-    for (int c0 = 0; c0 < C; c0 += kBN) {
-      if (nfull == kNaMaxTiles) return MUON_ERR_UNSUPPORTED;
-      full[nfull++] = make_int4(0, r0, c0, std::min(kBN, C - c0));
-    }
+  for_each_full_tile(R, C, [&](const TcTile& t) {
+    if (nfull == kNaMaxTiles) fits = false;
+    else full[nfull++] = t;
+  });
+  if (!fits) return MUON_ERR_UNSUPPORTED;
   MatPtrs mp{};
   mp.W = O_out;
   mp.G = X_in;
@@ -194,15 +193,15 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   // driver before the call returns) and clear what must start at zero
   MatInfo* mats_d = reinterpret_cast<MatInfo*>(base + kOffMat);
   MatPtrs* ptrs_d = reinterpret_cast<MatPtrs*>(base + kOffPtrs);
-  TileDesc* sym_d = reinterpret_cast<TileDesc*>(base + kOffSym);
-  TileDesc* full_d = reinterpret_cast<TileDesc*>(base + kOffFull);
+  TcTile* sym_d = reinterpret_cast<TcTile*>(base + kOffSym);
+  TcTile* full_d = reinterpret_cast<TcTile*>(base + kOffFull);
   ChunkDesc* chunks_d = reinterpret_cast<ChunkDesc*>(base + kOffChunks);
   void* tmaps_d = base + kOffTmaps;
   cudaError_t e = cudaSuccess;
   e = e == cudaSuccess ? cudaMemcpyAsync(mats_d, &mi, sizeof(mi), cudaMemcpyHostToDevice, st) : e;
   e = e == cudaSuccess ? cudaMemcpyAsync(ptrs_d, &mp, sizeof(mp), cudaMemcpyHostToDevice, st) : e;
-  e = e == cudaSuccess ? cudaMemcpyAsync(sym_d, sym, nsym * sizeof(TileDesc), cudaMemcpyHostToDevice, st) : e;
-  e = e == cudaSuccess ? cudaMemcpyAsync(full_d, full, nfull * sizeof(TileDesc), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(sym_d, sym, nsym * sizeof(TcTile), cudaMemcpyHostToDevice, st) : e;
+  e = e == cudaSuccess ? cudaMemcpyAsync(full_d, full, nfull * sizeof(TcTile), cudaMemcpyHostToDevice, st) : e;
   e = e == cudaSuccess ? cudaMemcpyAsync(chunks_d, chunks, nch * sizeof(ChunkDesc), cudaMemcpyHostToDevice, st) : e;
   e = e == cudaSuccess ? cudaMemcpyAsync(tmaps_d, tm, sizeof(tm), cudaMemcpyHostToDevice, st) : e;
   e = e == cudaSuccess ? cudaMemsetAsync(ws.norm_count, 0, sizeof(unsigned), st) : e;

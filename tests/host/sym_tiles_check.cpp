@@ -1,47 +1,63 @@
-// Host check of the symmetric-product tile list (for_each_sym_tile).
+// Host check of the symmetric-product tiling of the tensor-core path
+// (for_each_sym_tile and sym_block_mode, the functions the kernel uses).
 //
-// For every m in [1, 2100] the list must:
-//  - put every tile on the 256 x 256 grid with 1 <= need <= 256 columns
-//    inside the matrix;
-//  - have full rows (row0 + 256 <= m) in every tile whose rows are not the
-//    diagonal block of the last, ragged row block;
-//  - cover each element (i, j), j <= i, of the lower triangle exactly once,
-//    counting a transposed tile (col0 > row0) by its mirror.
-// Prints "ok <tiles for m = 1408>" or the first violation.
+// For every m in [1, 2100]:
+//  - every tile has 1 <= n_need <= 256 columns, rows and staged B rows that
+//    start on a multiple of 16 elements (TMA alignment), and a contiguous
+//    tile's second half starts where its first ends;
+//  - walking each CTA's 32-row groups and each 32-column chunk of the
+//    accumulator exactly as the epilogue does, the blocks that
+//    sym_block_mode writes cover each element (i, j), j <= i, of the lower
+//    triangle exactly once (a block written with its mirror covers (i, j)
+//    for all its elements, a diagonal block the elements with j <= i).
+// Prints "ok <tiles for m = 1408> <tiles for m = 2048>" or the first violation.
 #include "muon_internal.cuh"
 
 #include <cstdio>
 #include <vector>
 
 int main() {
-  using muon::kTileM;
-  int tiles_1408 = 0;
+  using namespace muon;
+  int tiles_1408 = 0, tiles_2048 = 0;
   for (int m = 1; m <= 2100; ++m) {
     std::vector<unsigned char> cover(static_cast<size_t>(m) * m, 0);
     bool bad = false;
     int count = 0;
-    muon::for_each_sym_tile(m, [&](int row0, int col0, int need) {
+    for_each_sym_tile(m, [&](const TcTile& t) {
       ++count;
-      if (row0 % kTileM || col0 % kTileM || need < 1 || need > kTileM || row0 >= m || col0 + need > m) {
-        std::printf("m=%d: tile (%d, %d, %d) off the grid\n", m, row0, col0, need);
+      const int n_mma = tile_n_mma(t.n_need), half = n_mma / 2;
+      if (t.n_need < 1 || t.n_need > 256 || t.r0 % 16 || t.r1 % 16 || t.c0 % 16 || t.c1 % 16 || t.r0 >= m ||
+          t.c0 >= m) {
+        std::printf("m=%d: tile (%d %d | %d %d, %d) malformed\n", m, t.r0, t.r1, t.c0, t.c1, t.n_need);
         bad = true;
         return;
       }
-      const bool transposed = col0 > row0;
-      if (row0 + kTileM > m && !(col0 == row0 && !transposed)) {
-        std::printf("m=%d: tile (%d, %d) has ragged rows off the diagonal\n", m, row0, col0);
-        bad = true;
-      }
-      for (int i = row0; i < row0 + kTileM && i < m; ++i)
-        for (int j = col0; j < col0 + need; ++j) {
-          const int r = transposed ? j : i, c = transposed ? i : j;
-          if (c > r) continue;  // the upper half of a diagonal tile is not an output
-          if (++cover[static_cast<size_t>(r) * m + c] > 1) {
-            std::printf("m=%d: element (%d, %d) covered twice\n", m, r, c);
-            bad = true;
-            return;
+      for (int rank = 0; rank < 2 && !bad; ++rank) {
+        const int rbase = rank ? t.r1 : t.r0;
+        for (int q4 = 0; q4 < 4 && !bad; ++q4) {
+          const int i_lo = rbase + 32 * q4;
+          for (int cc = 0; cc < t.n_need && !bad; cc += 32) {
+            const int j0 = cc < half ? t.c0 + cc : t.c1 + (cc - half);
+            const int md = sym_block_mode(t.flags, rank, i_lo, j0);
+            if (md == 0) continue;
+            for (int i = i_lo; i < i_lo + 32 && i < m; ++i)
+              for (int j = j0; j < j0 + 32 && j < m; ++j) {
+                if (md == 2 && j > i) continue;
+                const int r = i >= j ? i : j, c = i >= j ? j : i;
+                if (md == 1 && j > i) {
+                  std::printf("m=%d: block (%d, %d) above the diagonal written whole\n", m, i_lo, j0);
+                  bad = true;
+                  return;
+                }
+                if (++cover[static_cast<size_t>(r) * m + c] > 1) {
+                  std::printf("m=%d: element (%d, %d) written twice\n", m, r, c);
+                  bad = true;
+                  return;
+                }
+              }
           }
         }
+      }
     });
     for (int r = 0; r < m && !bad; ++r)
       for (int c = 0; c <= r; ++c)
@@ -52,7 +68,8 @@ int main() {
         }
     if (bad) return 1;
     if (m == 1408) tiles_1408 = count;
+    if (m == 2048) tiles_2048 = count;
   }
-  std::printf("ok %d\n", tiles_1408);
+  std::printf("ok %d %d\n", tiles_1408, tiles_2048);
   return 0;
 }
