@@ -234,6 +234,15 @@ __device__ __forceinline__ void tc_commit(uint32_t bar_cluster) {
                : "memory");
 }
 
+// The same arrive on the barrier at this shared-memory offset in both CTAs of
+// the pair (one instruction).
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
@@ -577,6 +586,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // lanes the B boxes, all in one instruction; lane 0 owns the barriers.
     const int pp = (warp == kWarpProducer) ? 0 : warp - kWarpProducer2 + 1;
     long fills = 0;  // fills of all producers, in order
+    int fstage = 0;        // stage of fill `fills`
+    uint32_t fphase = 0;   // its ring pass parity
+    const uint32_t full0 = map_to_rank(full_bar(0), 0);  // the leader's full barriers
     HeadPipe hp;
     for (hp.start(g, pair, npairs); hp.valid(); hp.advance(g)) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
@@ -590,9 +602,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 1) prefetch_tensormap(c.b.tmap);
       bool ok = true;
       for (int kb = 0; kb < c.nk; ++kb, ++fills) {
-        if (fills % kProducers != pp) continue;
-        const int stage = static_cast<int>(fills % nst);
-        const uint32_t phase = static_cast<uint32_t>((fills / nst) & 1);
+        const int stage = fstage;
+        const uint32_t phase = fphase;
+        if (++fstage == nst) {
+          fstage = 0;
+          fphase ^= 1u;
+        }
+        if (static_cast<int>(fills % kProducers) != pp) continue;
         int ready = 0;
         if (lane == 0) {
           ready = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag) ? 1 : 0;
@@ -604,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t fb = map_to_rank(full_bar(stage), 0);
+        const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
         const uint32_t sa = sbase + SmemLayout::kStages + stage * kStageBytes;
         const uint32_t sb = sa + kOpBytes;
         const int k0 = kb * kBK;
@@ -681,16 +697,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         (kb | kk) != 0 ? 1u : 0u);
           issued = true;
           // free the stage in both CTAs once these MMAs have read it
-          tc_commit(empty_bar(stage));
-          tc_commit(map_to_rank(empty_bar(stage), 1));
+          tc_commit_pair(empty_bar(stage));
           if (++stage == nst) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(tfull_bar(acc));  // accumulator complete, both halves
-        tc_commit(map_to_rank(tfull_bar(acc), 1));
+        tc_commit_pair(tfull_bar(acc));  // accumulator complete, both halves
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
