@@ -367,7 +367,61 @@ __global__ void __launch_bounds__(kEwThreads) rms_finalize_kernel(const MatInfo*
   if (threadIdx.x == 0) out[blockIdx.x] = (float)sqrt(sum / ((double)mi.rows * (double)mi.cols));
 }
 
+// Split-K reduction of a symmetric product: one CTA of 32 x 8 threads per
+// 32 x 32 block on or below the diagonal.  Each element's parts are summed in
+// part order (so the result does not depend on which CTA pair computed which
+// part), the phase's epilogue arithmetic is applied, the bf16 value is
+// written and, through a shared-memory transpose, its mirror.
+__global__ void __launch_bounds__(256) split_reduce_kernel(const int4* __restrict__ blocks,
+                                                           const MatInfo* __restrict__ mats, Workspace ws,
+                                                           StepScalars sc, int phase, int iter, int split) {
+  __shared__ __nv_bfloat16 tile[32][34];
+  const int4 bk = blocks[blockIdx.x];
+  const MatInfo mi = mats[bk.x];
+  const int i0 = bk.y, j0 = bk.z, m = mi.m;
+  const float s = ws.s[bk.x];
+  if (s == 0.0f) return;  // Y == 0: the matrix is skipped, as in the tensor-core launches
+  __nv_bfloat16* out = (phase == kPhaseGram ? ws.A : ws.B) + mi.off_a;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int j = j0 + tx;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = ty + 8 * k;
+    const int i = i0 + r;
+    __nv_bfloat16 h = __float2bfloat16_rn(0.0f);
+    if (i < m && j < m && j <= i) {
+      const size_t e = static_cast<size_t>(i) * mi.lda + j;
+      float acc = 0.0f;
+      for (int p = 0; p < split; ++p) acc += ws.part[p * ws.part_stride + mi.off_a + e];
+      float v;
+      if (phase == kPhaseGram) {
+        v = (iter == 0) ? (acc * s) * s : acc;
+      } else {
+        v = fmaf(sc.c, acc, sc.b * __bfloat162float(ws.A[mi.off_a + e])) + (i == j ? sc.a : 0.0f);
+      }
+      h = __float2bfloat16_rn(v);
+      out[e] = h;
+    }
+    tile[r][tx] = h;
+  }
+  __syncthreads();
+  // mirror: element (j0 + r, i0 + tx) = tile[tx][r], for (i0 + tx) > (j0 + r)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = ty + 8 * k;
+    const int jr = j0 + r, ic = i0 + tx;
+    if (jr < m && ic < m && ic > jr) out[static_cast<size_t>(jr) * mi.lda + ic] = tile[tx][r];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_split_reduce(const int4* blocks, int nblocks, const MatInfo* mats, Workspace ws, StepScalars sc,
+                                int phase, int iter, int split, cudaStream_t st) {
+  if (nblocks == 0) return cudaSuccess;
+  split_reduce_kernel<<<nblocks, dim3(32, 8), 0, st>>>(blocks, mats, ws, sc, phase, iter, split);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
                       Workspace ws, StepScalars sc, int mode, int fp32_path, cudaStream_t st) {

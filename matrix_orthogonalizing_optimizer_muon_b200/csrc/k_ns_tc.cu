@@ -317,6 +317,7 @@ struct Operand {
 
 struct TileCfg {
   int p, n_need, n_mma, half, nk, nch, skip, flags;
+  int kb0, kpart;      // first K stage of this tile's part, and the part (split K)
   int r0, r1, c0, c1;  // see TcTile
   Operand a, b;
   __device__ __forceinline__ int arow(uint32_t rank) const { return rank ? r1 : r0; }
@@ -389,7 +390,16 @@ __device__ __forceinline__ TileCfg make_cfg(const GemmArgs& g, const TileHead& h
       c.b = make_operand(g, c.p, hi, 1, c.half);
     }
   }
-  c.nk = (K + kBK - 1) / kBK;
+  const int nk_all = (K + kBK - 1) / kBK;
+  c.kpart = h.d.kpart;
+  if (g.split > 1 && g.phase != kPhaseUpdate) {
+    // part k of `split` takes stages [k nk / split, (k + 1) nk / split)
+    c.kb0 = (c.kpart * nk_all) / g.split;
+    c.nk = ((c.kpart + 1) * nk_all) / g.split - c.kb0;
+  } else {
+    c.kb0 = 0;
+    c.nk = nk_all;
+  }
   c.skip = (h.s == 0.0f) ? 1 : 0;
   return c;
 }
@@ -637,7 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
         const uint32_t sa = sbase + SmemLayout::kStages + stage * kStageBytes;
         const uint32_t sb = sa + kOpBytes;
-        const int k0 = kb * kBK;
+        const int k0 = (c.kb0 + kb) * kBK;
         const bool is_a = lane < c.a.nbox;
         const Operand& o = is_a ? c.a : c.b;
         const int h = is_a ? lane : lane - c.a.nbox;
@@ -770,7 +780,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const __nv_bfloat16* in0 = upd ? g.ws.lo + mi.off_x : g.ws.A + mi.off_a;
       const int ld_in = upd ? mi.ld : mi.lda;
       const int rows_in = upd ? mi.rows : mi.m, cols_in = upd ? mi.cols : mi.m;
-      const bool poly = (g.phase == kPhasePoly);
+      // split K: this tile computes one part of the K range; its raw fp32
+      // accumulator goes to ws.part and a reduction pass forms the product
+      const bool splitk = sym && g.split > 1;
+      const bool poly = (g.phase == kPhasePoly) && !splitk;
       // how chunk ch of this warp is written: always in the X update, by
       // sym_block_mode in a symmetric product (0 = not at all)
       auto mode = [&](int ch) { return sym ? sym_block_mode(c.flags, static_cast<int>(rank), i_lo, c.col(ch * kEpiBoxCols)) : 1; };
@@ -862,6 +875,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           prefetch_from(ch + kEpiGroups);
         }
         tmem_ld_wait();
+        if (splitk) {
+          if (inside) {
+            // this thread's row (128 bytes) into the 4 KiB staging pair,
+            // 16-byte chunk q at q ^ (row & 7): the 128-byte swizzle of the
+            // part map's 32 x 32 fp32 box
+            staging_free();
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(blk0 + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(tmap_of(g, c.p, kMapStPart), blk0_s, j0, i_lo, c.kpart);
+              bulk_commit();
+            }
+          } else if (i < mi.m) {
+            float* prow = g.ws.part + c.kpart * g.ws.part_stride + mi.off_a + static_cast<size_t>(i) * mi.lda;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (j0 + q < mi.m) prow[j0 + q] = u2f(v[q]);
+          }
+          continue;
+        }
         float val[32];
         if (g.phase == kPhaseGram) {
           const bool first = (g.iter == 0);

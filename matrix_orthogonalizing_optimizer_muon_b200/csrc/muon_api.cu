@@ -82,16 +82,36 @@ bool encode_bf16_pair(CUtensorMap* tm, void* base, int rows, int cols, int ld, l
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 tensor map over `nparts` [rows, cols] arrays with row pitch `ld`,
+// `part_bytes` apart: boxes {32, 32, 1}, 128-byte swizzle (the split-K parts).
+bool encode_f32_parts(CUtensorMap* tm, void* base, int rows, int cols, int ld, long long part_bytes, int nparts) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr || part_bytes <= 0 || part_bytes % 16 != 0 || nparts < 1) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(nparts)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 4, static_cast<cuuint64_t>(part_bytes)};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 // Operand maps (64 x 128 and 64 x 64 boxes) and epilogue store maps (32 x 32,
 // hi and lo together) of one matrix's workspace arrays, in MapIndex order.
-// lo must lie after hi0 and hi1 in memory.
+// lo must lie after hi0 and hi1 in memory.  Without split-K parts the part
+// map repeats the A store map (it is never used then).
 bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0, __nv_bfloat16* hi1,
-                              __nv_bfloat16* lo, __nv_bfloat16* A, __nv_bfloat16* B) {
+                              __nv_bfloat16* lo, __nv_bfloat16* A, __nv_bfloat16* B, float* part,
+                              int64_t part_stride, int nparts) {
   CUtensorMap* t = static_cast<CUtensorMap*>(maps);
   const int R = mi.rows, C = mi.cols, m = mi.m;
-  return encode_bf16_2d(t + kMapHi0, hi0, R, C, mi.ld, kBoxInner, 128) &&
+  const bool parts_ok = part != nullptr
+                            ? encode_f32_parts(t + kMapStPart, part, m, m, mi.lda, part_stride * 4, nparts)
+                            : encode_bf16_2d(t + kMapStPart, A, m, m, mi.lda, kEpiBoxCols, 32);
+  return parts_ok && encode_bf16_2d(t + kMapHi0, hi0, R, C, mi.ld, kBoxInner, 128) &&
          encode_bf16_2d(t + kMapHi1, hi1, R, C, mi.ld, kBoxInner, 128) &&
          encode_bf16_2d(t + kMapA, A, m, m, mi.lda, kBoxInner, 128) &&
          encode_bf16_2d(t + kMapB, B, m, m, mi.lda, kBoxInner, 128) &&
@@ -118,6 +138,8 @@ struct ProfRec {
 // A plan without a workspace cap has one wave holding every matrix.
 struct Wave {
   int sym_off = 0, n_sym = 0;      // bf16 path, symmetric products
+  int symg_off = 0, n_symg = 0;    // the Gram product's tiles with their split-K parts
+  int red_off = 0, n_red = 0;      // split-K reduction blocks
   int full_off = 0, n_full = 0;    // bf16 path, X update
   int sym32_off = 0, n_sym32 = 0;  // fp32 path
   int full32_off = 0, n_full32 = 0;
@@ -148,6 +170,9 @@ struct muon_plan_s {
   ChunkDesc* chunks_d = nullptr;
   int nchunks = 0;
   std::vector<Wave> waves;     // run one after another; their workspace is shared
+  int split = 1;               // split-K parts of the Gram product (1: none)
+  TcTile* symg_d = nullptr;    // the Gram tiles with their parts (split > 1)
+  int4* reduce_d = nullptr;    // split-K reduction blocks, wave by wave
   uint64_t inject_wait_ns = 0; // failure-detection test: consumed by the next call's first GEMM launch
   void* tmaps_d = nullptr;
   // Per-call pointer tables, kept resident on the device: a call whose
@@ -296,8 +321,10 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
           e = launch_gemm_f32(a, st);
         } else {
           GemmArgs a{};
-          a.tiles = (ph == kPhaseUpdate) ? pl->full_d + w.full_off : pl->sym_d + w.sym_off;
-          a.ntiles = (ph == kPhaseUpdate) ? w.n_full : w.n_sym;
+          const bool gsplit = (ph == kPhaseGram && pl->split > 1);
+          a.tiles = (ph == kPhaseUpdate) ? pl->full_d + w.full_off
+                                         : (gsplit ? pl->symg_d + w.symg_off : pl->sym_d + w.sym_off);
+          a.ntiles = (ph == kPhaseUpdate) ? w.n_full : (gsplit ? w.n_symg : w.n_sym);
           a.phase = ph;
           a.iter = it;
           a.cur = cur;
@@ -307,8 +334,11 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
           a.ws = pl->ws;
           a.sc = sc;
           a.test_wait_ns = pl->inject_wait_ns;
+          a.split = gsplit ? pl->split : 1;
           pl->inject_wait_ns = 0;
           e = launch_gemm_tc(a, pl->npairs, st);
+          if (e == cudaSuccess && a.split > 1)
+            e = launch_split_reduce(pl->reduce_d + w.red_off, w.n_red, pl->mats_d, pl->ws, sc, ph, it, a.split, st);
         }
         if (e != cudaSuccess) return MUON_ERR_CUDA;
         rec.mark(1 + ph);
@@ -443,7 +473,7 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   }
   // bytes per element of the iterate arrays (hi0, hi1, lo; + x32[2]) and of the
   // symmetric arrays (A, B; + a32, b32)
-  const size_t bx = pl->fp32_ws ? 6 + 8 : 6, ba = pl->fp32_ws ? 4 + 8 : 4;
+  size_t bx = pl->fp32_ws ? 6 + 8 : 6, ba = pl->fp32_ws ? 4 + 8 : 4;
   // LPT order of matrices (largest Newton-Schulz work first): the order of the
   // GEMM schedules and of the wave packing
   std::vector<int> order(n);
@@ -455,8 +485,9 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return work(x) > work(y); });
 
   // ---- the small device structures every plan holds, whatever its waves
-  std::vector<TcTile> sym, full;
+  std::vector<TcTile> sym, symg, full;
   std::vector<TileDesc> sym32, full32;
+  std::vector<int4> red;
   std::vector<ChunkDesc> chunks;
   std::vector<int> wave_of(n, 0);
   auto fixed_bytes = [&](size_t ntile_sym, size_t ntile_full, size_t ntile_sym32, size_t ntile_full32,
@@ -492,8 +523,40 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
     const int rows_per_chunk = std::max(1, kChunkElems / mi.cols);
     cnt_chunk += (mi.rows + rows_per_chunk - 1) / rows_per_chunk;
   }
-  const size_t fixed = fixed_bytes(cnt_sym, cnt_full, cnt_sym32, cnt_full32, cnt_chunk);
+  // ---- split K of the Gram product: a plan whose symmetric launches hold
+  // too few tiles to fill the CTA pairs, and whose Gram products have a long
+  // K (= n), splits each Gram tile's K range into 2 or 4 parts (fp32 partial
+  // products, then a fixed-order reduction) while every part keeps at least
+  // 32 stages; shorter parts measured no faster than the unsplit product.
+  // The choice depends on the plan's shapes only, so every wave of a capped
+  // plan makes the same one.
+  {
+    int nk_min = 1 << 30;
+    for (int i = 0; i < n; ++i) nk_min = std::min(nk_min, (pl->mats[i].n + kBK - 1) / kBK);
+    int split = 1;
+    for (int sp : {4, 2})
+      if (cnt_sym * sp * 5 <= static_cast<size_t>(pl->npairs) * 6 && nk_min >= 32 * sp) {
+        split = sp;
+        break;
+      }
+    if (const char* env = std::getenv("MUON_SPLITK")) {  // diagnostic: force the split (1, 2 or 4)
+      const int v = std::atoi(env);
+      if ((v == 1 || v == 2 || v == 4) && nk_min >= 4 * v) split = v;
+    }
+    pl->split = split;
+  }
+  const int split = pl->split;
+  size_t cnt_red = 0;  // 32 x 32 blocks on or below the diagonal of every symmetric product
+  if (split > 1)
+    for (int i = 0; i < n; ++i) {
+      const size_t b = (pl->mats[i].m + 31) / 32;
+      cnt_red += b * (b + 1) / 2;
+    }
+  const size_t fixed = fixed_bytes(cnt_sym, cnt_full, cnt_sym32, cnt_full32, cnt_chunk) +
+                       round_up(cnt_red * sizeof(int4), 256) +
+                       (split > 1 ? round_up(cnt_sym * split * sizeof(TcTile), 256) : 0);
 
+  if (split > 1) ba += 4 * static_cast<size_t>(split);  // fp32 parts of the symmetric products
   // ---- waves: with a workspace cap, matrices are packed first-fit in LPT
   // order into waves whose iterate and symmetric arrays fit what the cap
   // leaves after the fixed structures.  The arrays are shared by all waves and
@@ -575,6 +638,7 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
     }
     wv.nchunks = static_cast<int>(chunks.size()) - wv.chunk_off;
     wv.sym_off = static_cast<int>(sym.size());
+    wv.symg_off = static_cast<int>(symg.size());
     wv.full_off = static_cast<int>(full.size());
     wv.sym32_off = static_cast<int>(sym32.size());
     wv.full32_off = static_cast<int>(full32.size());
@@ -584,6 +648,11 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
       for_each_sym_tile(mi.m, [&](TcTile t) {
         t.p = i;
         sym.push_back(t);
+        if (split > 1)
+          for (int kp = 0; kp < split; ++kp) {  // the parts of a tile side by side
+            t.kpart = kp;
+            symg.push_back(t);
+          }
       });
       for_each_full_tile(mi.rows, mi.cols, [&](TcTile t) {
         t.p = i;
@@ -597,6 +666,16 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
       }
     }
     wv.n_sym = static_cast<int>(sym.size()) - wv.sym_off;
+    wv.n_symg = static_cast<int>(symg.size()) - wv.symg_off;
+    wv.red_off = static_cast<int>(red.size());
+    if (split > 1)
+      for (int i : order) {
+        if (wave_of[i] != w) continue;
+        const int m = pl->mats[i].m;
+        for (int i0 = 0; i0 < m; i0 += 32)
+          for (int j0 = 0; j0 <= i0; j0 += 32) red.push_back(make_int4(i, i0, j0, 0));
+      }
+    wv.n_red = static_cast<int>(red.size()) - wv.red_off;
     wv.n_full = static_cast<int>(full.size()) - wv.full_off;
     wv.n_sym32 = static_cast<int>(sym32.size()) - wv.sym32_off;
     wv.n_full32 = static_cast<int>(full32.size()) - wv.full32_off;
@@ -617,6 +696,7 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   };
   const size_t o_hi0 = take(total_x * 2), o_hi1 = take(total_x * 2), o_lo = take(total_x * 2);
   const size_t o_A = take(total_a * 2), o_B = take(total_a * 2);
+  const size_t o_part = split > 1 ? take(total_a * 4 * static_cast<size_t>(split)) : 0;
   size_t o_x0 = 0, o_x1 = 0, o_a32 = 0, o_b32 = 0;
   if (pl->fp32_ws) {
     o_x0 = take(total_x * 4);
@@ -639,6 +719,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   const size_t o_full32 = take(std::max<size_t>(1, full32.size()) * sizeof(TileDesc));
   const size_t o_chunks = take(chunks.size() * sizeof(ChunkDesc));
   const size_t o_tmaps = take(static_cast<size_t>(n) * kMapsPerMat * sizeof(CUtensorMap));
+  const size_t o_red = take(std::max<size_t>(1, red.size()) * sizeof(int4));
+  const size_t o_symg = take(std::max<size_t>(1, symg.size()) * sizeof(TcTile));
   pl->dbytes = off;
   if (capped && pl->dbytes > max_workspace_bytes) {  // the packing above accounts for every byte
     free_plan(pl);
@@ -668,6 +750,12 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   ws.rms_part = reinterpret_cast<float*>(b + o_rms);
   ws.status = reinterpret_cast<unsigned*>(b + o_status);
   ws.unorm = reinterpret_cast<float*>(b + o_unorm);
+  if (split > 1) {
+    ws.part = reinterpret_cast<float*>(b + o_part);
+    ws.part_stride = static_cast<int64_t>(total_a);
+  }
+  pl->reduce_d = reinterpret_cast<int4*>(b + o_red);
+  pl->symg_d = reinterpret_cast<TcTile*>(b + o_symg);
   pl->mats_d = reinterpret_cast<MatInfo*>(b + o_mats);
   for (int k = 0; k < muon_plan_s::kPtrSlots; ++k) pl->slots[k].dev = reinterpret_cast<MatPtrs*>(b + o_ptrs) + k * n;
   pl->ptrs_d = pl->slots[0].dev;
@@ -683,7 +771,8 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
   for (int i = 0; i < n; ++i) {
     const MatInfo& mi = pl->mats[i];
     if (!encode_matrix_maps(&tmaps[static_cast<size_t>(kMapsPerMat) * i], mi, ws.hi[0] + mi.off_x,
-                            ws.hi[1] + mi.off_x, ws.lo + mi.off_x, ws.A + mi.off_a, ws.B + mi.off_a)) {
+                            ws.hi[1] + mi.off_x, ws.lo + mi.off_x, ws.A + mi.off_a, ws.B + mi.off_a,
+                            split > 1 ? ws.part + mi.off_a : nullptr, ws.part_stride, split)) {
       free_plan(pl);
       return MUON_ERR_CUDA;
     }
@@ -701,6 +790,10 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
                                            cudaMemcpyHostToDevice) == cudaSuccess);
   ok = ok && cudaMemcpy(pl->chunks_d, chunks.data(), chunks.size() * sizeof(ChunkDesc), cudaMemcpyHostToDevice) ==
                  cudaSuccess;
+  ok = ok && (red.empty() || cudaMemcpy(pl->reduce_d, red.data(), red.size() * sizeof(int4), cudaMemcpyHostToDevice) ==
+                                 cudaSuccess);
+  ok = ok && (symg.empty() || cudaMemcpy(pl->symg_d, symg.data(), symg.size() * sizeof(TcTile),
+                                         cudaMemcpyHostToDevice) == cudaSuccess);
   ok = ok && cudaMemcpy(pl->tmaps_d, tmaps.data(), tmaps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) ==
                  cudaSuccess;
   ok = ok && cudaMemset(ws.norm_count, 0, n * sizeof(unsigned)) == cudaSuccess;

@@ -48,12 +48,16 @@ constexpr int kT32 = 64;           // fp32 path tile edge
 //                         lo in one 3-D box {32, 32, 2} (the third dimension steps from hi to
 //                         lo), 64-byte swizzle
 //   kMapStA, kMapStB      epilogue store boxes of 32 x 32, 64-byte swizzle
+//   kMapStPart            split-K partial products (fp32): a 32 x 32 box of one
+//                         part, 3-D {cols, rows, part}, 128-byte swizzle
 enum MapIndex : int {
   kMapHi0 = 0, kMapHi1 = 1, kMapA = 2, kMapB = 3,
   kMapHi0S = 4, kMapHi1S = 5, kMapAS = 6, kMapBS = 7,
   kMapStHiLo0 = 8, kMapStHiLo1 = 9, kMapStA = 10, kMapStB = 11,
-  kMapsPerMat = 12
+  kMapStPart = 12,
+  kMapsPerMat = 13
 };
+constexpr int kMaxSplit = 4;  // split-K parts of a symmetric product
 constexpr int kEpiBoxCols = 32;
 
 // device status bits (sticky, cleared by muon_get_status)
@@ -119,7 +123,7 @@ struct TcTile {
   int32_t p;       // matrix
   int32_t n_need;  // accumulator columns that hold output (1..256)
   int32_t flags;   // kTileGhost1, kTileDiagOnly
-  int32_t pad_;
+  int32_t kpart;   // split-K part of the K range (0 unless the launch splits K)
   int32_t r0, r1;  // first output row of CTA 0 / CTA 1
   int32_t c0, c1;  // first B-operand row (output column) staged by CTA 0 / CTA 1
 };
@@ -212,6 +216,8 @@ struct Workspace {
   float* rms_part;      // per tile-warp / chunk: sum of O^2
   unsigned* status;
   float* unorm;         // per matrix: rms_scale / RMS(O) of the Eq. 6 update norm
+  float* part;          // split-K partial products, part k at part + k * part_stride, A's layout
+  int64_t part_stride;  // elements between parts
 };
 
 struct StepScalars {
@@ -242,6 +248,7 @@ struct GemmArgs {
   Workspace ws;
   StepScalars sc;
   unsigned long long test_wait_ns;  // 0; > 0 only for the failure-detection test (see muon_inject_wait_timeout)
+  int split;            // > 1: this symmetric launch computes K in `split` parts into ws.part
 };
 
 // Arguments of the fp32 SIMT GEMM kernel.
@@ -275,7 +282,14 @@ cudaError_t launch_gemm_tc(const GemmArgs& args, int npairs, cudaStream_t st);
 // Encode the kMapsPerMat TMA descriptors of one matrix (host); false if the
 // driver entry point is missing or rejects a descriptor.
 bool encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0, __nv_bfloat16* hi1, __nv_bfloat16* lo,
-                        __nv_bfloat16* A, __nv_bfloat16* B);
+                        __nv_bfloat16* A, __nv_bfloat16* B, float* part = nullptr, int64_t part_stride = 0,
+                        int nparts = 0);
+// Sum the split-K parts of a symmetric product in part order, apply the
+// phase's epilogue arithmetic (Gram: scale; polynomial: b A + c (.) + a I),
+// round to bf16 and write the lower triangle and its mirror into A or B.
+// blocks: (matrix, i0, j0, 0) for every 32 x 32 block with i0 >= j0.
+cudaError_t launch_split_reduce(const int4* blocks, int nblocks, const MatInfo* mats, Workspace ws, StepScalars sc,
+                                int phase, int iter, int split, cudaStream_t st);
 int gemm_tc_max_pairs();
 cudaError_t launch_gemm_f32(const Gemm32Args& args, cudaStream_t st);
 int gemm_tc_smem_bytes();

@@ -71,6 +71,45 @@ def test_symmetric_products_row_by_row(coeffs):
     assert max(worst.values()) <= TOL_ROW, worst
 
 
+@pytest.mark.parametrize("split", [2, 4])
+def test_split_k_gram_row_by_row(split, monkeypatch):
+    """One matrix per plan with the Gram product's K range split into parts
+    (fp32 partial products and a fixed-order reduction).  Plans choose the
+    split for single matrices with a long K (2048 x 8192 takes 2 parts);
+    MUON_SPLITK forces it here on every shape.  Same row-by-row check of
+    X1 = (X X^T) X, and a repeated call is bitwise equal."""
+    monkeypatch.setenv("MUON_SPLITK", str(split))
+    abc = tuple(f32(v) for v in (0.0, 1.0, 0.0))
+    worst = {}
+    for k, s in enumerate(SHAPES):
+        plan = MuonPlan([s])
+        x, h = random_bf16(s, 800 + k)
+        o1 = torch.full(s, float("nan"), device="cuda")
+        o2 = torch.full(s, float("nan"), device="cuda")
+        plan.orthogonalize([x], [o1], ns_steps=1, coeffs=abc)
+        plan.orthogonalize([x], [o2], ns_steps=1, coeffs=abc)
+        torch.cuda.synchronize()
+        assert plan.status() == 0
+        assert torch.equal(o1, o2)
+        got, want = host64(o1), orc.newton_schulz(h, 1, abc)
+        if s[0] > s[1]:
+            got, want = got.T, want.T
+        worst[s] = float(_row_errors(got, want).max())
+        plan.close()
+    assert max(worst.values()) <= TOL_ROW, worst
+    # and the method's five iterations on the same plans, within the acceptance bound
+    errs = {}
+    for k, s in enumerate(SHAPES):
+        plan = MuonPlan([s])
+        x, h = random_bf16(s, 900 + k)
+        o = torch.full(s, float("nan"), device="cuda")
+        plan.orthogonalize([x], [o], ns_steps=5, coeffs=ABC32)
+        torch.cuda.synchronize()
+        errs[s] = rel_f(host64(o), orc.newton_schulz(h, 5, ABC32))
+        plan.close()
+    assert max(errs.values()) <= TOL_O_BF16, errs
+
+
 def test_symmetric_tiles_five_iterations():
     """The method's five iterations on the same shapes, within the acceptance bound."""
     plan = MuonPlan(SHAPES)
