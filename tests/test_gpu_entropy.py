@@ -12,6 +12,12 @@ Bounds, from the arithmetic:
 - The outputs are fp32: H (|H| <= 1) is rounded to 6e-8 and each singular
   value to 6e-8 relative, so sigma^2 to 1.2e-7 relative.
 So H is checked to 2e-7 absolute and sigma^2 to 3e-7 sigma_max^2 per value.
+That sigma^2 bound is relative to the largest eigenvalue only: the 1e-6 stop
+allows an absolute error of a few 1e-9 sigma_max^2 on every eigenvalue, so on
+a spectrum spanning three decades of sigma (six of sigma^2) the smallest
+sigma^2 may be off by about 1e-3 of itself.  H is insensitive to that (those
+values carry almost no energy); a user who needs the small singular values
+to a relative accuracy would need a tighter stop.
 """
 
 import math
