@@ -62,15 +62,15 @@ def kernel_source_hash() -> str:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
-def ncu_traffic(units: float):
-    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary,
-    scaled to this run's launch size; None unless the summary was taken on
-    the current kernel source."""
+def ncu_traffic(workload: str):
+    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary
+    (scaled there to one launch of the workload it names); None unless the
+    summary was taken on the current kernel source and on this workload."""
     p = os.path.join(ROOT, "profiles", "ns_gemm_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("kernel_sha256_16") != kernel_source_hash():
+    if d.get("kernel_sha256_16") != kernel_source_hash() or d.get("workload") != workload:
         return None
     return d.get("bytes_per_launch")
 
@@ -198,19 +198,13 @@ def bench_adamw(dev, steps: int = 20, warmup: int = 3):
             "peak_source": f"hbm_gbs ({kind})", "frac": gbs / peak, "bytes_per_elem": ADAMW_BYTES_PER_ELEM}
 
 
-# fp64 CUDA-core peak, derived: 148 SMs x 64 FP64 FMA per clock x 2 FLOP x 1.965 GHz
-FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
-
-
-def entropy_update_flops(shapes, sweeps) -> float:
-    """FLOPs of jacobi_update_kernel over a call: per matrix and sweep, nb - 1
-    rounds of (nb/2)(nb/2 + 1)/2 super-blocks, each two 64 x 64 x 64 products."""
+def entropy_trailing_bytes(shapes) -> float:
+    """Bytes the tridiagonal reduction streams for G0 v: the trailing
+    (m-1-j) x (m-1-j) fp64 block once per column j, summed over columns."""
     total = 0.0
-    for (r, c), sw in zip(shapes, sweeps):
-        nb = -(-min(r, c) // 32)
-        nb += nb % 2
-        pairs = nb // 2
-        total += sw * (nb - 1) * pairs * (pairs + 1) / 2 * 4 * 64 ** 3
+    for r, c in shapes:
+        m = min(r, c)
+        total += 8.0 * (m - 1) * m * (2 * m - 1) / 6.0
     return total
 
 
@@ -234,15 +228,18 @@ def bench_entropy(Ws, calls: int = 2):
     phases = plan.profile_read()
     st, sweeps = plan.status()
     plan.close()
-    flops = entropy_update_flops(shapes, sweeps)
-    achieved = flops / (phases["jacobi"] * 1e-3) / 1e12
-    return {"what": "SVD entropy (Sec. 3.4) of every weight matrix after the timed steps: fp64 Gram, "
-                    "two-sided block Jacobi, entropy; one call covers all matrices",
+    nbytes = entropy_trailing_bytes(shapes)
+    achieved = nbytes / (phases["tridiagonal"] * 1e-3) / 1e9
+    peaks, kind = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"what": "SVD entropy (Sec. 3.4) of every weight matrix after the timed steps: fp64 Gram, Householder "
+                    "tridiagonal reduction, bisection on Sturm counts, entropy; one call covers all matrices",
             "matrices": len(Ws), "ms_per_call": ms, "phases_ms": phases, "status": st,
-            "sweeps": [min(sweeps), max(sweeps)], "kernel": "jacobi_update_kernel (fp64 CUDA cores)",
-            "bound": "alu", "achieved": achieved, "unit": "TFLOP/s (fp64)", "peak": FP64_PEAK_TFLOPS,
-            "peak_source": "derived: 148 SMs x 64 FP64 FMA/clk x 2 x 1.965 GHz", "frac": achieved / FP64_PEAK_TFLOPS,
-            "achieved_basis": "update-kernel FLOPs over the whole Jacobi phase (solves and checks included)"}
+            "computed": [min(sweeps), max(sweeps)], "kernel": "tridiag_kernel (fp64, one CTA per matrix)",
+            "bound": "hbm", "achieved": achieved, "unit": "GB/s", "peak": hbm, "peak_source": f"hbm_gbs ({kind})",
+            "frac": achieved / hbm,
+            "achieved_basis": "the trailing block streamed once per column for G0 v (8 sum L^2 bytes per matrix) "
+                              "over the whole reduction phase (panel updates and reflectors included)"}
 
 
 # ---------------------------------------------------------------------- oracle (CPU) legs
@@ -415,7 +412,7 @@ def hybrid_mixed8(dev, steps: int = 5, warmup: int = 3):
         opt.step(mats, vecs, t=t, lr=4.2e-4, weight_decay=0.1)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    opt.muon.profile(True)
+    opt.muon.profile(True, spans=True)
     opt.muon.profile_read()
     e0.record()
     for t in range(warmup + 1, warmup + steps + 1):
@@ -427,7 +424,7 @@ def hybrid_mixed8(dev, steps: int = 5, warmup: int = 3):
     st = opt.status()
     opt.close()
     nz = sum(ns_flops(r, c, 5) for i, (r, c) in enumerate(shapes) if i not in wl.zero_grad)
-    gemm_ms = sum(prof["ms"][x] for x in ("gram", "poly", "x_update")) / max(prof["calls"], 1)
+    gemm_ms = prof["ms"]["newton_schulz"] / max(prof["calls"], 1)
     del mats, vecs, Wbuf, Gbuf, Mbuf
     torch.cuda.empty_cache()
     return {"what": "full optimizer step of the 8-layer mixed MoE: Muon over 1624 matrices + AdamW over 16 decayed "
@@ -571,7 +568,11 @@ def main(argv=None) -> int:
     # ---- timed region: inputs resident in HBM
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    plan.profile(True)
+    # span profile: CUDA events after the momentum pass, around each wave's
+    # Newton-Schulz chain and after the update passes, none between two
+    # product launches (their set-up overlaps through programmatic dependent
+    # launch, which an event in between would serialise)
+    plan.profile(True, spans=True)
     plan.profile_read()
     barrier()
     torch.cuda.synchronize()
@@ -586,6 +587,17 @@ def main(argv=None) -> int:
     prof = plan.profile_read()
     ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
     value = replica_tflops(world, nz_flops, ms_step)
+
+    # ---- per-phase breakdown: a few more steps after the timed region with
+    # an event after every launch (diagnostic; not part of `value`)
+    diag_steps = min(args.steps, 5)
+    plan.profile(True)
+    plan.profile_read()
+    for _ in range(diag_steps):
+        plan.step(**hp, update_rms=rms)
+    torch.cuda.synchronize()
+    plan.profile(False)
+    prof_launch = plan.profile_read()
 
     # ---- end to end: pinned host gradients in, update RMS out, every step.
     # Two device gradient buffers: the copy of step k+1's gradients (its own
@@ -655,14 +667,16 @@ def main(argv=None) -> int:
 
     peaks, peak_kind = load_peaks()
     calls = max(prof["calls"], 1)
-    gemm_ms = sum(prof["ms"][k] for k in ("gram", "poly", "x_update")) / calls
-    gemm_launches = sum(prof["launches"][k] for k in ("gram", "poly", "x_update")) / calls
-    per_step_launches = sum(prof["launches"].values()) / calls
+    gemm_ms = prof["ms"]["newton_schulz"] / calls
+    gemm_launches = prof["launches"]["newton_schulz"] / calls
+    per_step_launches = sum(v for k, v in prof["launches"].items() if k != "newton_schulz") / calls
+    dcalls = max(prof_launch["calls"], 1)
+    phase_launch_ms = {k: v / dcalls for k, v in prof_launch["ms"].items()}
     achieved = nz_flops / (gemm_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     k1_ms = prof["ms"]["momentum_normalise"] / calls
     k1_gbs = total * K1_BYTES_PER_ELEM / (k1_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(gemm_launches)
+    traffic = ncu_traffic(wl.name)
 
     context = None
     if not args.no_context:
@@ -714,8 +728,14 @@ def main(argv=None) -> int:
         "ns_ms_per_step": gemm_ms, "ns_tflops": achieved,
         "ns_pct_of_bf16_peak": 100.0 * achieved / peak,
         "ns_tflops_dense_equivalent": dense_flops / (gemm_ms * 1e-3) / 1e12,
-        "phase_ms_per_step": {k: v / calls for k, v in prof["ms"].items()},
+        "phase_ms_per_step": {k: v / calls for k, v in prof["ms"].items() if k not in ("gram", "poly", "x_update")},
+        "phase_ms_per_step_launch_events": dict(
+            phase_launch_ms, note=f"{diag_steps} steps after the timed region with a CUDA event after every launch "
+                                  "(no launch overlap); diagnostic, not part of value"),
         "roofline": {"kernel": "ns_gemm_kernel (tcgen05, all Gram/poly/X-update launches)", "bound": "tensor",
+                     "launch_time_source": "CUDA events on the launching stream around each wave's Newton-Schulz "
+                                           "chain inside the timed region; average launch duration = span / "
+                                           "launches",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"bf16_tflops_sustained ({peak_kind})", "traffic": traffic,
                      "algorithmic_flops_per_launch": nz_flops / gemm_launches},

@@ -56,7 +56,7 @@ typedef enum {
   MUON_ERR_NONFINITE = 6,      /* (muon_get_status) a Frobenius norm was NaN or Inf */
   MUON_ERR_TIMEOUT = 7,        /* (muon_get_status) a device-side wait gave up; results of that call are invalid */
   MUON_ERR_ALIAS = 8,          /* W, G, M (or X_in, O_out) buffers overlap */
-  MUON_ERR_NOT_CONVERGED = 9   /* (muon_entropy_get_status) an eigenvalue iteration hit its sweep limit */
+  MUON_ERR_NOT_CONVERGED = 9   /* reserved: an iteration hit its limit (the current solvers have none) */
 } muon_status_t;
 
 typedef enum { MUON_DT_BF16 = 0, MUON_DT_FP32 = 1 } muon_dtype_t;
@@ -210,12 +210,26 @@ MUON_API void muon_destroy(muon_plan_t plan);
 /* Static English text for a status code (never NULL). */
 MUON_API const char* muon_status_string(muon_status_t s);
 
-/* Phase timing, for measurement.  When enabled, every step/orthogonalize call
- * records CUDA events on its stream at each phase boundary.  Phases:
- * 0 momentum/normalise, 1 Gram (X X^T), 2 polynomial (b A + c A^2),
- * 3 X update (a X + B X), 4 the update pass over the last iterate (weight
- * update or O output), the Eq. 6 reduction and the RMS finalisation. */
-#define MUON_NUM_PHASES 5
+/* Phase timing, for measurement.  Phases: 0 momentum/normalise, 1 Gram
+ * (X X^T), 2 polynomial (b A + c A^2), 3 X update (a X + B X), 4 the update
+ * pass over the last iterate (weight update or O output), the Eq. 6
+ * reduction and the RMS finalisation, 5 Newton-Schulz (phases 1-3 together,
+ * split-K reductions included).
+ *
+ * enable = MUON_PROFILE_LAUNCHES (1): every step/orthogonalize call records a
+ * CUDA event on its stream after every launch; each launch's time goes to its
+ * phase, and the product launches' time also to phase 5.
+ * enable = MUON_PROFILE_SPANS (2): events only where the kernel class
+ * changes (after the momentum pass, after the last product launch of each
+ * wave, after each update pass).  Phases 1-3 then count launches but get no
+ * time and phase 5 gets each wave's whole Newton-Schulz span.  The product
+ * launches overlap by their set-up (programmatic dependent launch), which an
+ * event between two of them prevents, so this mode times the chain as it
+ * runs unprofiled.
+ * enable = 0 stops recording.  Other values: MUON_ERR_INVALID_ARG. */
+#define MUON_NUM_PHASES 6
+#define MUON_PROFILE_LAUNCHES 1
+#define MUON_PROFILE_SPANS 2
 MUON_API muon_status_t muon_profile_enable(muon_plan_t plan, int32_t enable);
 
 /* Synchronizes, then adds the elapsed milliseconds of every recorded call
@@ -345,17 +359,19 @@ MUON_API void muon_adamw_destroy(muon_adamw_plan_t plan);
  *   H = -(1 / log n) sum_i p_i log p_i,   p_i = sigma_i^2 / sum_j sigma_j^2
  * with 0 log 0 = 0.  H is NaN for a zero matrix, for n = 1 (both 0 / 0) and
  * for a matrix with non-finite entries.
- * sigma_i^2 are the eigenvalues of the fp32 Gram matrix of the wide
- * orientation, found by two-sided block Jacobi in fp64 (32-row blocks, at
- * most 24 sweeps, stopped once the off-diagonal Frobenius norm is below 1e-6
- * of the whole); the entropy sums run in fp64 too.
+ * sigma_i^2 are the eigenvalues of the Gram matrix of the wide orientation,
+ * formed in fp64 from the fp32 entries, reduced to tridiagonal form by
+ * Householder reflections (fp64, one CTA per matrix) and found by bisection
+ * on Sturm counts (fp64, to 2 eps of the largest); the entropy sums run in
+ * fp64 too.
  * ------------------------------------------------------------------------ */
 typedef struct muon_entropy_plan_s* muon_entropy_plan_t;
 
 /* Plan for n >= 1 fp32 matrices: shapes[2 i] = rows, shapes[2 i + 1] = cols,
  * each >= 1 with rows * cols < 2^31.  min(rows, cols) <= 8192, else
  * MUON_ERR_UNSUPPORTED.  Allocates the fp64 Gram workspace (about 8 m^2 bytes
- * per matrix, m = min(rows, cols)) and the rotation store.  Errors:
+ * per matrix, m = min(rows, cols)) and a panel store of 512 m bytes per
+ * matrix.  Errors:
  * INVALID_ARG, UNSUPPORTED, NO_MEMORY, CUDA. */
 MUON_API muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64_t* shapes, int32_t n, void* stream);
 
@@ -377,18 +393,20 @@ MUON_API muon_status_t muon_entropy_compute(muon_entropy_plan_t plan, const floa
 MUON_API int64_t muon_entropy_num_singular_values(muon_entropy_plan_t plan);
 
 /* Synchronises the plan's last stream, then returns and clears the sticky
- * status of the calls since the previous read: MUON_OK, MUON_ERR_NONFINITE
- * (a matrix had non-finite entries; its H is NaN) or MUON_ERR_NOT_CONVERGED
- * (a matrix used all 24 sweeps; its H comes from the last iterate).
+ * status of the calls since the previous read: MUON_OK or
+ * MUON_ERR_NONFINITE (a matrix had non-finite entries; its H and singular
+ * values are NaN).
  * sweeps_out: NULL or a host int32 array [n] that receives, for the last
- * call, the sweeps each matrix needed (0: not converged or non-finite).
+ * call, 1 for each matrix whose eigenvalues were computed (one reduction and
+ * bisection pass) and 0 for a non-finite one.
  * CUDA errors: MUON_ERR_CUDA. */
 MUON_API muon_status_t muon_entropy_get_status(muon_entropy_plan_t plan, int32_t* sweeps_out);
 
 /* Per-phase timing of the next calls with CUDA events when enable != 0.
- * ms_out: NULL, or a host double array [3] that receives the Gram, Jacobi
- * and entropy phase times of the last profiled call (waits for its events;
- * MUON_ERR_INVALID_ARG if no call was profiled). */
+ * ms_out: NULL, or a host double array [4] that receives the Gram,
+ * tridiagonal reduction, bisection and entropy phase times of the last
+ * profiled call (waits for its events; MUON_ERR_INVALID_ARG if no call was
+ * profiled). */
 MUON_API muon_status_t muon_entropy_profile(muon_entropy_plan_t plan, int32_t enable, double* ms_out);
 
 /* Waits for the plan's last stream and frees it; NULL is ignored. */

@@ -32,8 +32,11 @@ MUON_INIT_ZERO_MOMENTUM = 0x1
 MUON_INIT_FP32_NS = 0x2
 MUON_INIT_MAX_WORKSPACE = 0x4
 MUON_SCALE_MAX_DIM, MUON_SCALE_HIDDEN, MUON_SCALE_UPDATE_NORM = 0, 1, 2
-MUON_NUM_PHASES = 5
-PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize")
+MUON_NUM_PHASES = 6
+MUON_PROFILE_LAUNCHES = 1
+MUON_PROFILE_SPANS = 2
+PHASE_NAMES = ("momentum_normalise", "gram", "poly", "x_update", "finalize", "newton_schulz")
+ENTROPY_NUM_PHASES = 4
 
 EXPORTED = ("muon_hparams_default", "muon_init", "muon_init_ex", "muon_num_waves", "muon_inject_wait_timeout",
             "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
@@ -239,8 +242,8 @@ def muon_destroy(plan) -> None:
     load().muon_destroy(plan)
 
 
-def muon_profile_enable(plan, enable: bool) -> None:
-    check(load().muon_profile_enable(plan, 1 if enable else 0), "muon_profile_enable")
+def muon_profile_enable(plan, mode: int) -> None:
+    check(load().muon_profile_enable(plan, int(mode)), "muon_profile_enable")
 
 
 def muon_profile_read(plan):
@@ -297,7 +300,7 @@ def muon_entropy_get_status(plan, n: int):
 
 
 def muon_entropy_profile(plan, enable: bool, read: bool = False):
-    ms = (ctypes.c_double * 3)()
+    ms = (ctypes.c_double * ENTROPY_NUM_PHASES)()
     check(load().muon_entropy_profile(plan, 1 if enable else 0, ms if read else None), "muon_entropy_profile")
     return list(ms) if read else None
 

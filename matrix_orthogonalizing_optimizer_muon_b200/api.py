@@ -172,8 +172,12 @@ class MuonPlan:
         """Synchronizing read-and-clear of the device status (an int status code)."""
         return L.muon_get_status(self._plan)
 
-    def profile(self, enable: bool = True) -> None:
-        L.muon_profile_enable(self._plan, enable)
+    def profile(self, enable: bool = True, spans: bool = False) -> None:
+        """Record phase times of the following calls: an event after every
+        launch, or with spans=True only where the kernel class changes (the
+        Newton-Schulz chain of each wave as one span, phase newton_schulz)."""
+        mode = 0 if not enable else (L.MUON_PROFILE_SPANS if spans else L.MUON_PROFILE_LAUNCHES)
+        L.muon_profile_enable(self._plan, mode)
 
     def profile_read(self):
         ms, cnt, calls = L.muon_profile_read(self._plan)
@@ -329,7 +333,7 @@ class EntropyPlan:
     current device (Sec. 3.4): H = -(1/log n) sum p_i log p_i with
     p_i = sigma_i^2 / sum sigma_j^2 over the n = min(rows, cols) singular values."""
 
-    _PHASES = ("gram", "jacobi", "entropy")
+    _PHASES = ("gram", "tridiagonal", "bisection", "entropy")
 
     def __init__(self, shapes, *, stream=None):
         self.shapes = [tuple(int(v) for v in s) for s in shapes]
@@ -360,7 +364,8 @@ class EntropyPlan:
         return H
 
     def status(self):
-        """(status code, sweeps per matrix of the last call); synchronising."""
+        """(status code, per matrix of the last call 1 if its eigenvalues were
+        computed and 0 if it was non-finite); synchronising."""
         return L.muon_entropy_get_status(self._plan, self.n)
 
     def profile(self, enable: bool = True) -> None:

@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kEwThreads) k1_kernel(const ChunkDesc* __restr
                                                         StepScalars sc, int mode, int fp32_path) {
   __shared__ double red[kEwThreads / 32];
   __shared__ int am_last;
+  pdl_wait();
+  pdl_trigger();
   const ChunkDesc ch = chunks[blockIdx.x];
   const int p = ch.x;
   const MatInfo mi = mats[p];
@@ -223,6 +225,8 @@ __global__ void __launch_bounds__(kEwThreads) apply_update_kernel(const ChunkDes
                                                                   StepScalars sc, int final_mode, int fp32_path,
                                                                   int xbuf, int mul_s) {
   __shared__ float red[kEwThreads / 32];
+  pdl_wait();
+  pdl_trigger();
   const ChunkDesc ch = chunks[blockIdx.x];
   const int p = ch.x;
   const MatInfo mi = mats[p];
@@ -297,6 +301,8 @@ __global__ void __launch_bounds__(kEwThreads) update_norm_kernel(const ChunkDesc
                                                                  float* __restrict__ update_rms) {
   __shared__ double red[kEwThreads / 32];
   __shared__ bool am_last;
+  pdl_wait();
+  pdl_trigger();
   const ChunkDesc ch = chunks[blockIdx.x];
   const int p = ch.x;
   const MatInfo mi = mats[p];
@@ -360,6 +366,8 @@ __global__ void __launch_bounds__(kEwThreads) rms_finalize_kernel(const MatInfo*
                                                                   const float* __restrict__ part,
                                                                   float* __restrict__ out) {
   __shared__ double red[kEwThreads / 32];
+  pdl_wait();
+  pdl_trigger();
   const MatInfo mi = mats[blockIdx.x];
   double t = 0.0;
   for (int i = threadIdx.x; i < mi.nchunks; i += blockDim.x) t += (double)part[mi.chunk_base + i];
@@ -376,6 +384,8 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const int4* __restric
                                                            const MatInfo* __restrict__ mats, Workspace ws,
                                                            StepScalars sc, int phase, int iter, int split) {
   __shared__ __nv_bfloat16 tile[32][34];
+  pdl_wait();
+  pdl_trigger();
   const int4 bk = blocks[blockIdx.x];
   const MatInfo mi = mats[bk.x];
   const int i0 = bk.y, j0 = bk.z, m = mi.m;
@@ -419,34 +429,32 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const int4* __restric
 cudaError_t launch_split_reduce(const int4* blocks, int nblocks, const MatInfo* mats, Workspace ws, StepScalars sc,
                                 int phase, int iter, int split, cudaStream_t st) {
   if (nblocks == 0) return cudaSuccess;
-  split_reduce_kernel<<<nblocks, dim3(32, 8), 0, st>>>(blocks, mats, ws, sc, phase, iter, split);
-  return cudaGetLastError();
+  return launch_pdl(kPdlElementwise, split_reduce_kernel, dim3(nblocks), dim3(32, 8), 0, st, blocks, mats, ws, sc,
+                    phase, iter, split);
 }
 
 cudaError_t launch_k1(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
                       Workspace ws, StepScalars sc, int mode, int fp32_path, cudaStream_t st) {
-  k1_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, mode, fp32_path);
-  return cudaGetLastError();
+  return launch_pdl(kPdlElementwise, k1_kernel, dim3(nchunks), dim3(kEwThreads), 0, st, chunks, mats, ptrs, ws, sc,
+                    mode, fp32_path);
 }
 
 cudaError_t launch_apply_update(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, const MatPtrs* ptrs,
                                 Workspace ws, StepScalars sc, int final_mode, int fp32_path, int xbuf, int mul_s,
                                 cudaStream_t st) {
-  apply_update_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ptrs, ws, sc, final_mode, fp32_path, xbuf,
-                                                      mul_s);
-  return cudaGetLastError();
+  return launch_pdl(kPdlElementwise, apply_update_kernel, dim3(nchunks), dim3(kEwThreads), 0, st, chunks, mats,
+                    ptrs, ws, sc, final_mode, fp32_path, xbuf, mul_s);
 }
 
 cudaError_t launch_update_norm(const ChunkDesc* chunks, int nchunks, const MatInfo* mats, Workspace ws,
                                StepScalars sc, int fp32_path, int xbuf, int mul_s, float* update_rms,
                                cudaStream_t st) {
-  update_norm_kernel<<<nchunks, kEwThreads, 0, st>>>(chunks, mats, ws, sc, fp32_path, xbuf, mul_s, update_rms);
-  return cudaGetLastError();
+  return launch_pdl(kPdlElementwise, update_norm_kernel, dim3(nchunks), dim3(kEwThreads), 0, st, chunks, mats, ws,
+                    sc, fp32_path, xbuf, mul_s, update_rms);
 }
 
 cudaError_t launch_rms_finalize(const MatInfo* mats, int nmat, const float* part, float* out, cudaStream_t st) {
-  rms_finalize_kernel<<<nmat, kEwThreads, 0, st>>>(mats, part, out);
-  return cudaGetLastError();
+  return launch_pdl(kPdlElementwise, rms_finalize_kernel, dim3(nmat), dim3(kEwThreads), 0, st, mats, part, out);
 }
 
 }  // namespace muon

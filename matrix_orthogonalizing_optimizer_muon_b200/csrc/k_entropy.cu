@@ -7,38 +7,53 @@
 // over its n = min(rows, cols) singular values.
 //
 // sigma_i^2 are the eigenvalues of the Gram matrix G = X X^T of the wide
-// orientation X (m x n, m <= n) of W.  The path, all matrices of a plan per
-// launch:
+// orientation X (m x n, m <= n) of W.  Only the eigenvalues are needed, no
+// vectors, so G is reduced to a symmetric tridiagonal matrix T with the same
+// eigenvalues and those are found by bisection.  The path, all matrices of a
+// plan per launch:
 //   1. gram_kernel: G in fp64 on the CUDA cores (64 x 64 tiles of the lower
 //      triangle, each also written mirrored), zero-padded to m_pad, a
 //      multiple of 64.  Products of fp32 entries are exact in fp64.
-//   2. Two-sided block Jacobi on G.  The 32-row blocks are paired by a
-//      round-robin tournament, nb - 1 rounds per sweep.  In a round, every
-//      pair's 64 x 64 subproblem [G_PP G_PQ; G_QP G_QQ] gets one sweep of
-//      cyclic Jacobi in shared memory (jacobi_solve_kernel), which keeps the
-//      accumulated rotation V (re-orthonormalised by one polar Newton-Schulz
-//      step at the end); then G <- J^T G J for the block-diagonal J of all
-//      pairs, one 64 x 64 super-block per CTA iteration
-//      (jacobi_update_kernel: two small GEMMs, V_u^T T V_v).
-//   3. After each sweep, off_norm_kernel and converge_kernel compare the
-//      off-diagonal Frobenius norm with ||G||_F (fp64, fixed order).  A
-//      matrix below kOffTol is done; once all are done, every later launch
-//      returns at once.
-//   4. entropy_kernel: the diagonal now holds sigma_i^2.  fp64 sums in a
-//      fixed order give H; a bitonic sort gives the singular values,
-//      descending.
-// The zero padding never mixes with the matrix: a padded index has a zero
-// row and column, so every rotation that touches it is the identity.
-// Everything is deterministic (no atomics, fixed reduction orders).
+//   2. tridiag_kernel, one CTA per matrix: Householder reduction
+//      Q^T G Q = T (Golub and Van Loan, "Matrix Computations", Sec. 8.3.1) in
+//      panels of kTdNb columns, the blocked form of Dongarra, Sorensen and
+//      Hammarling ("Block reduction of matrices to condensed forms for
+//      eigenvalue computations", 1989).  Within a panel the matrix is
+//      G0 - V W^T - W V^T, G0 the matrix at the panel's start and V, W one
+//      column per reflector so far.  Column j is brought up to date from
+//      row j of G0 (G0 is symmetric) and V, W; its reflector
+//      H = I - tau v v^T (v_{j+1} = 1) zeroes rows j+2 .. m-1; then
+//      y = tau (G0 v - V (W^T v) - W (V^T v)) and w = y - (tau/2)(v^T y) v,
+//      because H B H = B - v w^T - w v^T for a symmetric B.  G0 v is the one
+//      pass over the trailing matrix per column.  At the panel's end the
+//      trailing matrix becomes G0 - V W^T - W V^T, computed on 64 x 64 tiles
+//      of the lower triangle and written with their mirror, so the stored
+//      matrix stays exactly symmetric.
+//   3. bisect_kernel: every eigenvalue of T by bisection on the Sturm count
+//      of T - x I (Golub and Van Loan, Sec. 8.4.1), one thread per
+//      eigenvalue.  The count is the number of negative pivots of the
+//      LDL^T factorisation, q_i = (d_i - x) - e_{i-1}^2 / q_{i-1}, the form
+//      whose floating-point count is exact for a matrix within a few ulps of
+//      T (Kahan); a pivot of magnitude below pivmin is replaced by -pivmin.
+//      Bisection runs from the Gershgorin interval to a width of
+//      2 eps ||T||, about 52 halvings.
+//   4. entropy_kernel: H from the eigenvalues with fp64 sums in a fixed
+//      order, and the singular values, descending (a bitonic sort makes the
+//      order exact).
+// Everything is deterministic: reductions run in a fixed order and the only
+// atomic is the sticky status flag.
 //
 // The arithmetic is fp64 throughout.  H weighs every eigenvalue by
 // -p log p, whose slope is unbounded near p = 0: with an fp32 Gram matrix the
 // rounding floor (about 1e-7 of the largest eigenvalue) alone moved H of a
-// rank-10 200 x 300 matrix by about 6e-5.
+// rank-10 200 x 300 matrix by about 6e-5.  The reduction is backward stable:
+// T has the eigenvalues of a matrix within a small multiple of
+// m eps ||G|| of G, and bisection adds 2 eps ||T||.
 #include "muon.h"
 #include "muon_internal.cuh"
 
 #include <algorithm>
+#include <cfloat>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -47,35 +62,26 @@
 namespace muon {
 namespace {
 
-constexpr int kEb = 32;              // rows of a Jacobi block
-constexpr int kEs = 2 * kEb;         // order of a block-pair subproblem
-constexpr int kEsLd = kEs + 1;       // shared-memory row pitch (conflict-free columns)
-constexpr int kEsElems = kEs * kEs;  // 4096
 constexpr int kEThreads = 256;
 constexpr int kGramTile = 64;
 constexpr int kGramK = 32;
-constexpr int kMaxSweeps = 24;
-// One cyclic sweep per subproblem and round: solving the 64 x 64 problems to
-// convergence (up to 10 sweeps) saved at most one outer sweep in fp64
-// simulations of 704 x 704 Gram matrices (Gaussian: 11 against 10; three
-// decades of singular values: 17 against 17) for five times the inner work.
-constexpr int kInnerSweeps = 1;
 constexpr int kMaxDim = 8192;        // min(rows, cols) limit (the sort stages 8192 values)
 constexpr int kSortThreads = 1024;
-// A pair (a, b) of a subproblem is rotated when |S_ab| > kInnerTol max(|S_aa|, |S_bb|):
-// a skipped entry moves an eigenvalue by at most S_ab^2 / |S_aa - S_bb|, or by
-// |S_ab| itself for a near-degenerate pair.
-constexpr double kInnerTol = 1e-13;
-// A matrix is done when off(G) <= kOffTol ||G||_F (Frobenius norms).  The
-// rest moves the eigenvalues by second-order amounts: in the same
-// simulations at most 3e-9 of the largest eigenvalue, and H by 1e-10, far
-// below the rounding of the fp32 outputs.
-constexpr double kOffTol = 1e-6;
-constexpr size_t kSolveSmem = 2 * kEs * kEsLd * sizeof(double);
-constexpr size_t kUpdSmem = 3 * kEs * (kEs + 2) * sizeof(double);
+
+constexpr int kTdThreads = 512;      // tridiagonal reduction: one CTA per matrix
+constexpr int kTdWarps = kTdThreads / 32;
+constexpr int kTdNb = 32;            // columns per panel
+constexpr int kTdTile = 64;          // trailing-update tile
+// shared memory of tridiag_kernel, in doubles: the column x, the reflector
+// v and the product y (m_pad each) plus small arrays; the trailing update
+// reuses the space for its operand tiles and the output tile
+constexpr int kTdSmall = 4 * kTdNb + 2 * kTdWarps + 16;
+constexpr int kTdTrail = 4 * kTdNb * kTdTile + kTdTile * (kTdTile + 1);
+
+constexpr int kBisThreads = 256;     // bisection: one thread per eigenvalue
+constexpr int kBisMaxIter = 64;
 
 // conv[] values
-constexpr int kConvRunning = 0;
 constexpr int kConvDone = 1;
 constexpr int kConvNonFinite = 2;
 
@@ -83,40 +89,21 @@ struct EntMat {
   int rows, cols;
   int m, n;         // min and max of rows, cols
   int tall;         // rows > cols: X = W^T
-  int nb;           // 32-row blocks, even; m_pad = 32 nb
-  int rb_first;     // first row block of this matrix in the off-norm partials
-  int pad_;
-  int64_t off_g;    // doubles into the G workspace (m_pad x m_pad, row-major)
-  int64_t off_v;    // doubles into the rotation store (nb / 2 blocks of 64 x 64)
-  int64_t sv_off;   // first singular value of this matrix in sigma_out
+  int mp;           // m rounded up to a multiple of 64: G's row pitch
+  int64_t off_g;    // doubles into the G workspace (mp x mp, row-major)
+  int64_t off_vw;   // doubles into the panel store (V then W, kTdNb x mp each)
+  int64_t sv_off;   // first eigenvalue / singular value of this matrix
 };
 
 struct EntCtl {
   int* conv;        // [n] kConv*
-  int* sweeps;      // [n] sweeps until done (0: not done)
-  int* all_done;    // [1] every matrix is done
-  unsigned* status; // [1] sticky: kStatusNonFinite, kStatusNotConverged
+  int* sweeps;      // [n] 1 once the eigenvalues are computed, 0 for a non-finite matrix
+  unsigned* status; // [1] sticky: kStatusNonFinite
 };
 
-constexpr unsigned kStatusNotConverged = 4u;
-
-// round-robin tournament over nb players (nb even), round r in [0, nb - 1):
-// player nb - 1 meets r, and for u >= 1 player (r + u) mod (nb - 1) meets
-// (r - u) mod (nb - 1).  Every pair meets once per nb - 1 rounds.
-__host__ __device__ __forceinline__ int2 tournament(int nb, int r, int u) {
-  int a, b;
-  if (u == 0) {
-    a = nb - 1;
-    b = r;
-  } else {
-    a = (r + u) % (nb - 1);
-    b = (r - u + (nb - 1)) % (nb - 1);
-  }
-  return make_int2(a < b ? a : b, a < b ? b : a);
+size_t tridiag_smem_bytes(int mp) {
+  return static_cast<size_t>(std::max(3 * mp + kTdSmall, kTdTrail)) * sizeof(double);
 }
-
-// row of G for index a in [0, 64) of the subproblem of block pair (P, Q)
-__device__ __forceinline__ int sub_row(int2 pq, int a) { return a < kEb ? pq.x * kEb + a : pq.y * kEb + (a - kEb); }
 
 // ---------------------------------------------------------------- 1. Gram
 __device__ __forceinline__ float x_at(const float* W, const EntMat& mi, int i, int k) {
@@ -178,7 +165,7 @@ __global__ void __launch_bounds__(kEThreads) gram_kernel(const int4* __restrict_
     for (int w = 0; w < 4; ++w) Cs[ty * 4 + q][tx + 16 * w] = acc[q][w];
   __syncthreads();
   double* g = G + mi.off_g;
-  const size_t ld = static_cast<size_t>(kEb) * mi.nb;
+  const size_t ld = static_cast<size_t>(mi.mp);
   for (int e = t; e < kGramTile * kGramTile; e += kEThreads) {
     const int r = e >> 6, c = e & 63;
     g[(i0 + r) * ld + j0 + c] = Cs[r][c];
@@ -186,307 +173,344 @@ __global__ void __launch_bounds__(kEThreads) gram_kernel(const int4* __restrict_
   }
 }
 
-// ---------------------------------------------------------------- 2a. subproblem solve
-// 64 x 64 product C = A^T B or A B (row pitch kEsLd) into acc: thread
-// (tx, ty) owns rows 4 ty + q and columns tx + 16 w, so a warp reads 16
-// consecutive doubles of a row of B (no bank conflicts) and broadcasts A
-template <bool kTransA>
-__device__ __forceinline__ void small_gemm(const double* A, const double* B, double (&acc)[4][4], int tx, int ty) {
+// ---------------------------------------------------------------- 2. tridiagonal reduction
+// Sum over a warp; lane 0 holds the result (a fixed butterfly order).
+__device__ __forceinline__ double warp_sum(double s) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// Sum over the CTA, the same value in every thread: warp sums, then the
+// warps' partials in warp order.  red holds kTdWarps doubles.
+__device__ __forceinline__ double td_block_sum(double s, double* red) {
+  s = warp_sum(s);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  double tot = 0.0;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) acc[q][w] = 0.0;
-#pragma unroll 4
-  for (int k = 0; k < kEs; ++k) {
-    double a[4], b[4];
+  for (int w = 0; w < kTdWarps; ++w) tot += red[w];
+  __syncthreads();
+  return tot;
+}
+
+// A[r][c] -= sum_k (V_k[r] W_k[c] + W_k[r] V_k[c]) over the lower 64 x 64
+// tiles of the trailing block [t0, m)^2, each written with its mirror.  The
+// k-sum of one element and of its mirror would round differently, so the
+// mirror is copied, not recomputed.
+__device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, const double* Vg, const double* Wg,
+                                   double* sm) {
+  double* Vr = sm;                         // [kTdNb][64]: V_k[r0 + rr]
+  double* Wr = Vr + kTdNb * kTdTile;
+  double* Vc = Wr + kTdNb * kTdTile;       // [kTdNb][64]: V_k[c0 + cc]
+  double* Wc = Vc + kTdNb * kTdTile;
+  double* Cs = Wc + kTdNb * kTdTile;       // [64][65] updated tile
+  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;  // rows ty, ty + 32; columns tx + 16 q
+  const int nt = (m - t0 + kTdTile - 1) / kTdTile;
+  for (int a = 0; a < nt; ++a) {
+    for (int b = 0; b <= a; ++b) {
+      const int r0 = t0 + a * kTdTile, c0 = t0 + b * kTdTile;
+      for (int e = t; e < kTdNb * kTdTile; e += kTdThreads) {
+        const int k = e >> 6, q = e & 63;
+        const bool kin = k < nbk;
+        Vr[e] = (kin && r0 + q < m) ? Vg[static_cast<size_t>(k) * ld + r0 + q] : 0.0;
+        Wr[e] = (kin && r0 + q < m) ? Wg[static_cast<size_t>(k) * ld + r0 + q] : 0.0;
+        Vc[e] = (kin && c0 + q < m) ? Vg[static_cast<size_t>(k) * ld + c0 + q] : 0.0;
+        Wc[e] = (kin && c0 + q < m) ? Wg[static_cast<size_t>(k) * ld + c0 + q] : 0.0;
+      }
+      __syncthreads();
+      double acc[2][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      a[q] = kTransA ? A[k * kEsLd + ty * 4 + q] : A[(ty * 4 + q) * kEsLd + k];
-      b[q] = B[k * kEsLd + tx + 16 * q];
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[u][q] = 0.0;
+      for (int k = 0; k < nbk; ++k) {
+        double vr[2], wr[2], vc[4], wc[4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          vr[u] = Vr[k * kTdTile + ty + 32 * u];
+          wr[u] = Wr[k * kTdTile + ty + 32 * u];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          vc[q] = Vc[k * kTdTile + tx + 16 * q];
+          wc[q] = Wc[k * kTdTile + tx + 16 * q];
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[u][q] = fma(vr[u], wc[q], fma(wr[u], vc[q], acc[u][q]));
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = r0 + ty + 32 * u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = c0 + tx + 16 * q;
+          double val = 0.0;
+          if (r < m && c < m) val = A[static_cast<size_t>(r) * ld + c] - acc[u][q];
+          Cs[(ty + 32 * u) * (kTdTile + 1) + tx + 16 * q] = val;
+        }
+      }
+      __syncthreads();
+      // write the tile's lower part (all of it off the diagonal) and the mirror
+      for (int e = t; e < kTdTile * kTdTile; e += kTdThreads) {
+        const int rr = e >> 6, cc = e & 63;
+        const int r = r0 + rr, c = c0 + cc;
+        if (r < m && c < m && (a != b || rr >= cc)) A[static_cast<size_t>(r) * ld + c] = Cs[rr * (kTdTile + 1) + cc];
+        // mirror: element (c0 + rr, r0 + cc) = tile element (cc, rr)
+        const int mr = c0 + rr, mc = r0 + cc;
+        if (mr < m && mc < m && (a != b || cc > rr)) A[static_cast<size_t>(mr) * ld + mc] = Cs[cc * (kTdTile + 1) + rr];
+      }
+      __syncthreads();
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) acc[q][w] = fma(a[q], b[w], acc[q][w]);
   }
 }
 
-// Cyclic Jacobi on S (64 x 64, symmetric) with the same tournament over its
-// 64 indices: 63 rounds of 32 disjoint rotations per sweep.  For a pair with
-// alpha = S_aa, beta = S_bb, gamma = S_ab the rotation J = [c s; -s c] zeroes
-// S_ab in J^T S J when t = s / c is the smaller root of t^2 + 2 tau t - 1 = 0,
-// tau = (beta - alpha) / (2 gamma) (the symmetric 2 x 2 Schur decomposition);
-// with d = beta - alpha that root is t = 2 gamma sgn(d) / (|d| + sqrt(d^2 + 4 gamma^2)).
-// A round applies its rotations to the rows of S, then to the columns of S
-// and V; each warp works on one pair and 32 consecutive rows or columns.
-__global__ void __launch_bounds__(kEThreads) jacobi_solve_kernel(const int2* __restrict__ pairs, int npairs,
-                                                                 const EntMat* __restrict__ mats, const double* __restrict__ G,
-                                                                 double* __restrict__ Vst, const EntCtl ctl, int round) {
-  extern __shared__ double smem_d[];
-  double* S = smem_d;
-  double* V = S + kEs * kEsLd;
-  __shared__ double rc[kEb], rs[kEb];
-  __shared__ int ra[kEb], rb[kEb];
-  if (*ctl.all_done) return;
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  for (int item = blockIdx.x; item < npairs; item += gridDim.x) {
-    const int2 pm = pairs[item];
-    const EntMat mi = mats[pm.x];
-    if (ctl.conv[pm.x] != kConvRunning || round >= mi.nb - 1) continue;
-    const int2 pq = tournament(mi.nb, round, pm.y);
-    const double* g = G + mi.off_g;
-    const size_t ld = static_cast<size_t>(kEb) * mi.nb;
-    __syncthreads();  // the previous item's V has been written out
-    for (int e = t; e < kEsElems; e += kEThreads) {
-      const int a = e >> 6, b = e & 63;
-      S[a * kEsLd + b] = g[sub_row(pq, a) * ld + sub_row(pq, b)];
-      V[a * kEsLd + b] = (a == b) ? 1.0 : 0.0;
-    }
-    __syncthreads();
-    for (int sweep = 0; sweep < kInnerSweeps; ++sweep) {
-      int rotated = 0;
-      for (int rr = 0; rr < kEs - 1; ++rr) {
-        int rot = 0;
-        if (t < kEb) {
-          const int2 ab = tournament(kEs, rr, t);
-          const double alpha = S[ab.x * kEsLd + ab.x], beta = S[ab.y * kEsLd + ab.y], gamma = S[ab.x * kEsLd + ab.y];
-          double c = 1.0, s = 0.0;
-          if (fabs(gamma) > kInnerTol * fmax(fabs(alpha), fabs(beta))) {
-            const double d = beta - alpha;
-            const double tt = (d >= 0.0 ? 2.0 * gamma : -2.0 * gamma) / (fabs(d) + sqrt(fma(d, d, 4.0 * gamma * gamma)));
-            c = rsqrt(fma(tt, tt, 1.0));
-            s = tt * c;
-            rot = 1;
+__global__ void __launch_bounds__(kTdThreads, 1)
+    tridiag_kernel(const EntMat* __restrict__ mats, double* __restrict__ G, double* __restrict__ VW,
+                   double* __restrict__ d_out, double* __restrict__ e_out, const EntCtl ctl) {
+  extern __shared__ double td_smem[];
+  const int p = blockIdx.x;
+  const EntMat mi = mats[p];
+  const int m = mi.m, ld = mi.mp;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  double* A = G + mi.off_g;
+  double* Vg = VW + mi.off_vw;  // V_k[r] = Vg[k ld + r]
+  double* Wg = Vg + static_cast<size_t>(kTdNb) * ld;
+  double* d = d_out + mi.sv_off;
+  double* e = e_out + mi.sv_off;
+  double* x = td_smem;          // column j, rows j .. m-1
+  double* v = x + ld;           // reflector, zero outside j+1 .. m-1 (and over the padding)
+  double* y = v + ld;           // G0 v, then w
+  double* vj = y + ld;          // V_k[j], W_k[j] for the panel's earlier reflectors
+  double* wj = vj + kTdNb;
+  double* pq = wj + kTdNb;      // [2 kTdNb]: V_k^T v, W_k^T v interleaved
+  double* red = pq + 2 * kTdNb; // [kTdWarps]
+
+  for (int k = 0; k < m - 1; k += kTdNb) {
+    const int nbk = min(kTdNb, m - 1 - k);
+    for (int i = 0; i < nbk; ++i) {
+      const int j = k + i;
+      if (t < i) {
+        vj[t] = Vg[static_cast<size_t>(t) * ld + j];
+        wj[t] = Wg[static_cast<size_t>(t) * ld + j];
+      }
+      __syncthreads();
+      // column j of the current matrix: row j of G0 minus the panel's terms
+      double s2 = 0.0;
+      for (int r = j + t; r < m; r += kTdThreads) {
+        double a = __ldcg(A + static_cast<size_t>(j) * ld + r);
+        for (int c = 0; c < i; ++c)
+          a -= fma(Vg[static_cast<size_t>(c) * ld + r], wj[c], Wg[static_cast<size_t>(c) * ld + r] * vj[c]);
+        x[r] = a;
+        if (r >= j + 2) s2 = fma(a, a, s2);
+      }
+      s2 = td_block_sum(s2, red);  // also orders the x writes before the reads below
+      const double alpha = x[j + 1];
+      double tau = 0.0, sc = 0.0, ej = alpha;
+      if (s2 != 0.0) {
+        const double beta = -copysign(sqrt(fma(alpha, alpha, s2)), alpha);
+        tau = (beta - alpha) / beta;
+        sc = 1.0 / (alpha - beta);
+        ej = beta;
+      }
+      if (t == 0) {
+        d[j] = x[j];
+        e[j] = ej;
+      }
+      // v over the whole padded range (zero outside j+1 .. m-1); V_i = v
+      for (int r = t; r < ld; r += kTdThreads) {
+        double val = 0.0;
+        if (tau != 0.0) {
+          if (r == j + 1) val = 1.0;
+          else if (r > j + 1 && r < m) val = x[r] * sc;
+        }
+        v[r] = val;
+        if (r > j && r < m) Vg[static_cast<size_t>(i) * ld + r] = val;
+      }
+      __syncthreads();
+      if (tau == 0.0) {  // the reflector is the identity (tau is the same in every thread)
+        for (int r = j + 1 + t; r < m; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = 0.0;
+        __syncthreads();
+        continue;
+      }
+      // y = G0 v over rows j+1 .. m-1: one warp per row pair, 16-byte loads
+      // from the 64-aligned column at or below j+1 to the padded end (v and
+      // the padding are zero there)
+      {
+        const int cs = (j + 1) & ~63;
+        const int nq = (ld - cs) >> 6;
+        const double2* vv = reinterpret_cast<const double2*>(v + cs) + lane;
+        for (int r = j + 1 + warp; r < m; r += 2 * kTdWarps) {
+          const int r2 = r + kTdWarps;
+          const bool two = r2 < m;
+          const double2* a1 = reinterpret_cast<const double2*>(A + static_cast<size_t>(r) * ld + cs) + lane;
+          const double2* a2 = reinterpret_cast<const double2*>(A + static_cast<size_t>(two ? r2 : r) * ld + cs) + lane;
+          double s1 = 0.0, s2r = 0.0;
+#pragma unroll 4
+          for (int q = 0; q < nq; ++q) {
+            const double2 b = vv[32 * q];
+            const double2 u1 = __ldcg(a1 + 32 * q);
+            const double2 u2 = __ldcg(a2 + 32 * q);
+            s1 = fma(u1.y, b.y, fma(u1.x, b.x, s1));
+            s2r = fma(u2.y, b.y, fma(u2.x, b.x, s2r));
           }
-          ra[t] = ab.x;
-          rb[t] = ab.y;
-          rc[t] = c;
-          rs[t] = s;
+          s1 = warp_sum(s1);
+          s2r = warp_sum(s2r);
+          if (lane == 0) {
+            y[r] = s1;
+            if (two) y[r2] = s2r;
+          }
         }
-        if (!__syncthreads_or(rot)) continue;  // nothing to rotate in this round
-        rotated = 1;
-        // rows: S <- J^T S (pair k, column j; a warp takes one pair, 32 columns)
-        for (int e = t; e < kEb * kEs; e += kEThreads) {
-          const int k = e >> 6, j = e & 63;
-          const double c = rc[k], s = rs[k];
-          if (s == 0.0) continue;
-          const int a = ra[k], b = rb[k];
-          const double sa = S[a * kEsLd + j], sb = S[b * kEsLd + j];
-          S[a * kEsLd + j] = c * sa - s * sb;
-          S[b * kEsLd + j] = s * sa + c * sb;
+        // V_k^T v and W_k^T v of the panel's earlier reflectors, one warp per dot
+        for (int dd = warp; dd < 2 * i; dd += kTdWarps) {
+          const double* src = ((dd & 1) ? Wg : Vg) + static_cast<size_t>(dd >> 1) * ld;
+          double s = 0.0;
+          for (int r = j + 1 + lane; r < m; r += 32) s = fma(src[r], v[r], s);
+          s = warp_sum(s);
+          if (lane == 0) pq[dd] = s;
         }
-        __syncthreads();
-        // columns: S <- S J and V <- V J (pair k, row i; a warp takes one pair, 32 rows)
-        for (int e = t; e < kEb * kEs; e += kEThreads) {
-          const int k = e >> 6, i = e & 63;
-          const double c = rc[k], s = rs[k];
-          if (s == 0.0) continue;
-          const int a = ra[k], b = rb[k];
-          const double sa = S[i * kEsLd + a], sb = S[i * kEsLd + b];
-          S[i * kEsLd + a] = c * sa - s * sb;
-          S[i * kEsLd + b] = s * sa + c * sb;
-          const double va = V[i * kEsLd + a], vb = V[i * kEsLd + b];
-          V[i * kEsLd + a] = c * va - s * vb;
-          V[i * kEsLd + b] = s * va + c * vb;
-        }
-        __syncthreads();
       }
-      if (!__syncthreads_or(rotated)) break;
-    }
-    // Hundreds of rotations leave V a few hundred ulps from orthogonal, and
-    // the update would scale G's eigenvalues by that much every round.  One
-    // Newton-Schulz step towards the polar factor, V <- V - V (V^T V - I) / 2,
-    // squares the error (down to rounding).  E = V^T V - I goes into S.
-    double acc[4][4];
-    small_gemm<true>(V, V, acc, tx, ty);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int w = 0; w < 4; ++w)
-        S[(ty * 4 + q) * kEsLd + tx + 16 * w] = acc[q][w] - ((ty * 4 + q == tx + 16 * w) ? 1.0 : 0.0);
-    __syncthreads();
-    small_gemm<false>(V, S, acc, tx, ty);
-    double* vout = Vst + mi.off_v + static_cast<size_t>(pm.y) * kEsElems;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = ty * 4 + q;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) vout[i * kEs + tx + 16 * w] = fma(-0.5, acc[q][w], V[i * kEsLd + tx + 16 * w]);
-    }
-  }
-}
-
-// ---------------------------------------------------------------- 2b. G <- J^T G J
-// Super-block (u, v), u <= v: T = G[rows of pair u][rows of pair v] (64 x 64)
-// becomes V_u^T T V_v, and its transpose is written to (v, u).
-// Shared memory holds T transposed (Tt), R = T V_v and one rotation block
-// (V_v, then V_u), each 64 rows of kUpdLd doubles (16-byte aligned rows).
-// Thread (tx, ty) owns rows 4 ty + q and columns 2 tx + {0, 1} + 32 {0, 1} of
-// each product, so every operand fetch is a double2: the A side is a
-// broadcast within a half-warp, the B side 256 contiguous bytes.
-constexpr int kUpdLd = kEs + 2;
-
-// acc[q][w] = sum_k A[k][4 ty + q] B[k][col(w)], A and B row-major with pitch kUpdLd
-__device__ __forceinline__ void gemm_tn(const double* A, const double* B, double (&acc)[4][4], int tx, int ty) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) acc[q][w] = 0.0;
-#pragma unroll 4
-  for (int k = 0; k < kEs; ++k) {
-    const double2 a01 = *reinterpret_cast<const double2*>(A + k * kUpdLd + ty * 4);
-    const double2 a23 = *reinterpret_cast<const double2*>(A + k * kUpdLd + ty * 4 + 2);
-    const double2 b01 = *reinterpret_cast<const double2*>(B + k * kUpdLd + tx * 2);
-    const double2 b23 = *reinterpret_cast<const double2*>(B + k * kUpdLd + tx * 2 + 32);
-    const double a[4] = {a01.x, a01.y, a23.x, a23.y};
-    const double b[4] = {b01.x, b01.y, b23.x, b23.y};
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) acc[q][w] = fma(a[q], b[w], acc[q][w]);
-  }
-}
-
-__device__ __forceinline__ int upd_col(int tx, int w) { return tx * 2 + (w & 1) + 32 * (w >> 1); }
-
-__global__ void __launch_bounds__(kEThreads) jacobi_update_kernel(const int4* __restrict__ sblk, int nsblk,
-                                                                  const EntMat* __restrict__ mats, double* __restrict__ G,
-                                                                  const double* __restrict__ Vst, const EntCtl ctl, int round) {
-  extern __shared__ __align__(16) double smem_d[];
-  double* Tt = smem_d;             // T transposed, then T' (row-major)
-  double* R = Tt + kEs * kUpdLd;   // T V_v
-  double* Vb = R + kEs * kUpdLd;   // V_v, then V_u
-  if (*ctl.all_done) return;
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  for (int item = blockIdx.x; item < nsblk; item += gridDim.x) {
-    const int4 sb = sblk[item];
-    const EntMat mi = mats[sb.x];
-    if (ctl.conv[sb.x] != kConvRunning || round >= mi.nb - 1) continue;
-    const int2 pu = tournament(mi.nb, round, sb.y), pv = tournament(mi.nb, round, sb.z);
-    double* g = G + mi.off_g;
-    const size_t ld = static_cast<size_t>(kEb) * mi.nb;
-    const double* vu = Vst + mi.off_v + static_cast<size_t>(sb.y) * kEsElems;
-    const double* vv = Vst + mi.off_v + static_cast<size_t>(sb.z) * kEsElems;
-    __syncthreads();  // the previous item's T' has been written out
-    for (int e = t; e < kEsElems; e += kEThreads) {
-      const int a = e >> 6, b = e & 63;
-      Tt[b * kUpdLd + a] = g[sub_row(pu, a) * ld + sub_row(pv, b)];
-      Vb[a * kUpdLd + b] = vv[e];
-    }
-    __syncthreads();
-    double acc[4][4];
-    gemm_tn(Tt, Vb, acc, tx, ty);  // R = T V_v
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) R[(ty * 4 + q) * kUpdLd + upd_col(tx, w)] = acc[q][w];
-    __syncthreads();
-    for (int e = t; e < kEsElems; e += kEThreads) Vb[(e >> 6) * kUpdLd + (e & 63)] = vu[e];
-    __syncthreads();
-    gemm_tn(Vb, R, acc, tx, ty);   // T' = V_u^T R
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) Tt[(ty * 4 + q) * kUpdLd + upd_col(tx, w)] = acc[q][w];
-    __syncthreads();
-    const bool diag = (sb.y == sb.z);
-    for (int e = t; e < kEsElems; e += kEThreads) {
-      const int a = e >> 6, b = e & 63;
-      if (diag) {
-        // keep G exactly symmetric: the lower half, mirrored
-        g[sub_row(pu, a) * ld + sub_row(pu, b)] = (a >= b) ? Tt[a * kUpdLd + b] : Tt[b * kUpdLd + a];
-      } else {
-        g[sub_row(pu, a) * ld + sub_row(pv, b)] = Tt[a * kUpdLd + b];
-        g[sub_row(pv, a) * ld + sub_row(pu, b)] = Tt[b * kUpdLd + a];
+      __syncthreads();
+      // y <- tau (y - V (W^T v) - W (V^T v)); then w = y - (tau/2)(v^T y) v
+      double sv = 0.0;
+      for (int r = j + 1 + t; r < m; r += kTdThreads) {
+        double yy = y[r];
+        for (int c = 0; c < i; ++c)
+          yy -= fma(Vg[static_cast<size_t>(c) * ld + r], pq[2 * c + 1], Wg[static_cast<size_t>(c) * ld + r] * pq[2 * c]);
+        yy *= tau;
+        y[r] = yy;
+        sv = fma(yy, v[r], sv);
       }
+      sv = td_block_sum(sv, red);
+      const double a2 = -0.5 * tau * sv;
+      for (int r = j + 1 + t; r < m; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = fma(a2, v[r], y[r]);
+      __syncthreads();
     }
+    td_trailing_update(A, ld, m, k + nbk, nbk, Vg, Wg, td_smem);
   }
-}
-
-// ---------------------------------------------------------------- 3. convergence
-// Per 32-row block: fp64 sums of the squared off-diagonal and diagonal entries.
-__global__ void __launch_bounds__(kEThreads) off_norm_kernel(const int2* __restrict__ rblk, const EntMat* __restrict__ mats,
-                                                             const double* __restrict__ G, double* __restrict__ part,
-                                                             const EntCtl ctl) {
-  __shared__ double red[2][kEThreads];
-  if (*ctl.all_done) return;
-  const int2 rm = rblk[blockIdx.x];
-  const EntMat mi = mats[rm.x];
-  if (ctl.conv[rm.x] != kConvRunning) return;
-  const int mp = kEb * mi.nb;
-  const double* g = G + mi.off_g + static_cast<size_t>(rm.y) * kEb * mp;
-  double off = 0.0, dia = 0.0;
-  for (int e = threadIdx.x; e < kEb * mp; e += kEThreads) {
-    const int r = e / mp, c = e - r * mp;
-    const double v = g[e];
-    if (c == rm.y * kEb + r) dia += v * v;
-    else off += v * v;
-  }
-  red[0][threadIdx.x] = off;
-  red[1][threadIdx.x] = dia;
-  __syncthreads();
-  for (int s = kEThreads / 2; s > 0; s >>= 1) {
-    if (threadIdx.x < s) {
-      red[0][threadIdx.x] += red[0][threadIdx.x + s];
-      red[1][threadIdx.x] += red[1][threadIdx.x + s];
-    }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    part[2 * blockIdx.x] = red[0][0];
-    part[2 * blockIdx.x + 1] = red[1][0];
-  }
-}
-
-__global__ void converge_kernel(const EntMat* __restrict__ mats, int n, const double* __restrict__ part,
-                                const EntCtl ctl, int sweep, int last) {
-  if (*ctl.all_done) return;
-  __shared__ int running;
-  if (threadIdx.x == 0) running = 0;
-  __syncthreads();
-  for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    if (ctl.conv[p] == kConvRunning) {
-      const EntMat& mi = mats[p];
-      double off = 0.0, dia = 0.0;
-      for (int k = 0; k < mi.nb; ++k) {
-        off += part[2 * (mi.rb_first + k)];
-        dia += part[2 * (mi.rb_first + k) + 1];
-      }
-      if (!isfinite(off) || !isfinite(dia)) {
-        ctl.conv[p] = kConvNonFinite;
-        atomicOr(ctl.status, kStatusNonFinite);
-      } else if (off <= kOffTol * kOffTol * (off + dia)) {
-        ctl.conv[p] = kConvDone;
-        ctl.sweeps[p] = sweep + 1;
-      } else if (last) {
-        atomicOr(ctl.status, kStatusNotConverged);
-      } else {
-        running = 1;
-      }
-    }
+  // the last diagonal element, then the finiteness check of T
+  if (t == 0) {
+    d[m - 1] = A[static_cast<size_t>(m - 1) * ld + m - 1];
   }
   __syncthreads();
-  if (threadIdx.x == 0 && (!running || last)) *ctl.all_done = 1;
+  int bad = 0;
+  for (int r = t; r < m; r += kTdThreads) {
+    if (!isfinite(d[r])) bad = 1;
+    if (r < m - 1 && !isfinite(e[r])) bad = 1;
+  }
+  bad = __syncthreads_or(bad);
+  if (t == 0) {
+    if (bad) {
+      ctl.conv[p] = kConvNonFinite;
+      ctl.sweeps[p] = 0;
+      atomicOr(ctl.status, kStatusNonFinite);
+    } else {
+      ctl.conv[p] = kConvDone;
+      ctl.sweeps[p] = 1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- 3. bisection
+// blocks: (matrix, first eigenvalue index) for every kBisThreads indices.
+// Eigenvalue k in ascending order (0-based) is the x where the count of
+// eigenvalues below x passes k; it is written at position m-1-k, so each
+// matrix's eigenvalues come out descending.
+__global__ void __launch_bounds__(kBisThreads) bisect_kernel(const int2* __restrict__ blocks,
+                                                             const EntMat* __restrict__ mats,
+                                                             const double* __restrict__ d_in,
+                                                             const double* __restrict__ e_in,
+                                                             double* __restrict__ lam, const EntCtl ctl) {
+  extern __shared__ double bis_smem[];
+  __shared__ double rlo[kBisThreads / 32], rhi[kBisThreads / 32], rem[kBisThreads / 32];
+  const int2 bk = blocks[blockIdx.x];
+  const EntMat mi = mats[bk.x];
+  if (ctl.conv[bk.x] == kConvNonFinite) return;  // the entropy pass writes NaN for it
+  const int m = mi.m, t = threadIdx.x;
+  double* dd = bis_smem;     // [m]
+  double* e2 = dd + m;       // [m - 1]: e_i^2
+  const double* d = d_in + mi.sv_off;
+  const double* e = e_in + mi.sv_off;
+  // Gershgorin interval of T and the largest e_i^2 (min / max are exact, so
+  // the reduction order does not matter)
+  double lo = INFINITY, hi = -INFINITY, emax = 0.0;
+  for (int i = t; i < m; i += kBisThreads) {
+    const double di = d[i];
+    const double el = i > 0 ? fabs(e[i - 1]) : 0.0;
+    const double er = i < m - 1 ? fabs(e[i]) : 0.0;
+    dd[i] = di;
+    if (i < m - 1) e2[i] = er * er;
+    lo = fmin(lo, di - el - er);
+    hi = fmax(hi, di + el + er);
+    emax = fmax(emax, er * er);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    emax = fmax(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  }
+  if ((t & 31) == 0) {
+    rlo[t >> 5] = lo;
+    rhi[t >> 5] = hi;
+    rem[t >> 5] = emax;
+  }
+  __syncthreads();
+  lo = rlo[0];
+  hi = rhi[0];
+  emax = rem[0];
+  for (int w = 1; w < kBisThreads / 32; ++w) {
+    lo = fmin(lo, rlo[w]);
+    hi = fmax(hi, rhi[w]);
+    emax = fmax(emax, rem[w]);
+  }
+  const int k = bk.y + t;
+  if (k >= m) return;  // no barrier follows
+  const double tnorm = fmax(fabs(lo), fabs(hi));
+  const double pivmin = DBL_MIN * fmax(1.0, emax);
+  // widen the interval by the rounding of the counts themselves
+  const double slack = 2.1 * tnorm * DBL_EPSILON * m + 4.2 * pivmin;
+  lo -= slack;
+  hi += slack;
+  const double tol = 2.0 * DBL_EPSILON * tnorm;
+  for (int it = 0; it < kBisMaxIter && hi - lo > tol; ++it) {
+    const double x = 0.5 * (lo + hi);
+    int cnt = 0;
+    double q = dd[0] - x;
+    if (fabs(q) < pivmin) q = -pivmin;
+    cnt += q < 0.0 ? 1 : 0;
+    for (int i = 1; i < m; ++i) {
+      q = (dd[i] - x) - e2[i - 1] / q;
+      if (fabs(q) < pivmin) q = -pivmin;
+      cnt += q < 0.0 ? 1 : 0;
+    }
+    if (cnt > k) hi = x;
+    else lo = x;
+  }
+  lam[mi.sv_off + (m - 1 - k)] = 0.5 * (lo + hi);
 }
 
 // ---------------------------------------------------------------- 4. entropy
-__global__ void __launch_bounds__(kSortThreads) entropy_kernel(const EntMat* __restrict__ mats, const double* __restrict__ G,
+__global__ void __launch_bounds__(kSortThreads) entropy_kernel(const EntMat* __restrict__ mats, const double* __restrict__ lam_in,
                                                                float* __restrict__ H_out, float* __restrict__ sigma_out,
                                                                const EntCtl ctl) {
   __shared__ float sv[kMaxDim];
   __shared__ double red[kSortThreads];
   const int p = blockIdx.x, t = threadIdx.x;
   const EntMat mi = mats[p];
-  const double* g = G + mi.off_g;
-  const size_t ld = static_cast<size_t>(kEb) * mi.nb;
+  const double* lam_p = lam_in + mi.sv_off;
   const bool finite = ctl.conv[p] != kConvNonFinite;
-  // sigma_i^2 = G_ii, clamped at 0 (G is positive semi-definite)
+  // sigma_i^2, clamped at 0 (G is positive semi-definite)
   auto lam = [&](int i) {
-    const double v = g[i * ld + i];
+    const double v = lam_p[i];
     return v > 0.0 ? v : 0.0;
   };
   double s_local = 0.0;
-  for (int i = t; i < mi.m; i += kSortThreads) s_local += lam(i);
+  if (finite)
+    for (int i = t; i < mi.m; i += kSortThreads) s_local += lam(i);
   red[t] = s_local;
   __syncthreads();
   for (int s = kSortThreads / 2; s > 0; s >>= 1) {
@@ -496,7 +520,7 @@ __global__ void __launch_bounds__(kSortThreads) entropy_kernel(const EntMat* __r
   const double total = red[0];
   __syncthreads();
   double h_local = 0.0;
-  if (total > 0.0) {
+  if (finite && total > 0.0) {
     for (int i = t; i < mi.m; i += kSortThreads) {
       const double q = lam(i) / total;
       if (q > 0.0) h_local += q * log(q);
@@ -548,20 +572,19 @@ using namespace muon;
 struct muon_entropy_plan_s {
   int device = 0;
   int n = 0;
-  int nb_max = 2;
-  int ntiles = 0, npairs = 0, nsblk = 0, nrb = 0;
-  int grid_solve = 1, grid_update = 1;
+  int ntiles = 0, nbis = 0;
+  int mp_max = 64, m_max = 1;
   int64_t total_sv = 0;
   std::vector<EntMat> mats;
   char* dmem = nullptr;
   double* G = nullptr;
-  double* V = nullptr;
+  double* VW = nullptr;
+  double* dvec = nullptr;
+  double* evec = nullptr;
+  double* lam = nullptr;
   EntMat* mats_d = nullptr;
   int4* tiles_d = nullptr;
-  int2* pairs_d = nullptr;
-  int4* sblk_d = nullptr;
-  int2* rb_d = nullptr;
-  double* part_d = nullptr;
+  int2* bis_d = nullptr;
   const float** wptr_d = nullptr;
   EntCtl ctl{};
   const float** pinned = nullptr;
@@ -569,7 +592,7 @@ struct muon_entropy_plan_s {
   bool cache_valid = false;
   bool ev_pending = false;
   cudaEvent_t ev = nullptr;
-  cudaEvent_t prof[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaEvent_t prof[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
   bool profiling = false;
   bool prof_recorded = false;
   cudaStream_t last_stream = nullptr;
@@ -610,9 +633,9 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
   pl->device = dev;
   pl->n = n;
   pl->mats.resize(n);
-  std::vector<int4> tiles, sblk;
-  std::vector<int2> pairs, rbs;
-  int64_t off_g = 0, off_v = 0, sv = 0;
+  std::vector<int4> tiles;
+  std::vector<int2> bis;
+  int64_t off_g = 0, off_vw = 0, sv = 0;
   for (int i = 0; i < n; ++i) {
     EntMat& mi = pl->mats[i];
     mi.rows = static_cast<int>(shapes[2 * i]);
@@ -620,35 +643,23 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
     mi.m = std::min(mi.rows, mi.cols);
     mi.n = std::max(mi.rows, mi.cols);
     mi.tall = mi.rows > mi.cols ? 1 : 0;
-    int nb = (mi.m + kEb - 1) / kEb;
-    nb += nb & 1;
-    mi.nb = nb;
-    mi.rb_first = static_cast<int>(rbs.size());
-    mi.pad_ = 0;
+    mi.mp = (mi.m + kGramTile - 1) / kGramTile * kGramTile;
     mi.off_g = off_g;
-    mi.off_v = off_v;
+    mi.off_vw = off_vw;
     mi.sv_off = sv;
-    const int mp = kEb * nb;
-    off_g += static_cast<int64_t>(align256(static_cast<size_t>(mp) * mp * sizeof(double)) / sizeof(double));
-    off_v += static_cast<int64_t>(nb / 2) * kEsElems;
+    off_g += static_cast<int64_t>(align256(static_cast<size_t>(mi.mp) * mi.mp * sizeof(double)) / sizeof(double));
+    off_vw += static_cast<int64_t>(2) * kTdNb * mi.mp;
     sv += mi.m;
-    pl->nb_max = std::max(pl->nb_max, nb);
-    const int nt = mp / kGramTile;
+    pl->mp_max = std::max(pl->mp_max, mi.mp);
+    pl->m_max = std::max(pl->m_max, mi.m);
+    const int nt = mi.mp / kGramTile;
     for (int a = 0; a < nt; ++a)
       for (int b = 0; b <= a; ++b) tiles.push_back(make_int4(i, a, b, 0));
-    for (int u = 0; u < nb / 2; ++u) pairs.push_back(make_int2(i, u));
-    for (int u = 0; u < nb / 2; ++u)
-      for (int v = u; v < nb / 2; ++v) sblk.push_back(make_int4(i, u, v, 0));
-    for (int k = 0; k < nb; ++k) rbs.push_back(make_int2(i, k));
+    for (int k = 0; k < mi.m; k += kBisThreads) bis.push_back(make_int2(i, k));
   }
   pl->ntiles = static_cast<int>(tiles.size());
-  pl->npairs = static_cast<int>(pairs.size());
-  pl->nsblk = static_cast<int>(sblk.size());
-  pl->nrb = static_cast<int>(rbs.size());
+  pl->nbis = static_cast<int>(bis.size());
   pl->total_sv = sv;
-  const int sms = prop.multiProcessorCount;
-  pl->grid_solve = std::max(1, std::min(pl->npairs, sms * 3));
-  pl->grid_update = std::max(1, std::min(pl->nsblk, sms * 2));
 
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -657,17 +668,16 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
     return o;
   };
   const size_t o_g = take(static_cast<size_t>(off_g) * sizeof(double));
-  const size_t o_v = take(static_cast<size_t>(off_v) * sizeof(double));
+  const size_t o_vw = take(static_cast<size_t>(off_vw) * sizeof(double));
+  const size_t o_d = take(static_cast<size_t>(sv) * sizeof(double));
+  const size_t o_e = take(static_cast<size_t>(sv) * sizeof(double));
+  const size_t o_l = take(static_cast<size_t>(sv) * sizeof(double));
   const size_t o_m = take(n * sizeof(EntMat));
   const size_t o_t = take(tiles.size() * sizeof(int4));
-  const size_t o_p = take(pairs.size() * sizeof(int2));
-  const size_t o_s = take(sblk.size() * sizeof(int4));
-  const size_t o_r = take(rbs.size() * sizeof(int2));
-  const size_t o_part = take(rbs.size() * 2 * sizeof(double));
+  const size_t o_b = take(bis.size() * sizeof(int2));
   const size_t o_w = take(n * sizeof(float*));
   const size_t o_conv = take(n * sizeof(int));
   const size_t o_sw = take(n * sizeof(int));
-  const size_t o_ad = take(sizeof(int));
   const size_t o_st = take(sizeof(unsigned));
   if (cudaMalloc(&pl->dmem, off) != cudaSuccess) {
     cudaGetLastError();
@@ -676,34 +686,31 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
   }
   char* b = pl->dmem;
   pl->G = reinterpret_cast<double*>(b + o_g);
-  pl->V = reinterpret_cast<double*>(b + o_v);
+  pl->VW = reinterpret_cast<double*>(b + o_vw);
+  pl->dvec = reinterpret_cast<double*>(b + o_d);
+  pl->evec = reinterpret_cast<double*>(b + o_e);
+  pl->lam = reinterpret_cast<double*>(b + o_l);
   pl->mats_d = reinterpret_cast<EntMat*>(b + o_m);
   pl->tiles_d = reinterpret_cast<int4*>(b + o_t);
-  pl->pairs_d = reinterpret_cast<int2*>(b + o_p);
-  pl->sblk_d = reinterpret_cast<int4*>(b + o_s);
-  pl->rb_d = reinterpret_cast<int2*>(b + o_r);
-  pl->part_d = reinterpret_cast<double*>(b + o_part);
+  pl->bis_d = reinterpret_cast<int2*>(b + o_b);
   pl->wptr_d = reinterpret_cast<const float**>(b + o_w);
   pl->ctl.conv = reinterpret_cast<int*>(b + o_conv);
   pl->ctl.sweeps = reinterpret_cast<int*>(b + o_sw);
-  pl->ctl.all_done = reinterpret_cast<int*>(b + o_ad);
   pl->ctl.status = reinterpret_cast<unsigned*>(b + o_st);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   bool ok = cudaMemcpy(pl->mats_d, pl->mats.data(), n * sizeof(EntMat), cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(pl->tiles_d, tiles.data(), tiles.size() * sizeof(int4), cudaMemcpyHostToDevice) == cudaSuccess &&
-            cudaMemcpy(pl->pairs_d, pairs.data(), pairs.size() * sizeof(int2), cudaMemcpyHostToDevice) == cudaSuccess &&
-            cudaMemcpy(pl->sblk_d, sblk.data(), sblk.size() * sizeof(int4), cudaMemcpyHostToDevice) == cudaSuccess &&
-            cudaMemcpy(pl->rb_d, rbs.data(), rbs.size() * sizeof(int2), cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemcpy(pl->bis_d, bis.data(), bis.size() * sizeof(int2), cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(pl->ctl.status, 0, sizeof(unsigned)) == cudaSuccess &&
             cudaMemset(pl->ctl.sweeps, 0, n * sizeof(int)) == cudaSuccess;
   ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&pl->pinned), n * sizeof(float*), cudaHostAllocDefault) ==
                  cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&pl->ev, cudaEventDisableTiming) == cudaSuccess;
-  for (int k = 0; k < 4 && ok; ++k) ok = cudaEventCreate(&pl->prof[k]) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(jacobi_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(kSolveSmem)) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(jacobi_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(kUpdSmem)) == cudaSuccess;
+  for (int k = 0; k < 5 && ok; ++k) ok = cudaEventCreate(&pl->prof[k]) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(tridiag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tridiag_smem_bytes(pl->mp_max))) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bisect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(2 * pl->m_max * sizeof(double))) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_entropy(pl);
@@ -764,24 +771,20 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
   }
   const EntCtl ctl = pl->ctl;
   bool ok = cudaMemsetAsync(ctl.conv, 0, n * sizeof(int), st) == cudaSuccess &&
-            cudaMemsetAsync(ctl.sweeps, 0, n * sizeof(int), st) == cudaSuccess &&
-            cudaMemsetAsync(ctl.all_done, 0, sizeof(int), st) == cudaSuccess;
+            cudaMemsetAsync(ctl.sweeps, 0, n * sizeof(int), st) == cudaSuccess;
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[0], st) == cudaSuccess;
   if (ok) gram_kernel<<<pl->ntiles, kEThreads, 0, st>>>(pl->tiles_d, pl->mats_d, pl->wptr_d, pl->G);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[1], st) == cudaSuccess;
-  for (int sweep = 0; ok && sweep < kMaxSweeps; ++sweep) {
-    for (int r = 0; r < pl->nb_max - 1; ++r) {
-      jacobi_solve_kernel<<<pl->grid_solve, kEThreads, kSolveSmem, st>>>(pl->pairs_d, pl->npairs, pl->mats_d, pl->G,
-                                                                         pl->V, ctl, r);
-      jacobi_update_kernel<<<pl->grid_update, kEThreads, kUpdSmem, st>>>(pl->sblk_d, pl->nsblk, pl->mats_d, pl->G,
-                                                                         pl->V, ctl, r);
-    }
-    off_norm_kernel<<<pl->nrb, kEThreads, 0, st>>>(pl->rb_d, pl->mats_d, pl->G, pl->part_d, ctl);
-    converge_kernel<<<1, 1024, 0, st>>>(pl->mats_d, n, pl->part_d, ctl, sweep, sweep == kMaxSweeps - 1 ? 1 : 0);
-  }
+  if (ok)
+    tridiag_kernel<<<n, kTdThreads, tridiag_smem_bytes(pl->mp_max), st>>>(pl->mats_d, pl->G, pl->VW, pl->dvec,
+                                                                         pl->evec, ctl);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[2], st) == cudaSuccess;
-  if (ok) entropy_kernel<<<n, kSortThreads, 0, st>>>(pl->mats_d, pl->G, H_out, sigma_out, ctl);
+  if (ok)
+    bisect_kernel<<<pl->nbis, kBisThreads, 2 * pl->m_max * sizeof(double), st>>>(pl->bis_d, pl->mats_d, pl->dvec,
+                                                                                 pl->evec, pl->lam, ctl);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[3], st) == cudaSuccess;
+  if (ok) entropy_kernel<<<n, kSortThreads, 0, st>>>(pl->mats_d, pl->lam, H_out, sigma_out, ctl);
+  if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[4], st) == cudaSuccess;
   if (!ok || cudaGetLastError() != cudaSuccess) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
@@ -806,7 +809,6 @@ extern "C" muon_status_t muon_entropy_get_status(muon_entropy_plan_t pl, int32_t
     return MUON_ERR_CUDA;
   }
   if (s & kStatusNonFinite) return MUON_ERR_NONFINITE;
-  if (s & kStatusNotConverged) return MUON_ERR_NOT_CONVERGED;
   return MUON_OK;
 }
 
@@ -814,11 +816,11 @@ extern "C" muon_status_t muon_entropy_profile(muon_entropy_plan_t pl, int32_t en
   if (pl == nullptr) return MUON_ERR_INVALID_ARG;
   if (ms_out != nullptr) {
     if (!pl->prof_recorded) return MUON_ERR_INVALID_ARG;
-    if (cudaEventSynchronize(pl->prof[3]) != cudaSuccess) {
+    if (cudaEventSynchronize(pl->prof[4]) != cudaSuccess) {
       cudaGetLastError();
       return MUON_ERR_CUDA;
     }
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < 4; ++k) {
       float ms = 0.0f;
       if (cudaEventElapsedTime(&ms, pl->prof[k], pl->prof[k + 1]) != cudaSuccess) {
         cudaGetLastError();

@@ -582,6 +582,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   unsigned* status = g.ws.status;
+  // everything above touched only shared memory, TMEM and the kernel
+  // parameters: with programmatic dependent launch it overlaps the previous
+  // kernel's last CTAs; nothing below runs before that kernel has completed
+  pdl_wait();
+  pdl_trigger();
 
   if (g.test_wait_ns != 0) {
     // Failure-detection test (the same value in every CTA of the grid): one
@@ -1038,8 +1043,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& args, int npairs, cudaStream_t st) {
   if (!configure_device()) return cudaErrorInvalidDeviceFunction;
   npairs = npairs < args.ntiles ? npairs : args.ntiles;
   if (npairs < 1) npairs = 1;
-  ns_gemm_kernel<<<2 * npairs, kThreads, kSmemBytes, st>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(kPdlGemm, ns_gemm_kernel, dim3(2 * npairs), dim3(kThreads), kSmemBytes, st, args);
 }
 
 }  // namespace muon

@@ -32,6 +32,7 @@ namespace {
 constexpr int kMaxDim = 65536;
 constexpr int kMaxNsSteps = 32;
 constexpr int kEventPool = 4096;
+constexpr int kProfNs = 5;  // the Newton-Schulz phase of the profile (phases 1-3 together)
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -99,6 +100,16 @@ bool encode_f32_parts(CUtensorMap* tm, void* base, int rows, int cols, int ld, l
 
 }  // namespace
 
+bool muon::pdl_enabled(unsigned cls) {
+  static const unsigned mask = [] {
+    const char* env = std::getenv("MUON_PDL");
+    // default: the tensor-core launches only (on the elementwise passes the
+    // attribute measured no faster on small plans and slower on large ones)
+    return env != nullptr ? static_cast<unsigned>(std::atoi(env)) : static_cast<unsigned>(kPdlGemm);
+  }();
+  return (mask & cls) != 0;
+}
+
 // Operand maps (64 x 128 and 64 x 64 boxes) and epilogue store maps (32 x 32,
 // hi and lo together) of one matrix's workspace arrays, in MapIndex order.
 // lo must lie after hi0 and hi1 in memory.  Without split-K parts the part
@@ -127,10 +138,13 @@ bool muon::encode_matrix_maps(void* maps, const MatInfo& mi, __nv_bfloat16* hi0,
 
 namespace {
 
+// The events of one profiled call: segment k lies between events
+// first_event + k and first_event + k + 1 and its time goes to phase seg[k];
+// launches[] counts the call's launches per phase.
 struct ProfRec {
   int first_event = 0;
-  int nlaunch = 0;
-  std::vector<int> phases;
+  std::vector<int> seg;
+  int64_t launches[MUON_NUM_PHASES] = {};
 };
 
 // One wave of a plan: the matrices whose Newton-Schulz workspace is resident
@@ -194,8 +208,8 @@ struct muon_plan_s {
   MatPtrs* ptrs_d = nullptr;    // the table of the current call
   uint64_t use_clock = 0;
   cudaStream_t last_stream = nullptr;
-  // profiling
-  bool prof = false;
+  // profiling (0 off, MUON_PROFILE_LAUNCHES or MUON_PROFILE_SPANS)
+  int prof = 0;
   std::vector<cudaEvent_t> events;
   int ev_next = 0;
   std::vector<ProfRec> recs;
@@ -243,41 +257,58 @@ muon_status_t upload_ptrs(muon_plan_s* pl, const std::vector<MatPtrs>& t, cudaSt
 // ------------------------------------------------------------ profiling
 void prof_flush(muon_plan_s* pl) {
   for (const ProfRec& r : pl->recs) {
-    cudaEventSynchronize(pl->events[r.first_event + r.nlaunch]);
-    for (int k = 0; k < r.nlaunch; ++k) {
+    const int nseg = static_cast<int>(r.seg.size());
+    cudaEventSynchronize(pl->events[r.first_event + nseg]);
+    for (int k = 0; k < nseg; ++k) {
       float ms = 0.0f;
       cudaEventElapsedTime(&ms, pl->events[r.first_event + k], pl->events[r.first_event + k + 1]);
-      pl->prof_ms[r.phases[k]] += ms;
-      pl->prof_launches[r.phases[k]] += 1;
+      pl->prof_ms[r.seg[k]] += ms;
+      if (r.seg[k] >= kPhaseGram + 1 && r.seg[k] <= kPhaseUpdate + 1) pl->prof_ms[kProfNs] += ms;
     }
+    for (int p = 0; p < MUON_NUM_PHASES; ++p) pl->prof_launches[p] += r.launches[p];
     pl->prof_calls += 1;
   }
   pl->recs.clear();
   pl->ev_next = 0;
 }
 
+// Records a call's events.  mark(phase) follows every launch; in span mode a
+// product launch records no event, and span_end() closes the products of a
+// wave with one event whose segment goes to the Newton-Schulz phase.
 struct Recorder {
   muon_plan_s* pl;
   cudaStream_t st;
   ProfRec rec{};
   bool on = false;
+  bool spans = false;
+  int open = 0;  // launches since the last event
   Recorder(muon_plan_s* p, cudaStream_t s, int max_launches) : pl(p), st(s) {
-    if (!pl->prof) return;
+    if (pl->prof == 0) return;
+    spans = pl->prof == MUON_PROFILE_SPANS;
     if (max_launches + 1 > static_cast<int>(pl->events.size())) pl->events.resize(max_launches + 1, nullptr);
     for (auto& ev : pl->events)
       if (ev == nullptr && cudaEventCreate(&ev) != cudaSuccess) return;
     if (pl->ev_next + max_launches + 1 > static_cast<int>(pl->events.size())) prof_flush(pl);
     rec.first_event = pl->ev_next;
-    rec.nlaunch = 0;
-    rec.phases.reserve(max_launches);
+    rec.seg.reserve(max_launches);
     cudaEventRecord(pl->events[pl->ev_next++], st);
     on = true;
   }
+  void close(int phase) {
+    rec.seg.push_back(phase);
+    open = 0;
+    cudaEventRecord(pl->events[pl->ev_next++], st);
+  }
   void mark(int phase) {
     if (!on) return;
-    rec.phases.push_back(phase);
-    rec.nlaunch++;
-    cudaEventRecord(pl->events[pl->ev_next++], st);
+    rec.launches[phase] += 1;
+    if (phase >= kPhaseGram + 1 && phase <= kPhaseUpdate + 1) rec.launches[kProfNs] += 1;
+    ++open;
+    if (spans && phase >= kPhaseGram + 1 && phase <= kPhaseUpdate + 1) return;
+    close(phase);
+  }
+  void span_end() {
+    if (on && spans && open > 0) close(kProfNs);
   }
   ~Recorder() {
     if (on) pl->recs.push_back(rec);
@@ -345,6 +376,7 @@ muon_status_t run_ns(muon_plan_s* pl, const StepScalars& sc, int ns_steps, int p
       }
       cur ^= 1;  // the X update wrote the other buffer
     }
+    rec.span_end();
     if (norm_pass) {
       e = launch_update_norm(chunks, w.nchunks, pl->mats_d, pl->ws, sc, fp32, cur, mul_s, update_rms, st);
       if (e != cudaSuccess) return MUON_ERR_CUDA;
@@ -942,13 +974,13 @@ void muon_destroy(muon_plan_t pl) {
 }
 
 muon_status_t muon_profile_enable(muon_plan_t pl, int32_t enable) {
-  if (pl == nullptr) return MUON_ERR_INVALID_ARG;
+  if (pl == nullptr || enable < 0 || enable > MUON_PROFILE_SPANS) return MUON_ERR_INVALID_ARG;
   if (enable && pl->events.empty()) {
     pl->events.resize(kEventPool);
     for (auto& ev : pl->events)
       if (cudaEventCreate(&ev) != cudaSuccess) return MUON_ERR_CUDA;
   }
-  pl->prof = enable != 0;
+  pl->prof = enable;
   return MUON_OK;
 }
 

@@ -294,4 +294,36 @@ int gemm_tc_max_pairs();
 cudaError_t launch_gemm_f32(const Gemm32Args& args, cudaStream_t st);
 int gemm_tc_smem_bytes();
 
+// Programmatic dependent launch.  The step's kernels run back to back on one
+// stream and each reads what the previous one wrote.  Launched with
+// programmatic stream serialization, a kernel's CTAs may start (and run their
+// set-up: barriers, TMEM allocation) while the previous kernel's last CTAs
+// still run; every such kernel executes pdl_wait() before its first global
+// memory access, which returns once the previous grid has completed and its
+// writes are visible, and then pdl_trigger(), which lets the next kernel's
+// CTAs be scheduled as SMs free up.  Both are no-ops for a kernel launched
+// without the attribute.  The kernels are in two classes (the tensor-core
+// products and the elementwise passes); MUON_PDL in the environment, read
+// once per process, is a mask of the classes launched with the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+enum PdlClass : unsigned { kPdlGemm = 1u, kPdlElementwise = 2u };
+bool pdl_enabled(unsigned cls);
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(unsigned cls, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled(cls) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace muon

@@ -75,6 +75,11 @@ def test_binding_layouts_and_enums_match_the_header():
     for name in ("MUON_SCALE_MAX_DIM", "MUON_SCALE_HIDDEN", "MUON_SCALE_UPDATE_NORM", "MUON_NS_BF16", "MUON_NS_FP32"):
         m = re.search(name + r"\s*=\s*(\d+)", hdr)
         assert m and int(m.group(1)) == getattr(L, name), name
+    for name in ("MUON_NUM_PHASES", "MUON_PROFILE_LAUNCHES", "MUON_PROFILE_SPANS", "MUON_INIT_ZERO_MOMENTUM",
+                 "MUON_INIT_FP32_NS", "MUON_INIT_MAX_WORKSPACE"):
+        m = re.search(r"#define\s+" + name + r"\s+(0x[0-9a-fA-F]+|\d+)", hdr)
+        assert m and int(m.group(1), 0) == getattr(L, name), name
+    assert len(L.PHASE_NAMES) == L.MUON_NUM_PHASES
 
 
 def test_init_rejects_bad_arguments_before_any_cuda_call(lib):

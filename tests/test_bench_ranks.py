@@ -86,11 +86,10 @@ def test_reference_arm_line_on_rank_zero(monkeypatch):
     assert "workload" in line["config"]
 
 
-def test_entropy_update_flop_count():
-    # (64, 64): nb = 2 blocks, one round of one super-block per sweep, two 64^3 products
-    assert bench.entropy_update_flops([(64, 64)], [3]) == 3 * 4 * 64 ** 3
-    # min(1408, 2048) = 1408: 44 blocks, 43 rounds of 22 * 23 / 2 super-blocks
-    assert bench.entropy_update_flops([(2048, 1408)], [1]) == 43 * 253 * 4 * 64 ** 3
-    # 33 rows round up to 2 blocks; a matrix that took no sweep adds nothing
-    assert bench.entropy_update_flops([(33, 70), (500, 9)], [2, 0]) == 2 * 4 * 64 ** 3
-    assert abs(bench.FP64_PEAK_TFLOPS - 37.23) < 0.01
+def test_entropy_trailing_byte_count():
+    # brute force: the trailing block of column j is (m-1-j) x (m-1-j) doubles
+    for shape in [(1, 5), (2, 2), (7, 3), (64, 64), (2048, 1408)]:
+        m = min(shape)
+        want = sum(8 * (m - 1 - j) ** 2 for j in range(m - 1))
+        assert bench.entropy_trailing_bytes([shape]) == want
+    assert bench.entropy_trailing_bytes([(3, 4), (5, 2)]) == 8 * (4 + 1) + 8 * 1

@@ -135,7 +135,20 @@ def test_workspace_and_profile_accounting():
     assert prof["calls"] == 1
     assert prof["launches"]["gram"] == 5 and prof["launches"]["poly"] == 5 and prof["launches"]["x_update"] == 5
     assert prof["launches"]["momentum_normalise"] == 1
+    assert prof["launches"]["newton_schulz"] == 15
     assert all(v >= 0 for v in prof["ms"].values())
+    ns = sum(prof["ms"][k] for k in ("gram", "poly", "x_update"))
+    assert prof["ms"]["newton_schulz"] == pytest.approx(ns, rel=1e-9)
+    # span mode: the product launches of the call are one span
+    plan.profile(True, spans=True)
+    plan.step(list(zip(Ws, Gs, Ms)), lr=LR, weight_decay=WD, momentum=MU, coeffs=ABC32)
+    prof = plan.profile_read()
+    assert prof["calls"] == 1
+    assert prof["launches"]["gram"] == 5 and prof["launches"]["newton_schulz"] == 15
+    assert prof["ms"]["gram"] == prof["ms"]["poly"] == prof["ms"]["x_update"] == 0.0
+    assert prof["ms"]["newton_schulz"] > 0 and prof["ms"]["momentum_normalise"] > 0 and prof["ms"]["finalize"] > 0
+    with pytest.raises(L.MuonError):
+        L.muon_profile_enable(plan._plan, 3)
 
 
 def test_rotating_buffer_sets_use_their_own_pointers():

@@ -4,20 +4,18 @@ the fp64 oracle.
 Bounds, from the arithmetic:
 - The Gram matrix is fp64; products of fp32 entries are exact, and the sums
   of n <= 2048 terms are good to about 1e-13 of the largest eigenvalue.
-- The block Jacobi (fp64) stops at an off-diagonal norm of 1e-6 of
-  ||G||_F, which moves an eigenvalue by second-order amounts (below 1e-8 of
-  the largest in fp64 simulations of the same solver); skipped inner
-  rotations are below 1e-13 of the larger diagonal entry; each round
-  re-orthonormalises its rotations.
+- The Householder reduction to tridiagonal form (fp64) is backward stable:
+  T has the eigenvalues of a matrix within a small multiple of m eps ||G||
+  of G, about 1e-12 of the largest eigenvalue for m = 1408; bisection on
+  the Sturm counts stops at a width of 2 eps ||T||.
 - The outputs are fp32: H (|H| <= 1) is rounded to 6e-8 and each singular
   value to 6e-8 relative, so sigma^2 to 1.2e-7 relative.
 So H is checked to 2e-7 absolute and sigma^2 to 3e-7 sigma_max^2 per value.
-That sigma^2 bound is relative to the largest eigenvalue only: the 1e-6 stop
-allows an absolute error of a few 1e-9 sigma_max^2 on every eigenvalue, so on
-a spectrum spanning three decades of sigma (six of sigma^2) the smallest
-sigma^2 may be off by about 1e-3 of itself.  H is insensitive to that (those
-values carry almost no energy); a user who needs the small singular values
-to a relative accuracy would need a tighter stop.
+That sigma^2 bound is relative to the largest eigenvalue only: every
+eigenvalue carries an absolute error of about 1e-12 sigma_max^2 from the
+reduction, so a sigma^2 six decades below the largest is good to about 1e-6
+of itself, not to the fp32 rounding.  H, which weighs those values by their
+tiny energy share, is unaffected at its 2e-7 bound.
 """
 
 import math
@@ -171,4 +169,4 @@ def test_profile_phases():
     plan.profile(True)
     plan.compute(ws)
     ms = plan.profile_read()
-    assert set(ms) == {"gram", "jacobi", "entropy"} and all(v > 0 for v in ms.values())
+    assert set(ms) == {"gram", "tridiagonal", "bisection", "entropy"} and all(v > 0 for v in ms.values())
