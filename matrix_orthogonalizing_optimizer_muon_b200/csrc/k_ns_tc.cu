@@ -904,61 +904,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           continue;
         }
-        float val[32];
-        if (g.phase == kPhaseGram) {
-          const bool first = (g.iter == 0);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
-        } else if (poly) {
-          // B' = b A + c A A + a I (the a X term of the update rides on B' hi)
-#pragma unroll
-          for (int q = 0; q < 32; ++q)
-            val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q)) + (j0 + q == i ? a_c : 0.0f);
-        } else {
-          // X' = alpha (B' hi + a lo) = alpha (a X + B hi)
+        if (upd) {
+          // X' = alpha (B' hi + a lo) = alpha (a X + B hi), split into the
+          // new hi and lo; written 8 columns at a time so that only a
+          // quarter of the row's outputs are live at once
           const float alpha = (g.iter == 0) ? s : 1.0f;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) val[q] = alpha * fmaf(a_c, bf_at(xa, q), u2f(v[q]));
-        }
-        if (sym) {
-          __align__(16) __nv_bfloat16 h[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
-          if (inside && md == 1) {
-            // off-diagonal block: stage it and its transpose, store both
-            staging_free();
-            write_row32(blk0, lane, h);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
-            const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
-            publish(map, j0, i_lo, map, i_lo, j0);
-          } else {
-            // diagonal or ragged block: element-wise with masks (a ragged
-            // block below the diagonal is written whole, with its mirror)
-            const bool whole = (md == 1);
-            __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
-            __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const int j = j0 + q;
-              if (i < mi.m && j < mi.m) {
-                if (whole || j <= i) row[j] = h[q];
-                if (whole || j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
-              }
-            }
-          }
-        } else {
-          __align__(16) __nv_bfloat16 h[32];
-          __align__(16) __nv_bfloat16 l[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            h[q] = __float2bfloat16_rn(val[q]);
-            l[q] = __float2bfloat16_rn(val[q] - __bfloat162float(h[q]));
-          }
           if (inside) {
             staging_free();
-            write_row32(blk0, lane, h);
-            write_row32(blk1, lane, l);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              __align__(16) __nv_bfloat16 h8[8];
+              __align__(16) __nv_bfloat16 l8[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float val = alpha * fmaf(a_c, bf_at(xa, 8 * q4 + u), u2f(v[8 * q4 + u]));
+                h8[u] = __float2bfloat16_rn(val);
+                l8[u] = __float2bfloat16_rn(val - __bfloat162float(h8[u]));
+              }
+              *reinterpret_cast<uint4*>(blk0 + chunk_off(lane, q4)) = *reinterpret_cast<const uint4*>(h8);
+              *reinterpret_cast<uint4*>(blk1 + chunk_off(lane, q4)) = *reinterpret_cast<const uint4*>(l8);
+            }
             // blk1 follows blk0: one 3-D store writes the hi block and the lo block
             fence_proxy_async();
             __syncwarp();
@@ -973,9 +938,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q)
               if (j0 + q < mi.cols) {
-                hout[wi + q] = h[q];
-                lout[wi + q] = l[q];
+                const float val = alpha * fmaf(a_c, bf_at(xa, q), u2f(v[q]));
+                const __nv_bfloat16 h = __float2bfloat16_rn(val);
+                hout[wi + q] = h;
+                lout[wi + q] = __float2bfloat16_rn(val - __bfloat162float(h));
               }
+          }
+          continue;
+        }
+        float val[32];
+        if (g.phase == kPhaseGram) {
+          const bool first = (g.iter == 0);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
+        } else {
+          // B' = b A + c A A + a I (the a X term of the update rides on B' hi)
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q)) + (j0 + q == i ? a_c : 0.0f);
+        }
+        // symmetric products
+        __align__(16) __nv_bfloat16 h[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
+        if (inside && md == 1) {
+          // off-diagonal block: stage it and its transpose, store both
+          staging_free();
+          write_row32(blk0, lane, h);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
+          const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
+          publish(map, j0, i_lo, map, i_lo, j0);
+        } else {
+          // diagonal or ragged block: element-wise with masks (a ragged
+          // block below the diagonal is written whole, with its mirror)
+          const bool whole = (md == 1);
+          __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
+          __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int j = j0 + q;
+            if (i < mi.m && j < mi.m) {
+              if (whole || j <= i) row[j] = h[q];
+              if (whole || j < i) out[static_cast<size_t>(j) * mi.lda + i] = h[q];
+            }
           }
         }
       }
