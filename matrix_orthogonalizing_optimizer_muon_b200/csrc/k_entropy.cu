@@ -68,10 +68,13 @@ constexpr int kGramK = 32;
 constexpr int kMaxDim = 8192;        // min(rows, cols) limit (the sort stages 8192 values)
 constexpr int kSortThreads = 1024;
 
-constexpr int kTdThreads = 512;      // tridiagonal reduction: one CTA per matrix
+// tridiagonal reduction: one CTA per matrix, two CTAs per SM (so a batch of
+// up to 2 x 148 matrices is resident at once and no matrix waits for an SM)
+constexpr int kTdThreads = 256;
 constexpr int kTdWarps = kTdThreads / 32;
 constexpr int kTdNb = 32;            // columns per panel
 constexpr int kTdTile = 64;          // trailing-update tile
+constexpr int kSymvRows = 3;         // rows per warp and pass of G0 v (2, 3, 4, 8 measured: 3 best)
 // shared memory of tridiag_kernel, in doubles: the column x, the reflector
 // v and the product y (m_pad each) plus small arrays; the trailing update
 // reuses the space for its operand tiles and the output tile
@@ -206,7 +209,7 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
   double* Vc = Wr + kTdNb * kTdTile;       // [kTdNb][64]: V_k[c0 + cc]
   double* Wc = Vc + kTdNb * kTdTile;
   double* Cs = Wc + kTdNb * kTdTile;       // [64][65] updated tile
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;  // rows ty, ty + 32; columns tx + 16 q
+  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;  // rows ty + 16 u; columns tx + 16 q
   const int nt = (m - t0 + kTdTile - 1) / kTdTile;
   for (int a = 0; a < nt; ++a) {
     for (int b = 0; b <= a; ++b) {
@@ -220,17 +223,20 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
         Wc[e] = (kin && c0 + q < m) ? Wg[static_cast<size_t>(k) * ld + c0 + q] : 0.0;
       }
       __syncthreads();
-      double acc[2][4];
+      // each thread: kRows rows (ty + kTdThreads / 16 apart) x 4 columns (16 apart)
+      constexpr int kRows = kTdTile * kTdTile / (4 * kTdThreads);
+      static_assert(kRows * (kTdThreads / 16) == kTdTile, "trailing tile rows");
+      double acc[kRows][4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int u = 0; u < kRows; ++u)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[u][q] = 0.0;
       for (int k = 0; k < nbk; ++k) {
-        double vr[2], wr[2], vc[4], wc[4];
+        double vr[kRows], wr[kRows], vc[4], wc[4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          vr[u] = Vr[k * kTdTile + ty + 32 * u];
-          wr[u] = Wr[k * kTdTile + ty + 32 * u];
+        for (int u = 0; u < kRows; ++u) {
+          vr[u] = Vr[k * kTdTile + ty + (kTdThreads / 16) * u];
+          wr[u] = Wr[k * kTdTile + ty + (kTdThreads / 16) * u];
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -238,19 +244,19 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
           wc[q] = Wc[k * kTdTile + tx + 16 * q];
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < kRows; ++u)
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[u][q] = fma(vr[u], wc[q], fma(wr[u], vc[q], acc[u][q]));
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = r0 + ty + 32 * u;
+      for (int u = 0; u < kRows; ++u) {
+        const int r = r0 + ty + (kTdThreads / 16) * u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int c = c0 + tx + 16 * q;
           double val = 0.0;
           if (r < m && c < m) val = A[static_cast<size_t>(r) * ld + c] - acc[u][q];
-          Cs[(ty + 32 * u) * (kTdTile + 1) + tx + 16 * q] = val;
+          Cs[(ty + (kTdThreads / 16) * u) * (kTdTile + 1) + tx + 16 * q] = val;
         }
       }
       __syncthreads();
@@ -268,7 +274,7 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
   }
 }
 
-__global__ void __launch_bounds__(kTdThreads, 1)
+__global__ void __launch_bounds__(kTdThreads, 2)
     tridiag_kernel(const EntMat* __restrict__ mats, double* __restrict__ G, double* __restrict__ VW,
                    double* __restrict__ d_out, double* __restrict__ e_out, const EntCtl ctl) {
   extern __shared__ double td_smem[];
@@ -336,32 +342,36 @@ __global__ void __launch_bounds__(kTdThreads, 1)
         __syncthreads();
         continue;
       }
-      // y = G0 v over rows j+1 .. m-1: one warp per row pair, 16-byte loads
-      // from the 64-aligned column at or below j+1 to the padded end (v and
-      // the padding are zero there)
+      // y = G0 v over rows j+1 .. m-1: each warp takes kSymvRows rows at a
+      // time (kTdWarps apart), 16-byte loads from the 64-aligned column at or
+      // below j+1 to the padded end (v and the padding are zero there), so
+      // that kSymvRows x the unroll depth loads are in flight per lane
       {
         const int cs = (j + 1) & ~63;
         const int nq = (ld - cs) >> 6;
         const double2* vv = reinterpret_cast<const double2*>(v + cs) + lane;
-        for (int r = j + 1 + warp; r < m; r += 2 * kTdWarps) {
-          const int r2 = r + kTdWarps;
-          const bool two = r2 < m;
-          const double2* a1 = reinterpret_cast<const double2*>(A + static_cast<size_t>(r) * ld + cs) + lane;
-          const double2* a2 = reinterpret_cast<const double2*>(A + static_cast<size_t>(two ? r2 : r) * ld + cs) + lane;
-          double s1 = 0.0, s2r = 0.0;
+        for (int r = j + 1 + warp; r < m; r += kSymvRows * kTdWarps) {
+          const double2* ap[kSymvRows];
+          double sr[kSymvRows];
+#pragma unroll
+          for (int k = 0; k < kSymvRows; ++k) {
+            const int rk = r + k * kTdWarps;
+            ap[k] = reinterpret_cast<const double2*>(A + static_cast<size_t>(rk < m ? rk : r) * ld + cs) + lane;
+            sr[k] = 0.0;
+          }
 #pragma unroll 4
           for (int q = 0; q < nq; ++q) {
             const double2 b = vv[32 * q];
-            const double2 u1 = __ldcg(a1 + 32 * q);
-            const double2 u2 = __ldcg(a2 + 32 * q);
-            s1 = fma(u1.y, b.y, fma(u1.x, b.x, s1));
-            s2r = fma(u2.y, b.y, fma(u2.x, b.x, s2r));
+#pragma unroll
+            for (int k = 0; k < kSymvRows; ++k) {
+              const double2 u = __ldcg(ap[k] + 32 * q);
+              sr[k] = fma(u.y, b.y, fma(u.x, b.x, sr[k]));
+            }
           }
-          s1 = warp_sum(s1);
-          s2r = warp_sum(s2r);
-          if (lane == 0) {
-            y[r] = s1;
-            if (two) y[r2] = s2r;
+#pragma unroll
+          for (int k = 0; k < kSymvRows; ++k) {
+            const double tot = warp_sum(sr[k]);
+            if (lane == 0 && r + k * kTdWarps < m) y[r + k * kTdWarps] = tot;
           }
         }
         // V_k^T v and W_k^T v of the panel's earlier reflectors, one warp per dot
