@@ -78,7 +78,7 @@ constexpr int kSymvRows = 3;         // rows per warp and pass of G0 v (2, 3, 4,
 // shared memory of tridiag_kernel, in doubles: the column x, the reflector
 // v and the product y (m_pad each) plus small arrays; the trailing update
 // reuses the space for its operand tiles and the output tile
-constexpr int kTdSmall = 4 * kTdNb + 2 * kTdWarps + 16;
+constexpr int kTdSmall = 6 * kTdNb + 2 * kTdWarps + 16;
 constexpr int kTdTrail = 4 * kTdNb * kTdTile + kTdTile * (kTdTile + 1);
 
 constexpr int kBisThreads = 256;     // bisection: one thread per eigenvalue
@@ -107,6 +107,9 @@ struct EntCtl {
 size_t tridiag_smem_bytes(int mp) {
   return static_cast<size_t>(std::max(3 * mp + kTdSmall, kTdTrail)) * sizeof(double);
 }
+// With clusters, each CTA asks for more than half of an SM's shared memory,
+// so the cluster's CTAs land on different SMs.
+constexpr size_t kTdSpreadSmem = 116 * 1024;
 
 // ---------------------------------------------------------------- 1. Gram
 __device__ __forceinline__ float x_at(const float* W, const EntMat& mi, int i, int k) {
@@ -203,7 +206,7 @@ __device__ __forceinline__ double td_block_sum(double s, double* red) {
 // k-sum of one element and of its mirror would round differently, so the
 // mirror is copied, not recomputed.
 __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, const double* Vg, const double* Wg,
-                                   double* sm) {
+                                   double* sm, int rank, int C) {
   double* Vr = sm;                         // [kTdNb][64]: V_k[r0 + rr]
   double* Wr = Vr + kTdNb * kTdTile;
   double* Vc = Wr + kTdNb * kTdTile;       // [kTdNb][64]: V_k[c0 + cc]
@@ -211,16 +214,18 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
   double* Cs = Wc + kTdNb * kTdTile;       // [64][65] updated tile
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;  // rows ty + 16 u; columns tx + 16 q
   const int nt = (m - t0 + kTdTile - 1) / kTdTile;
+  int tix = 0;  // tile index; tile tix belongs to CTA tix mod C of the cluster
   for (int a = 0; a < nt; ++a) {
-    for (int b = 0; b <= a; ++b) {
+    for (int b = 0; b <= a; ++b, ++tix) {
+      if (tix % C != rank) continue;
       const int r0 = t0 + a * kTdTile, c0 = t0 + b * kTdTile;
       for (int e = t; e < kTdNb * kTdTile; e += kTdThreads) {
         const int k = e >> 6, q = e & 63;
         const bool kin = k < nbk;
-        Vr[e] = (kin && r0 + q < m) ? Vg[static_cast<size_t>(k) * ld + r0 + q] : 0.0;
-        Wr[e] = (kin && r0 + q < m) ? Wg[static_cast<size_t>(k) * ld + r0 + q] : 0.0;
-        Vc[e] = (kin && c0 + q < m) ? Vg[static_cast<size_t>(k) * ld + c0 + q] : 0.0;
-        Wc[e] = (kin && c0 + q < m) ? Wg[static_cast<size_t>(k) * ld + c0 + q] : 0.0;
+        Vr[e] = (kin && r0 + q < m) ? __ldcg(Vg + static_cast<size_t>(k) * ld + r0 + q) : 0.0;
+        Wr[e] = (kin && r0 + q < m) ? __ldcg(Wg + static_cast<size_t>(k) * ld + r0 + q) : 0.0;
+        Vc[e] = (kin && c0 + q < m) ? __ldcg(Vg + static_cast<size_t>(k) * ld + c0 + q) : 0.0;
+        Wc[e] = (kin && c0 + q < m) ? __ldcg(Wg + static_cast<size_t>(k) * ld + c0 + q) : 0.0;
       }
       __syncthreads();
       // each thread: kRows rows (ty + kTdThreads / 16 apart) x 4 columns (16 apart)
@@ -255,7 +260,7 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
         for (int q = 0; q < 4; ++q) {
           const int c = c0 + tx + 16 * q;
           double val = 0.0;
-          if (r < m && c < m) val = A[static_cast<size_t>(r) * ld + c] - acc[u][q];
+          if (r < m && c < m) val = __ldcg(A + static_cast<size_t>(r) * ld + c) - acc[u][q];
           Cs[(ty + (kTdThreads / 16) * u) * (kTdTile + 1) + tx + 16 * q] = val;
         }
       }
@@ -274,11 +279,50 @@ __device__ void td_trailing_update(double* A, int ld, int m, int t0, int nbk, co
   }
 }
 
+// Thread-block cluster helpers: the kernel runs one cluster of C CTAs per
+// matrix (C = 1 for large batches).
+__device__ __forceinline__ uint32_t cl_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster; release/acquire at cluster scope
+// orders the CTAs' global and shared writes before the other CTAs' reads
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a double in CTA `rank`'s shared memory at the address of `p` in this CTA
+__device__ __forceinline__ double cl_load(const double* p, uint32_t rank) {
+  const uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 __global__ void __launch_bounds__(kTdThreads, 2)
     tridiag_kernel(const EntMat* __restrict__ mats, double* __restrict__ G, double* __restrict__ VW,
                    double* __restrict__ d_out, double* __restrict__ e_out, const EntCtl ctl) {
   extern __shared__ double td_smem[];
-  const int p = blockIdx.x;
+  // one cluster of C CTAs per matrix.  Every CTA forms column j, the
+  // reflector and v in full (the same arithmetic on the same data, so the
+  // same values); the rows j+1 .. m-1 of G0 v, of the dot products and of w
+  // are split into C contiguous chunks, and the chunks' partial dot
+  // products are summed over the ranks in rank order.
+  const int C = static_cast<int>(cl_nctarank());
+  const uint32_t rank = cl_ctarank();
+  const int p = static_cast<int>(cl_id_x());
   const EntMat mi = mats[p];
   const int m = mi.m, ld = mi.mp;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -289,19 +333,29 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   double* e = e_out + mi.sv_off;
   double* x = td_smem;          // column j, rows j .. m-1
   double* v = x + ld;           // reflector, zero outside j+1 .. m-1 (and over the padding)
-  double* y = v + ld;           // G0 v, then w
+  double* y = v + ld;           // G0 v, then w (this CTA's rows)
   double* vj = y + ld;          // V_k[j], W_k[j] for the panel's earlier reflectors
   double* wj = vj + kTdNb;
   double* pq = wj + kTdNb;      // [2 kTdNb]: V_k^T v, W_k^T v interleaved
   double* red = pq + 2 * kTdNb; // [kTdWarps]
+  double* pq_part = red + kTdWarps;      // [2 kTdNb]: this CTA's chunk of the dots
+  double* sv_part = pq_part + 2 * kTdNb; // [1]
+  auto csync = [&]() {
+    if (C > 1) cl_sync();
+    else __syncthreads();
+  };
 
   for (int k = 0; k < m - 1; k += kTdNb) {
     const int nbk = min(kTdNb, m - 1 - k);
     for (int i = 0; i < nbk; ++i) {
       const int j = k + i;
+      // this CTA's rows of j+1 .. m-1
+      const int chunk = (m - 1 - j + C - 1) / C;
+      const int lo = min(m, j + 1 + static_cast<int>(rank) * chunk);
+      const int hi = min(m, lo + chunk);
       if (t < i) {
-        vj[t] = Vg[static_cast<size_t>(t) * ld + j];
-        wj[t] = Wg[static_cast<size_t>(t) * ld + j];
+        vj[t] = __ldcg(Vg + static_cast<size_t>(t) * ld + j);
+        wj[t] = __ldcg(Wg + static_cast<size_t>(t) * ld + j);
       }
       __syncthreads();
       // column j of the current matrix: row j of G0 minus the panel's terms
@@ -309,7 +363,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
       for (int r = j + t; r < m; r += kTdThreads) {
         double a = __ldcg(A + static_cast<size_t>(j) * ld + r);
         for (int c = 0; c < i; ++c)
-          a -= fma(Vg[static_cast<size_t>(c) * ld + r], wj[c], Wg[static_cast<size_t>(c) * ld + r] * vj[c]);
+          a -= fma(__ldcg(Vg + static_cast<size_t>(c) * ld + r), wj[c],
+                   __ldcg(Wg + static_cast<size_t>(c) * ld + r) * vj[c]);
         x[r] = a;
         if (r >= j + 2) s2 = fma(a, a, s2);
       }
@@ -322,11 +377,11 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         sc = 1.0 / (alpha - beta);
         ej = beta;
       }
-      if (t == 0) {
+      if (t == 0 && rank == 0) {
         d[j] = x[j];
         e[j] = ej;
       }
-      // v over the whole padded range (zero outside j+1 .. m-1); V_i = v
+      // v over the whole padded range (zero outside j+1 .. m-1); V_i = v on this CTA's rows
       for (int r = t; r < ld; r += kTdThreads) {
         double val = 0.0;
         if (tau != 0.0) {
@@ -334,15 +389,15 @@ __global__ void __launch_bounds__(kTdThreads, 2)
           else if (r > j + 1 && r < m) val = x[r] * sc;
         }
         v[r] = val;
-        if (r > j && r < m) Vg[static_cast<size_t>(i) * ld + r] = val;
+        if (r >= lo && r < hi) Vg[static_cast<size_t>(i) * ld + r] = val;
       }
       __syncthreads();
-      if (tau == 0.0) {  // the reflector is the identity (tau is the same in every thread)
-        for (int r = j + 1 + t; r < m; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = 0.0;
-        __syncthreads();
+      if (tau == 0.0) {  // the reflector is the identity (tau is the same in every thread of the cluster)
+        for (int r = lo + t; r < hi; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = 0.0;
+        csync();
         continue;
       }
-      // y = G0 v over rows j+1 .. m-1: each warp takes kSymvRows rows at a
+      // y = G0 v over this CTA's rows: each warp takes kSymvRows rows at a
       // time (kTdWarps apart), 16-byte loads from the 64-aligned column at or
       // below j+1 to the padded end (v and the padding are zero there), so
       // that kSymvRows x the unroll depth loads are in flight per lane
@@ -350,13 +405,13 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         const int cs = (j + 1) & ~63;
         const int nq = (ld - cs) >> 6;
         const double2* vv = reinterpret_cast<const double2*>(v + cs) + lane;
-        for (int r = j + 1 + warp; r < m; r += kSymvRows * kTdWarps) {
+        for (int r = lo + warp; r < hi; r += kSymvRows * kTdWarps) {
           const double2* ap[kSymvRows];
           double sr[kSymvRows];
 #pragma unroll
           for (int k = 0; k < kSymvRows; ++k) {
             const int rk = r + k * kTdWarps;
-            ap[k] = reinterpret_cast<const double2*>(A + static_cast<size_t>(rk < m ? rk : r) * ld + cs) + lane;
+            ap[k] = reinterpret_cast<const double2*>(A + static_cast<size_t>(rk < hi ? rk : r) * ld + cs) + lane;
             sr[k] = 0.0;
           }
 #pragma unroll 4
@@ -371,55 +426,69 @@ __global__ void __launch_bounds__(kTdThreads, 2)
 #pragma unroll
           for (int k = 0; k < kSymvRows; ++k) {
             const double tot = warp_sum(sr[k]);
-            if (lane == 0 && r + k * kTdWarps < m) y[r + k * kTdWarps] = tot;
+            if (lane == 0 && r + k * kTdWarps < hi) y[r + k * kTdWarps] = tot;
           }
         }
-        // V_k^T v and W_k^T v of the panel's earlier reflectors, one warp per dot
+        // this CTA's chunk of V_k^T v and W_k^T v, one warp per dot
         for (int dd = warp; dd < 2 * i; dd += kTdWarps) {
           const double* src = ((dd & 1) ? Wg : Vg) + static_cast<size_t>(dd >> 1) * ld;
           double s = 0.0;
-          for (int r = j + 1 + lane; r < m; r += 32) s = fma(src[r], v[r], s);
+          for (int r = lo + lane; r < hi; r += 32) s = fma(__ldcg(src + r), v[r], s);
           s = warp_sum(s);
-          if (lane == 0) pq[dd] = s;
+          if (lane == 0) pq_part[dd] = s;
         }
+      }
+      csync();
+      if (t < 2 * i) {
+        double s = 0.0;
+        for (int q = 0; q < C; ++q) s += (C > 1) ? cl_load(pq_part + t, static_cast<uint32_t>(q)) : pq_part[t];
+        pq[t] = s;
       }
       __syncthreads();
       // y <- tau (y - V (W^T v) - W (V^T v)); then w = y - (tau/2)(v^T y) v
       double sv = 0.0;
-      for (int r = j + 1 + t; r < m; r += kTdThreads) {
+      for (int r = lo + t; r < hi; r += kTdThreads) {
         double yy = y[r];
         for (int c = 0; c < i; ++c)
-          yy -= fma(Vg[static_cast<size_t>(c) * ld + r], pq[2 * c + 1], Wg[static_cast<size_t>(c) * ld + r] * pq[2 * c]);
+          yy -= fma(__ldcg(Vg + static_cast<size_t>(c) * ld + r), pq[2 * c + 1],
+                    __ldcg(Wg + static_cast<size_t>(c) * ld + r) * pq[2 * c]);
         yy *= tau;
         y[r] = yy;
         sv = fma(yy, v[r], sv);
       }
       sv = td_block_sum(sv, red);
+      if (C > 1) {
+        if (t == 0) sv_part[0] = sv;
+        csync();
+        sv = 0.0;
+        for (int q = 0; q < C; ++q) sv += cl_load(sv_part, static_cast<uint32_t>(q));
+      }
       const double a2 = -0.5 * tau * sv;
-      for (int r = j + 1 + t; r < m; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = fma(a2, v[r], y[r]);
-      __syncthreads();
+      for (int r = lo + t; r < hi; r += kTdThreads) Wg[static_cast<size_t>(i) * ld + r] = fma(a2, v[r], y[r]);
+      csync();  // W_i (and V_i) complete in every CTA of the cluster
     }
-    td_trailing_update(A, ld, m, k + nbk, nbk, Vg, Wg, td_smem);
+    td_trailing_update(A, ld, m, k + nbk, nbk, Vg, Wg, td_smem, static_cast<int>(rank), C);
+    csync();
   }
-  // the last diagonal element, then the finiteness check of T
-  if (t == 0) {
-    d[m - 1] = A[static_cast<size_t>(m - 1) * ld + m - 1];
-  }
-  __syncthreads();
-  int bad = 0;
-  for (int r = t; r < m; r += kTdThreads) {
-    if (!isfinite(d[r])) bad = 1;
-    if (r < m - 1 && !isfinite(e[r])) bad = 1;
-  }
-  bad = __syncthreads_or(bad);
-  if (t == 0) {
-    if (bad) {
-      ctl.conv[p] = kConvNonFinite;
-      ctl.sweeps[p] = 0;
-      atomicOr(ctl.status, kStatusNonFinite);
-    } else {
-      ctl.conv[p] = kConvDone;
-      ctl.sweeps[p] = 1;
+  // the last diagonal element, then the finiteness check of T (rank 0)
+  if (rank == 0) {
+    if (t == 0) d[m - 1] = __ldcg(A + static_cast<size_t>(m - 1) * ld + m - 1);
+    __syncthreads();
+    int bad = 0;
+    for (int r = t; r < m; r += kTdThreads) {
+      if (!isfinite(d[r])) bad = 1;
+      if (r < m - 1 && !isfinite(e[r])) bad = 1;
+    }
+    bad = __syncthreads_or(bad);
+    if (t == 0) {
+      if (bad) {
+        ctl.conv[p] = kConvNonFinite;
+        ctl.sweeps[p] = 0;
+        atomicOr(ctl.status, kStatusNonFinite);
+      } else {
+        ctl.conv[p] = kConvDone;
+        ctl.sweeps[p] = 1;
+      }
     }
   }
 }
@@ -584,6 +653,8 @@ struct muon_entropy_plan_s {
   int n = 0;
   int ntiles = 0, nbis = 0;
   int mp_max = 64, m_max = 1;
+  int td_cluster = 1;     // CTAs per matrix in the tridiagonal reduction
+  size_t td_smem = 0;     // its dynamic shared memory per CTA
   int64_t total_sv = 0;
   std::vector<EntMat> mats;
   char* dmem = nullptr;
@@ -717,8 +788,42 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
                  cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&pl->ev, cudaEventDisableTiming) == cudaSuccess;
   for (int k = 0; k < 5 && ok; ++k) ok = cudaEventCreate(&pl->prof[k]) == cudaSuccess;
+  // Cluster size of the reduction: the largest C in {16, 8, 4, 2} for which
+  // all n clusters are resident at once with one CTA per SM (a plan of a
+  // few large matrices then spreads each matrix over C SMs); otherwise one
+  // CTA per matrix, two per SM.
+  const size_t smem1 = tridiag_smem_bytes(pl->mp_max);
+  const size_t smem_c = std::max(smem1, kTdSpreadSmem);
   ok = ok && cudaFuncSetAttribute(tridiag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(tridiag_smem_bytes(pl->mp_max))) == cudaSuccess;
+                                  static_cast<int>(smem_c)) == cudaSuccess;
+  if (ok) {
+    const bool nonportable =
+        cudaFuncSetAttribute(tridiag_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    cudaGetLastError();
+    pl->td_cluster = 1;
+    pl->td_smem = smem1;
+    for (int c : {16, 8, 4, 2}) {
+      if (c > 8 && !nonportable) continue;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(kTdThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem_c;
+      cudaLaunchAttribute at;
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = c;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      cfg.attrs = &at;
+      cfg.numAttrs = 1;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, tridiag_kernel, &cfg) == cudaSuccess && nc >= n) {
+        pl->td_cluster = c;
+        pl->td_smem = smem_c;
+        break;
+      }
+      cudaGetLastError();
+    }
+  }
   ok = ok && cudaFuncSetAttribute(bisect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(2 * pl->m_max * sizeof(double))) == cudaSuccess;
   if (!ok) {
@@ -785,9 +890,22 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[0], st) == cudaSuccess;
   if (ok) gram_kernel<<<pl->ntiles, kEThreads, 0, st>>>(pl->tiles_d, pl->mats_d, pl->wptr_d, pl->G);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[1], st) == cudaSuccess;
-  if (ok)
-    tridiag_kernel<<<n, kTdThreads, tridiag_smem_bytes(pl->mp_max), st>>>(pl->mats_d, pl->G, pl->VW, pl->dvec,
-                                                                         pl->evec, ctl);
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n * pl->td_cluster), 1, 1);
+    cfg.blockDim = dim3(kTdThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl->td_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = static_cast<unsigned>(pl->td_cluster);
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    ok = cudaLaunchKernelEx(&cfg, tridiag_kernel, static_cast<const EntMat*>(pl->mats_d), pl->G, pl->VW, pl->dvec,
+                            pl->evec, ctl) == cudaSuccess;
+  }
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[2], st) == cudaSuccess;
   if (ok)
     bisect_kernel<<<pl->nbis, kBisThreads, 2 * pl->m_max * sizeof(double), st>>>(pl->bis_d, pl->mats_d, pl->dvec,
