@@ -392,6 +392,15 @@ MUON_API muon_status_t muon_entropy_compute(muon_entropy_plan_t plan, const floa
 /* Total number of singular values of the plan (sum of min(rows, cols)); -1 for NULL. */
 MUON_API int64_t muon_entropy_num_singular_values(muon_entropy_plan_t plan);
 
+/* CTAs per matrix of the plan's tridiagonal reduction (one thread-block
+ * cluster per matrix: 16, 8, 4 or 2 when all the plan's clusters fit on the
+ * GPU at once with one CTA per SM, else 1), chosen by muon_entropy_init;
+ * -1 for NULL.  The partial dot products of a column are summed over the
+ * cluster's CTAs in rank order, so results are bitwise reproducible for a
+ * given plan and may differ in the last bits between plans whose cluster
+ * sizes differ. */
+MUON_API int32_t muon_entropy_cluster_size(muon_entropy_plan_t plan);
+
 /* Synchronises the plan's last stream, then returns and clears the sticky
  * status of the calls since the previous read: MUON_OK or
  * MUON_ERR_NONFINITE (a matrix had non-finite entries; its H and singular

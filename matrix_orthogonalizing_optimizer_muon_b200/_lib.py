@@ -42,7 +42,7 @@ EXPORTED = ("muon_hparams_default", "muon_init", "muon_init_ex", "muon_num_waves
             "muon_step", "muon_orthogonalize", "muon_workspace_bytes",
             "muon_get_status", "muon_destroy", "muon_status_string", "muon_profile_enable", "muon_profile_read",
             "muon_orthogonalize_noalloc", "muon_adamw_hparams_default", "muon_adamw_init", "muon_adamw_step",
-            "muon_adamw_destroy", "muon_entropy_init", "muon_entropy_compute", "muon_entropy_num_singular_values",
+            "muon_adamw_destroy", "muon_entropy_init", "muon_entropy_compute", "muon_entropy_num_singular_values", "muon_entropy_cluster_size",
             "muon_entropy_get_status", "muon_entropy_profile", "muon_entropy_destroy", "muon_pack_init",
             "muon_pack_run", "muon_pack_destroy")
 
@@ -148,6 +148,8 @@ def load() -> ctypes.CDLL:
     lib.muon_entropy_compute.restype = ctypes.c_int
     lib.muon_entropy_num_singular_values.argtypes = [P]
     lib.muon_entropy_num_singular_values.restype = ctypes.c_int64
+    lib.muon_entropy_cluster_size.argtypes = [P]
+    lib.muon_entropy_cluster_size.restype = ctypes.c_int32
     lib.muon_entropy_get_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
     lib.muon_entropy_get_status.restype = ctypes.c_int
     lib.muon_entropy_profile.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]
@@ -290,6 +292,10 @@ def muon_entropy_compute(plan, w_ptrs, n: int, h_ptr: int, sigma_ptr: int | None
 
 def muon_entropy_num_singular_values(plan) -> int:
     return int(load().muon_entropy_num_singular_values(plan))
+
+
+def muon_entropy_cluster_size(plan) -> int:
+    return int(load().muon_entropy_cluster_size(plan))
 
 
 def muon_entropy_get_status(plan, n: int):

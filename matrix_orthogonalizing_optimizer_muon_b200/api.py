@@ -342,6 +342,8 @@ class EntropyPlan:
         self.n = len(self.shapes)
         self._plan = L.muon_entropy_init(self.shapes, _stream_handle(stream))
         self.num_singular_values = L.muon_entropy_num_singular_values(self._plan)
+        # CTAs per matrix in the tridiagonal reduction (a cluster per matrix)
+        self.cluster_size = L.muon_entropy_cluster_size(self._plan)
         self._w = (ctypes.c_void_p * self.n)()
 
     def compute(self, weights, H=None, sigma=None, *, stream=None) -> torch.Tensor:

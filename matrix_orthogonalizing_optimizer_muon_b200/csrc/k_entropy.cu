@@ -965,6 +965,8 @@ extern "C" int64_t muon_entropy_num_singular_values(muon_entropy_plan_t pl) {
   return pl == nullptr ? -1 : pl->total_sv;
 }
 
+extern "C" int32_t muon_entropy_cluster_size(muon_entropy_plan_t pl) { return pl == nullptr ? -1 : pl->td_cluster; }
+
 extern "C" void muon_entropy_destroy(muon_entropy_plan_t pl) {
   if (pl == nullptr) return;
   cudaStreamSynchronize(pl->last_stream);

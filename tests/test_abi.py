@@ -170,6 +170,7 @@ def test_entropy_entry_points_reject_bad_arguments_before_any_cuda_call(lib):
     assert lib.muon_entropy_get_status(None, None) == L.MUON_ERR_INVALID_ARG
     assert lib.muon_entropy_profile(None, 1, None) == L.MUON_ERR_INVALID_ARG
     assert lib.muon_entropy_num_singular_values(None) == -1
+    assert lib.muon_entropy_cluster_size(None) == -1
     lib.muon_entropy_destroy(None)
 
 

@@ -85,3 +85,35 @@ def test_large_batch_runs_one_cta_per_matrix():
         assert np.max(np.abs(got[off:off + m] ** 2 - want ** 2)) <= 3e-7 * want[0] ** 2
         off += m
     plan.close()
+
+
+def test_cluster_size_follows_the_plan_and_results_agree():
+    """The reduction's cluster size shrinks as the plan grows (up to 16 CTAs
+    per matrix for a few matrices, one CTA per matrix for large batches;
+    clusters are used only when all of them fit at once with one CTA per
+    SM).  One matrix computed inside plans of different sizes matches the
+    oracle's H and spectrum every time, whatever the cluster size."""
+    rng = np.random.default_rng(51)
+    W0 = np.ascontiguousarray(rng.standard_normal((300, 520)), dtype=np.float32)
+    want = ent.singular_values(W0)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    sizes = []
+    for count in (1, 6, 30, 40, 160):
+        mats = [W0] + [np.ascontiguousarray(rng.standard_normal((48, 80)), dtype=np.float32)
+                       for _ in range(count - 1)]
+        plan = EntropyPlan([W.shape for W in mats])
+        c = plan.cluster_size
+        assert c in (1, 2, 4, 8, 16)
+        assert c == 1 or c * count <= sms, (count, c)
+        sizes.append(c)
+        sig = torch.empty(plan.num_singular_values, device="cuda")
+        H = plan.compute([torch.from_numpy(W).cuda() for W in mats], sigma=sig)
+        torch.cuda.synchronize()
+        assert plan.status()[0] == L.MUON_OK
+        assert abs(float(H[0]) - ent.entropy_of_spectrum(want)) <= 2e-7, (count, c)
+        got = sig[:min(W0.shape)].cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(got ** 2 - want ** 2)) <= 3e-7 * want[0] ** 2, (count, c)
+        plan.close()
+    assert sizes == sorted(sizes, reverse=True), sizes
+    assert sizes[0] >= 8 and sizes[-1] == 1, sizes
+    assert len(set(sizes)) >= 3, sizes  # several cluster sizes were exercised
