@@ -215,6 +215,7 @@ def bench_entropy(Ws, calls: int = 2):
     from matrix_orthogonalizing_optimizer_muon_b200.api import EntropyPlan
     shapes = [tuple(W.shape) for W in Ws]
     plan = EntropyPlan(shapes)
+    plan_cluster = plan.cluster_size
     H = plan.compute(Ws)  # warm-up
     torch.cuda.synchronize()
     plan.profile(True)
@@ -226,7 +227,7 @@ def bench_entropy(Ws, calls: int = 2):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / calls
     phases = plan.profile_read()
-    st, sweeps = plan.status()
+    st, computed = plan.status()
     plan.close()
     nbytes = entropy_trailing_bytes(shapes)
     achieved = nbytes / (phases["tridiagonal"] * 1e-3) / 1e9
@@ -235,7 +236,8 @@ def bench_entropy(Ws, calls: int = 2):
     return {"what": "SVD entropy (Sec. 3.4) of every weight matrix after the timed steps: fp64 Gram, Householder "
                     "tridiagonal reduction, bisection on Sturm counts, entropy; one call covers all matrices",
             "matrices": len(Ws), "ms_per_call": ms, "phases_ms": phases, "status": st,
-            "computed": [min(sweeps), max(sweeps)], "kernel": "tridiag_kernel (fp64, one CTA per matrix)",
+            "computed": [min(computed), max(computed)],
+            "kernel": f"tridiag_kernel (fp64, {plan_cluster} CTA(s) per matrix)",
             "bound": "hbm", "achieved": achieved, "unit": "GB/s", "peak": hbm, "peak_source": f"hbm_gbs ({kind})",
             "frac": achieved / hbm,
             "achieved_basis": "the trailing block streamed once per column for G0 v (8 sum L^2 bytes per matrix) "

@@ -405,11 +405,11 @@ MUON_API int32_t muon_entropy_cluster_size(muon_entropy_plan_t plan);
  * status of the calls since the previous read: MUON_OK or
  * MUON_ERR_NONFINITE (a matrix had non-finite entries; its H and singular
  * values are NaN).
- * sweeps_out: NULL or a host int32 array [n] that receives, for the last
+ * computed_out: NULL or a host int32 array [n] that receives, for the last
  * call, 1 for each matrix whose eigenvalues were computed (one reduction and
  * bisection pass) and 0 for a non-finite one.
  * CUDA errors: MUON_ERR_CUDA. */
-MUON_API muon_status_t muon_entropy_get_status(muon_entropy_plan_t plan, int32_t* sweeps_out);
+MUON_API muon_status_t muon_entropy_get_status(muon_entropy_plan_t plan, int32_t* computed_out);
 
 /* Per-phase timing of the next calls with CUDA events when enable != 0.
  * ms_out: NULL, or a host double array [4] that receives the Gram,

@@ -299,10 +299,11 @@ def muon_entropy_cluster_size(plan) -> int:
 
 
 def muon_entropy_get_status(plan, n: int):
-    """(status code, sweeps per matrix) -- synchronising read-and-clear."""
-    sweeps = (ctypes.c_int32 * n)()
-    st = int(load().muon_entropy_get_status(plan, sweeps))
-    return st, list(sweeps)
+    """(status code, per matrix 1 if its eigenvalues were computed, 0 if it
+    was non-finite) -- synchronising read-and-clear."""
+    computed = (ctypes.c_int32 * n)()
+    st = int(load().muon_entropy_get_status(plan, computed))
+    return st, list(computed)
 
 
 def muon_entropy_profile(plan, enable: bool, read: bool = False):

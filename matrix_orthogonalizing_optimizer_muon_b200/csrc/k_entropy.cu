@@ -100,7 +100,7 @@ struct EntMat {
 
 struct EntCtl {
   int* conv;        // [n] kConv*
-  int* sweeps;      // [n] 1 once the eigenvalues are computed, 0 for a non-finite matrix
+  int* computed;    // [n] 1 once the eigenvalues are computed, 0 for a non-finite matrix
   unsigned* status; // [1] sticky: kStatusNonFinite
 };
 
@@ -483,11 +483,11 @@ __global__ void __launch_bounds__(kTdThreads, 2)
     if (t == 0) {
       if (bad) {
         ctl.conv[p] = kConvNonFinite;
-        ctl.sweeps[p] = 0;
+        ctl.computed[p] = 0;
         atomicOr(ctl.status, kStatusNonFinite);
       } else {
         ctl.conv[p] = kConvDone;
-        ctl.sweeps[p] = 1;
+        ctl.computed[p] = 1;
       }
     }
   }
@@ -776,14 +776,14 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
   pl->bis_d = reinterpret_cast<int2*>(b + o_b);
   pl->wptr_d = reinterpret_cast<const float**>(b + o_w);
   pl->ctl.conv = reinterpret_cast<int*>(b + o_conv);
-  pl->ctl.sweeps = reinterpret_cast<int*>(b + o_sw);
+  pl->ctl.computed = reinterpret_cast<int*>(b + o_sw);
   pl->ctl.status = reinterpret_cast<unsigned*>(b + o_st);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   bool ok = cudaMemcpy(pl->mats_d, pl->mats.data(), n * sizeof(EntMat), cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(pl->tiles_d, tiles.data(), tiles.size() * sizeof(int4), cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(pl->bis_d, bis.data(), bis.size() * sizeof(int2), cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(pl->ctl.status, 0, sizeof(unsigned)) == cudaSuccess &&
-            cudaMemset(pl->ctl.sweeps, 0, n * sizeof(int)) == cudaSuccess;
+            cudaMemset(pl->ctl.computed, 0, n * sizeof(int)) == cudaSuccess;
   ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&pl->pinned), n * sizeof(float*), cudaHostAllocDefault) ==
                  cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&pl->ev, cudaEventDisableTiming) == cudaSuccess;
@@ -886,7 +886,7 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
   }
   const EntCtl ctl = pl->ctl;
   bool ok = cudaMemsetAsync(ctl.conv, 0, n * sizeof(int), st) == cudaSuccess &&
-            cudaMemsetAsync(ctl.sweeps, 0, n * sizeof(int), st) == cudaSuccess;
+            cudaMemsetAsync(ctl.computed, 0, n * sizeof(int), st) == cudaSuccess;
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[0], st) == cudaSuccess;
   if (ok) gram_kernel<<<pl->ntiles, kEThreads, 0, st>>>(pl->tiles_d, pl->mats_d, pl->wptr_d, pl->G);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[1], st) == cudaSuccess;
@@ -922,7 +922,7 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
   return MUON_OK;
 }
 
-extern "C" muon_status_t muon_entropy_get_status(muon_entropy_plan_t pl, int32_t* sweeps_out) {
+extern "C" muon_status_t muon_entropy_get_status(muon_entropy_plan_t pl, int32_t* computed_out) {
   if (pl == nullptr) return MUON_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(pl->last_stream) != cudaSuccess) {
     cudaGetLastError();
@@ -931,8 +931,8 @@ extern "C" muon_status_t muon_entropy_get_status(muon_entropy_plan_t pl, int32_t
   unsigned s = 0;
   if (cudaMemcpy(&s, pl->ctl.status, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemset(pl->ctl.status, 0, sizeof(unsigned)) != cudaSuccess ||
-      (sweeps_out != nullptr &&
-       cudaMemcpy(sweeps_out, pl->ctl.sweeps, pl->n * sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)) {
+      (computed_out != nullptr &&
+       cudaMemcpy(computed_out, pl->ctl.computed, pl->n * sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)) {
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
