@@ -62,17 +62,18 @@ def kernel_source_hash() -> str:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
-    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary
-    (scaled there to one launch of the workload it names); None unless the
-    summary was taken on the current kernel source and on this workload."""
+def ncu_summary(workload: str):
+    """The committed ncu summary of the GEMM kernel (per-launch DRAM bytes,
+    scaled there to one launch of the workload it names, and the tensor-pipe
+    utilisation per phase); None unless it was taken on the current kernel
+    source and on this workload."""
     p = os.path.join(ROOT, "profiles", "ns_gemm_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     if d.get("kernel_sha256_16") != kernel_source_hash() or d.get("workload") != workload:
         return None
-    return d.get("bytes_per_launch")
+    return d
 
 
 class ClockSampler:
@@ -578,12 +579,22 @@ def main(argv=None) -> int:
     plan.profile_read()
     barrier()
     torch.cuda.synchronize()
+    # one more event per step boundary gives the per-step times (their
+    # median is reported beside the mean); a boundary event sits between two
+    # steps, not inside the Newton-Schulz chain
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
     with ClockSampler(local) as clk:
         ev0.record(stream)
-        for _ in range(args.steps):
+        for k in range(args.steps):
             plan.step(**hp, update_rms=rms)
+            if k < args.steps - 1:
+                step_ev[k].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize()
+    bounds = [ev0] + step_ev + [ev1]
+    step_ms = sorted(bounds[k].elapsed_time(bounds[k + 1]) for k in range(args.steps))
+    half = len(step_ms) // 2
+    ms_median = step_ms[half] if len(step_ms) % 2 else 0.5 * (step_ms[half - 1] + step_ms[half])
     barrier()
     plan.profile(False)
     prof = plan.profile_read()
@@ -678,7 +689,9 @@ def main(argv=None) -> int:
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     k1_ms = prof["ms"]["momentum_normalise"] / calls
     k1_gbs = total * K1_BYTES_PER_ELEM / (k1_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(wl.name)
+    summary = ncu_summary(wl.name)
+    traffic = summary.get("bytes_per_launch") if summary else None
+    tensor_pipe = summary.get("tensor_pipe_active_pct") if summary else None
 
     context = None
     if not args.no_context:
@@ -727,6 +740,7 @@ def main(argv=None) -> int:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+        "ms_per_step_median": ms_median,
         "ns_ms_per_step": gemm_ms, "ns_tflops": achieved,
         "ns_pct_of_bf16_peak": 100.0 * achieved / peak,
         "ns_tflops_dense_equivalent": dense_flops / (gemm_ms * 1e-3) / 1e12,
@@ -740,6 +754,7 @@ def main(argv=None) -> int:
                                            "launches",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"bf16_tflops_sustained ({peak_kind})", "traffic": traffic,
+                     "ncu_tensor_pipe_active_pct": tensor_pipe,
                      "algorithmic_flops_per_launch": nz_flops / gemm_launches},
         "elementwise": {"kernel": "k1_kernel (momentum, Nesterov, norm, bf16 split)", "bound": "hbm",
                         "achieved": k1_gbs, "peak": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
