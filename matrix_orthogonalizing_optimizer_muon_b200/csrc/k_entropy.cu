@@ -62,9 +62,12 @@
 namespace muon {
 namespace {
 
-constexpr int kEThreads = 256;
-constexpr int kGramTile = 64;
-constexpr int kGramK = 32;
+constexpr int kGramTile = 128;
+constexpr int kGramK = 16;
+constexpr int kGramLd = kGramTile + 2;  // shared-memory pitch of a staged operand row (doubles)
+constexpr int kGramThreads = 256;
+constexpr int kPad = 64;                // G's row pitch is m rounded up to a multiple of kPad
+constexpr size_t kGramSmem = static_cast<size_t>(kGramTile) * (kGramTile + 1) * sizeof(double);
 constexpr int kMaxDim = 8192;        // min(rows, cols) limit (the sort stages 8192 values)
 constexpr int kSortThreads = 1024;
 
@@ -117,65 +120,93 @@ __device__ __forceinline__ float x_at(const float* W, const EntMat& mi, int i, i
   return mi.tall ? __ldg(W + static_cast<size_t>(k) * mi.cols + i) : __ldg(W + static_cast<size_t>(i) * mi.cols + k);
 }
 
-__global__ void __launch_bounds__(kEThreads) gram_kernel(const int4* __restrict__ tiles, const EntMat* __restrict__ mats,
-                                                         const float* const* __restrict__ wptr, double* __restrict__ G) {
-  // the K-loop staging (As, Bs) and the output tile (Cs) share one buffer
-  __shared__ double buf[kGramTile * (kGramTile + 1)];
-  float (*As)[kGramTile + 1] = reinterpret_cast<float (*)[kGramTile + 1]>(buf);
-  float (*Bs)[kGramTile + 1] = As + kGramK;
-  double (*Cs)[kGramTile + 1] = reinterpret_cast<double (*)[kGramTile + 1]>(buf);
+// G = X X^T over 128 x 128 tiles of the lower triangle (written with their
+// mirror, so G is stored whole and exactly symmetric; a diagonal tile's two
+// halves are the same products in the same order, hence equal).  K runs in
+// chunks of kGramK: each chunk of both operands is converted to fp64 once,
+// into shared memory [k][row], double-buffered through registers; a thread
+// accumulates an 8 x 8 block (rows 8 ty + i, columns tx + 16 j) in k order,
+// so every element is the sequential fp64 sum of the exact fp32 products.
+__global__ void __launch_bounds__(kGramThreads, 1) gram_kernel(const int4* __restrict__ tiles,
+                                                               const EntMat* __restrict__ mats,
+                                                               const float* const* __restrict__ wptr,
+                                                               double* __restrict__ G) {
+  extern __shared__ double gsm[];
+  double* As = gsm;                              // [2][kGramK][kGramLd]
+  double* Bs = As + 2 * kGramK * kGramLd;        // [2][kGramK][kGramLd]
+  double* Cs = gsm;                              // [kGramTile][kGramTile + 1], after the K loop
   const int4 td = tiles[blockIdx.x];
   const EntMat mi = mats[td.x];
   const float* W = wptr[td.x];
   const int i0 = td.y * kGramTile, j0 = td.z * kGramTile;
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  double acc[4][4];
+  // staging: wide (X = W): thread t takes row t mod 128 and 8 consecutive k;
+  // tall (X = W^T): k = t mod 16 and 8 consecutive rows (W's contiguous dimension)
+  const int sr = mi.tall ? (t >> 4) * 8 : (t & 127);
+  const int sk = mi.tall ? (t & 15) : (t >> 7) * 8;
+  float ra[8], rb[8];
+  auto fetch = [&](int k0) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) acc[q][w] = 0.0;
-  for (int k0 = 0; k0 < mi.n; k0 += kGramK) {
-    // stage X[i0 + r][k0 + k] and X[j0 + r][k0 + k] as [k][r]; the global
-    // reads run along W's contiguous dimension
-    for (int e = t; e < kGramTile * kGramK; e += kEThreads) {
-      int r, k;
-      if (mi.tall) {
-        k = e >> 6;
-        r = e & 63;
-      } else {
-        r = e >> 5;
-        k = e & 31;
-      }
-      As[k][r] = x_at(W, mi, i0 + r, k0 + k);
-      Bs[k][r] = x_at(W, mi, j0 + r, k0 + k);
+    for (int q = 0; q < 8; ++q) {
+      const int r = mi.tall ? sr + q : sr, k = mi.tall ? sk : sk + q;
+      ra[q] = x_at(W, mi, i0 + r, k0 + k);
+      rb[q] = x_at(W, mi, j0 + r, k0 + k);
     }
-    __syncthreads();
-#pragma unroll 8
+  };
+  auto stash = [&](int buf) {
+    double* A_ = As + buf * kGramK * kGramLd;
+    double* B_ = Bs + buf * kGramK * kGramLd;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int r = mi.tall ? sr + q : sr, k = mi.tall ? sk : sk + q;
+      A_[k * kGramLd + r] = static_cast<double>(ra[q]);
+      B_[k * kGramLd + r] = static_cast<double>(rb[q]);
+    }
+  };
+  double acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+  const int nchunks = (mi.n + kGramK - 1) / kGramK;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  for (int c = 0; c < nchunks; ++c) {
+    const int buf = c & 1;
+    if (c + 1 < nchunks) fetch((c + 1) * kGramK);
+    const double* A_ = As + buf * kGramK * kGramLd;
+    const double* B_ = Bs + buf * kGramK * kGramLd;
+#pragma unroll 4
     for (int k = 0; k < kGramK; ++k) {
-      double a[4], b[4];
+      double av[8], bv[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        a[q] = As[k][ty * 4 + q];
-        b[q] = Bs[k][tx + 16 * q];
+        const double2 a2 = *reinterpret_cast<const double2*>(A_ + k * kGramLd + ty * 8 + 2 * q);
+        av[2 * q] = a2.x;
+        av[2 * q + 1] = a2.y;
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int j = 0; j < 8; ++j) bv[j] = B_[k * kGramLd + tx + 16 * j];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[q][w] = fma(a[q], b[w], acc[q][w]);
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
     }
+    if (c + 1 < nchunks) stash(buf ^ 1);  // that buffer's readers passed the previous barrier
     __syncthreads();
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int w = 0; w < 4; ++w) Cs[ty * 4 + q][tx + 16 * w] = acc[q][w];
+    for (int j = 0; j < 8; ++j) Cs[(ty * 8 + i) * (kGramTile + 1) + tx + 16 * j] = acc[i][j];
   __syncthreads();
   double* g = G + mi.off_g;
   const size_t ld = static_cast<size_t>(mi.mp);
-  for (int e = t; e < kGramTile * kGramTile; e += kEThreads) {
-    const int r = e >> 6, c = e & 63;
-    g[(i0 + r) * ld + j0 + c] = Cs[r][c];
-    if (td.y != td.z) g[(j0 + r) * ld + i0 + c] = Cs[c][r];
+  for (int e = t; e < kGramTile * kGramTile; e += kGramThreads) {
+    const int r = e >> 7, c = e & 127;
+    if (i0 + r < mi.mp && j0 + c < mi.mp) g[(i0 + r) * ld + j0 + c] = Cs[r * (kGramTile + 1) + c];
+    if (td.y != td.z && j0 + r < mi.mp && i0 + c < mi.mp) g[(j0 + r) * ld + i0 + c] = Cs[c * (kGramTile + 1) + r];
   }
 }
 
@@ -724,7 +755,7 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
     mi.m = std::min(mi.rows, mi.cols);
     mi.n = std::max(mi.rows, mi.cols);
     mi.tall = mi.rows > mi.cols ? 1 : 0;
-    mi.mp = (mi.m + kGramTile - 1) / kGramTile * kGramTile;
+    mi.mp = (mi.m + kPad - 1) / kPad * kPad;
     mi.off_g = off_g;
     mi.off_vw = off_vw;
     mi.sv_off = sv;
@@ -733,7 +764,7 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
     sv += mi.m;
     pl->mp_max = std::max(pl->mp_max, mi.mp);
     pl->m_max = std::max(pl->m_max, mi.m);
-    const int nt = mi.mp / kGramTile;
+    const int nt = (mi.mp + kGramTile - 1) / kGramTile;
     for (int a = 0; a < nt; ++a)
       for (int b = 0; b <= a; ++b) tiles.push_back(make_int4(i, a, b, 0));
     for (int k = 0; k < mi.m; k += kBisThreads) bis.push_back(make_int2(i, k));
@@ -824,6 +855,8 @@ extern "C" muon_status_t muon_entropy_init(muon_entropy_plan_t* out, const int64
       cudaGetLastError();
     }
   }
+  ok = ok && cudaFuncSetAttribute(gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kGramSmem)) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(bisect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(2 * pl->m_max * sizeof(double))) == cudaSuccess;
   if (!ok) {
@@ -888,7 +921,7 @@ extern "C" muon_status_t muon_entropy_compute(muon_entropy_plan_t pl, const floa
   bool ok = cudaMemsetAsync(ctl.conv, 0, n * sizeof(int), st) == cudaSuccess &&
             cudaMemsetAsync(ctl.computed, 0, n * sizeof(int), st) == cudaSuccess;
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[0], st) == cudaSuccess;
-  if (ok) gram_kernel<<<pl->ntiles, kEThreads, 0, st>>>(pl->tiles_d, pl->mats_d, pl->wptr_d, pl->G);
+  if (ok) gram_kernel<<<pl->ntiles, kGramThreads, kGramSmem, st>>>(pl->tiles_d, pl->mats_d, pl->wptr_d, pl->G);
   if (ok && pl->profiling) ok = cudaEventRecord(pl->prof[1], st) == cudaSuccess;
   if (ok) {
     cudaLaunchConfig_t cfg = {};
