@@ -11,8 +11,8 @@
 // vectors, so G is reduced to a symmetric tridiagonal matrix T with the same
 // eigenvalues and those are found by bisection.  The path, all matrices of a
 // plan per launch:
-//   1. gram_kernel: G in fp64 on the CUDA cores (64 x 64 tiles of the lower
-//      triangle, each also written mirrored), zero-padded to m_pad, a
+//   1. gram_kernel: G in fp64 on the CUDA cores (128 x 128 tiles of the
+//      lower triangle, each also written mirrored), zero-padded to m_pad, a
 //      multiple of 64.  Products of fp32 entries are exact in fp64.
 //   2. tridiag_kernel, one CTA per matrix: Householder reduction
 //      Q^T G Q = T (Golub and Van Loan, "Matrix Computations", Sec. 8.3.1) in
