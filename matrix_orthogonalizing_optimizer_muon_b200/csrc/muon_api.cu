@@ -578,13 +578,45 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
     pl->split = split;
   }
   const int split = pl->split;
+  // ---- split N of the symmetric and X-update tiles: a plan whose launches
+  // hold at most half as many tiles as CTA pairs halves its tiles along N
+  // (256 -> 128 -> 64 columns) while the count still gives each pair at most
+  // one, so that more pairs share a latency-bound launch.  The Gram product
+  // of a K-split plan keeps its unsplit tiles.
+  int nsplit_sym = 0, nsplit_full = 0;
+  {
+    auto levels = [&](size_t count) {
+      int lv = 0;
+      while (lv < 2 && count * 2 <= static_cast<size_t>(pl->npairs)) {
+        ++lv;
+        count *= 2;
+      }
+      return lv;
+    };
+    nsplit_sym = levels(cnt_sym);
+    nsplit_full = levels(cnt_full);
+    if (const char* env = std::getenv("MUON_NSPLIT")) {  // diagnostic: force the levels (0, 1 or 2)
+      const int v = std::atoi(env);
+      if (v >= 0 && v <= 2) nsplit_sym = nsplit_full = v;
+    }
+  }
+  size_t cnt_sym_n = 0, cnt_full_n = 0;  // list sizes after the N split
+  for (int i = 0; i < n; ++i) {
+    const MatInfo& mi = pl->mats[i];
+    for_each_sym_tile(mi.m, [&](const TcTile& t) {
+      split_n(t, nsplit_sym, mi.m, [&](const TcTile&) { ++cnt_sym_n; });
+    });
+    for_each_full_tile(mi.rows, mi.cols, [&](const TcTile& t) {
+      split_n(t, nsplit_full, mi.cols, [&](const TcTile&) { ++cnt_full_n; });
+    });
+  }
   size_t cnt_red = 0;  // 32 x 32 blocks on or below the diagonal of every symmetric product
   if (split > 1)
     for (int i = 0; i < n; ++i) {
       const size_t b = (pl->mats[i].m + 31) / 32;
       cnt_red += b * (b + 1) / 2;
     }
-  const size_t fixed = fixed_bytes(cnt_sym, cnt_full, cnt_sym32, cnt_full32, cnt_chunk) +
+  const size_t fixed = fixed_bytes(cnt_sym_n, cnt_full_n, cnt_sym32, cnt_full32, cnt_chunk) +
                        round_up(cnt_red * sizeof(int4), 256) +
                        (split > 1 ? round_up(cnt_sym * split * sizeof(TcTile), 256) : 0);
 
@@ -679,7 +711,7 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
       const MatInfo& mi = pl->mats[i];
       for_each_sym_tile(mi.m, [&](TcTile t) {
         t.p = i;
-        sym.push_back(t);
+        split_n(t, nsplit_sym, mi.m, [&](const TcTile& piece) { sym.push_back(piece); });
         if (split > 1)
           for (int kp = 0; kp < split; ++kp) {  // the parts of a tile side by side
             t.kpart = kp;
@@ -688,7 +720,7 @@ muon_status_t muon_init_ex(muon_plan_t* out, const muon_param_t* params, int32_t
       });
       for_each_full_tile(mi.rows, mi.cols, [&](TcTile t) {
         t.p = i;
-        full.push_back(t);
+        split_n(t, nsplit_full, mi.cols, [&](const TcTile& piece) { full.push_back(piece); });
       });
       if (pl->fp32_ws) {
         for (int r0 = 0; r0 < mi.m; r0 += kT32)

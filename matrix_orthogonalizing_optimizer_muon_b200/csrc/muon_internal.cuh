@@ -188,6 +188,35 @@ inline void for_each_sym_tile(int m, F&& emit) {
   }
 }
 
+// A tile split along N into its first `half` columns (from c0) and the rest
+// (from c1), each a tile of its own with the same rows and flags, `levels`
+// times over.  The epilogue writes whole 32-column blocks, so only tiles
+// whose half is a multiple of 32 columns are split (a ragged edge tile may
+// stay whole), and tiles of 64 columns or fewer stay whole.  sym_block_mode
+// decides the writes from the output block alone, so the pieces write the
+// elements the whole tile wrote.  A piece is clipped to the product's
+// `ncols` columns, and a piece with none is dropped (the second block of a
+// diagonal pair may be the ragged last one).  Used for plans with too few
+// tiles to give every CTA pair one.
+template <class F>
+inline void split_n(const TcTile& t, int levels, int ncols, F&& emit) {
+  const int half = tile_n_mma(t.n_need) / 2;
+  if (levels <= 0 || t.n_need <= 64 || half % 32 != 0) {
+    emit(t);
+    return;
+  }
+  int need_a = t.n_need < half ? t.n_need : half;
+  if (need_a > ncols - t.c0) need_a = ncols - t.c0;
+  if (need_a > 0)
+    split_n(TcTile{t.p, need_a, t.flags, t.kpart, t.r0, t.r1, t.c0, t.c0 + tile_n_mma(need_a) / 2}, levels - 1,
+            ncols, emit);
+  int need_b = t.n_need - half;
+  if (need_b > ncols - t.c1) need_b = ncols - t.c1;
+  if (need_b > 0)
+    split_n(TcTile{t.p, need_b, t.flags, t.kpart, t.r0, t.r1, t.c1, t.c1 + tile_n_mma(need_b) / 2}, levels - 1,
+            ncols, emit);
+}
+
 // Tiles of a full [R, C] product (the X update): rows [r0, r0 + 256) on the
 // pair, columns [c0, c0 + 256) contiguous.
 template <class F>

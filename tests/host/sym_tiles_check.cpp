@@ -1,7 +1,8 @@
 // Host check of the symmetric-product tiling of the tensor-core path
-// (for_each_sym_tile and sym_block_mode, the functions the kernel uses).
+// (for_each_sym_tile, split_n and sym_block_mode, the functions the kernel
+// and the plan use).
 //
-// For every m in [1, 2100]:
+// For every m in [1, 2100], and for the tiles split along N 0, 1 and 2 times:
 //  - every tile has 1 <= n_need <= 256 columns, rows and staged B rows that
 //    start on a multiple of 16 elements (TMA alignment), and a contiguous
 //    tile's second half starts where its first ends;
@@ -10,7 +11,9 @@
 //    sym_block_mode writes cover each element (i, j), j <= i, of the lower
 //    triangle exactly once (a block written with its mirror covers (i, j)
 //    for all its elements, a diagonal block the elements with j <= i).
-// Prints "ok <tiles for m = 1408> <tiles for m = 2048>" or the first violation.
+// Prints "ok <tiles for m = 1408> <tiles for m = 2048>" (unsplit), then
+// "split <level> <tiles for m = 1408> <tiles for m = 2048>" per level, or the
+// first violation.
 #include "muon_internal.cuh"
 
 #include <cstdio>
@@ -18,12 +21,13 @@
 
 int main() {
   using namespace muon;
+  for (int level = 0; level <= 2; ++level) {
   int tiles_1408 = 0, tiles_2048 = 0;
   for (int m = 1; m <= 2100; ++m) {
     std::vector<unsigned char> cover(static_cast<size_t>(m) * m, 0);
     bool bad = false;
     int count = 0;
-    for_each_sym_tile(m, [&](const TcTile& t) {
+    for_each_sym_tile(m, [&](const TcTile& whole) { split_n(whole, level, m, [&](const TcTile& t) {
       ++count;
       const int n_mma = tile_n_mma(t.n_need), half = n_mma / 2;
       if (t.n_need < 1 || t.n_need > 256 || t.r0 % 16 || t.r1 % 16 || t.c0 % 16 || t.c1 % 16 || t.r0 >= m ||
@@ -58,7 +62,7 @@ int main() {
           }
         }
       }
-    });
+    }); });
     for (int r = 0; r < m && !bad; ++r)
       for (int c = 0; c <= r; ++c)
         if (cover[static_cast<size_t>(r) * m + c] != 1) {
@@ -70,6 +74,8 @@ int main() {
     if (m == 1408) tiles_1408 = count;
     if (m == 2048) tiles_2048 = count;
   }
-  std::printf("ok %d %d\n", tiles_1408, tiles_2048);
+  if (level == 0) std::printf("ok %d %d\n", tiles_1408, tiles_2048);
+  else std::printf("split %d %d %d\n", level, tiles_1408, tiles_2048);
+  }
   return 0;
 }

@@ -110,6 +110,38 @@ def test_split_k_gram_row_by_row(split, monkeypatch):
     assert max(errs.values()) <= TOL_O_BF16, errs
 
 
+@pytest.mark.parametrize("levels", [1, 2])
+@pytest.mark.parametrize("coeffs", [(0.0, 1.0, 0.0), (0.0, 0.0, 1.0)], ids=["gram_update", "poly"])
+def test_n_split_tiles_row_by_row(levels, coeffs, monkeypatch):
+    """The symmetric and X-update tiles split along N (256 -> 128 -> 64
+    columns), which plans with few tiles choose (one 2048 x 2048 matrix
+    splits its symmetric tiles once, one 1024 x 1024 matrix every list
+    twice); MUON_NSPLIT forces it here on the whole multi-shape plan.  Same
+    stale-workspace and row-by-row check as above."""
+    monkeypatch.setenv("MUON_NSPLIT", str(levels))
+    abc = tuple(f32(v) for v in coeffs)
+    plan = MuonPlan(SHAPES)
+    xs0 = [random_bf16(s, 1500 + k, scale=3.0)[0] for k, s in enumerate(SHAPES)]
+    plan.orthogonalize(xs0, [torch.empty(s, device="cuda") for s in SHAPES], ns_steps=1, coeffs=abc)
+    xs, hosts = [], []
+    for k, s in enumerate(SHAPES):
+        x, h = random_bf16(s, 1600 + k)
+        xs.append(x)
+        hosts.append(h)
+    outs = [torch.full(s, float("nan"), device="cuda") for s in SHAPES]
+    plan.orthogonalize(xs, outs, ns_steps=1, coeffs=abc)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    worst = {}
+    for s, h, o in zip(SHAPES, hosts, outs):
+        got, want = host64(o), orc.newton_schulz(h, 1, abc)
+        if s[0] > s[1]:
+            got, want = got.T, want.T
+        worst[s] = float(_row_errors(got, want).max())
+    assert max(worst.values()) <= TOL_ROW, worst
+    plan.close()
+
+
 def test_symmetric_tiles_five_iterations():
     """The method's five iterations on the same shapes, within the acceptance bound."""
     plan = MuonPlan(SHAPES)
