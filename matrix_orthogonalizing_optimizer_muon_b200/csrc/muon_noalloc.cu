@@ -158,13 +158,31 @@ extern "C" muon_status_t muon_orthogonalize_noalloc(const void* X_in, float* O_o
   TcTile sym[kNaMaxTiles], full[kNaMaxTiles];
   int nsym = 0, nfull = 0;
   bool fits = true;
-  for_each_sym_tile(mi.m, [&](const TcTile& t) {
-    if (nsym == kNaMaxTiles) fits = false;
-    else sym[nsym++] = t;
+  // as in a plan: a list with at most half as many tiles as CTA pairs is
+  // split along N while each pair still gets at most one tile
+  int cs = 0, cf = 0;
+  for_each_sym_tile(mi.m, [&](const TcTile&) { ++cs; });
+  for_each_full_tile(R, C, [&](const TcTile&) { ++cf; });
+  auto levels = [&](int count) {
+    int lv = 0;
+    while (lv < 2 && count * 2 <= g_state[dev].npairs) {
+      ++lv;
+      count *= 2;
+    }
+    return lv;
+  };
+  const int ls = levels(cs), lf = levels(cf);
+  for_each_sym_tile(mi.m, [&](const TcTile& whole) {
+    split_n(whole, ls, mi.m, [&](const TcTile& t) {
+      if (nsym == kNaMaxTiles) fits = false;
+      else sym[nsym++] = t;
+    });
   });
-  for_each_full_tile(R, C, [&](const TcTile& t) {
-    if (nfull == kNaMaxTiles) fits = false;
-    else full[nfull++] = t;
+  for_each_full_tile(R, C, [&](const TcTile& whole) {
+    split_n(whole, lf, C, [&](const TcTile& t) {
+      if (nfull == kNaMaxTiles) fits = false;
+      else full[nfull++] = t;
+    });
   });
   if (!fits) return MUON_ERR_UNSUPPORTED;
   MatPtrs mp{};
