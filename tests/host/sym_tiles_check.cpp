@@ -77,5 +77,37 @@ int main() {
   if (level == 0) std::printf("ok %d %d\n", tiles_1408, tiles_2048);
   else std::printf("split %d %d %d\n", level, tiles_1408, tiles_2048);
   }
+  // The X-update tiles (for_each_full_tile), split 0, 1 and 2 times: walking
+  // each CTA's 128 rows and the accumulator's 32-column chunks as the
+  // epilogue does (rows and columns past the product masked), every element
+  // of the R x C output is written exactly once.
+  for (int level = 0; level <= 2; ++level) {
+    for (int R = 1; R <= 700; R += 23)
+      for (int C = 1; C <= 1100; C += 37) {
+        std::vector<unsigned char> cover(static_cast<size_t>(R) * C, 0);
+        bool bad = false;
+        for_each_full_tile(R, C, [&](const TcTile& whole) { split_n(whole, level, C, [&](const TcTile& t) {
+          const int half = tile_n_mma(t.n_need) / 2;
+          if (t.n_need < 1 || t.n_need > 256 || t.c0 % 16 || t.c1 % 16 || t.c0 >= C) {
+            std::printf("R=%d C=%d: tile (%d %d | %d %d, %d) malformed\n", R, C, t.r0, t.r1, t.c0, t.c1, t.n_need);
+            bad = true;
+            return;
+          }
+          for (int rank = 0; rank < 2; ++rank)
+            for (int i = rank ? t.r1 : t.r0, e = i + 128; i < e && i < R; ++i)
+              for (int cc = 0; cc < t.n_need; ++cc) {
+                const int j = cc < half ? t.c0 + cc : t.c1 + (cc - half);
+                if (j < C && ++cover[static_cast<size_t>(i) * C + j] > 1) bad = true;
+              }
+        }); });
+        for (size_t k = 0; k < cover.size() && !bad; ++k)
+          if (cover[k] != 1) bad = true;
+        if (bad) {
+          std::printf("full tiles R=%d C=%d split %d: an element not written exactly once\n", R, C, level);
+          return 1;
+        }
+      }
+  }
+  std::printf("full ok\n");
   return 0;
 }

@@ -1,5 +1,5 @@
 """The symmetric-product tiling of the tensor-core path, checked on the host:
-the real header functions (for_each_sym_tile, split_n, sym_block_mode), compiled with
+the real header functions (for_each_sym_tile, for_each_full_tile, split_n, sym_block_mode), compiled with
 g++ against csrc/muon_internal.cuh (no GPU), walked the way the epilogue
 walks a tile.  See tests/host/sym_tiles_check.cpp for the properties."""
 
@@ -24,4 +24,4 @@ def test_sym_tile_list_covers_the_lower_triangle_once(tmp_path):
     assert out.returncode == 0, out.stdout
     # 1408 = 11 blocks of 128 rows: 10 + 5 + 3 tiles; 2048 = 16 blocks: 28 + 8 tiles;
     # split along N once every 256-column tile becomes two, twice four
-    assert out.stdout.strip().splitlines() == ["ok 18 36", "split 1 36 72", "split 2 72 144"]
+    assert out.stdout.strip().splitlines() == ["ok 18 36", "split 1 36 72", "split 2 72 144", "full ok"]
