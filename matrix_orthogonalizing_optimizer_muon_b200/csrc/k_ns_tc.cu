@@ -559,10 +559,14 @@ __device__ __forceinline__ void load_row32_masked(const __nv_bfloat16* src, int 
   for (int q = 0; q < 4; ++q) out[q] = reinterpret_cast<const uint4*>(h)[q];
 }
 
-// element q (0..31) of a packed 32-value bf16 row segment
+// element q (0..31) of a packed 32-value bf16 row segment, as a float and as its bits
 __device__ __forceinline__ float bf_at(const uint4 (&p)[4], int q) {
   const uint32_t w = reinterpret_cast<const uint32_t*>(&p[q >> 3])[(q & 7) >> 1];
   return __uint_as_float((q & 1) ? (w & 0xFFFF0000u) : (w << 16));
+}
+__device__ __forceinline__ unsigned short bf_bits(const uint4 (&p)[4], int q) {
+  const uint32_t w = reinterpret_cast<const uint32_t*>(&p[q >> 3])[(q & 7) >> 1];
+  return static_cast<unsigned short>((q & 1) ? (w >> 16) : (w & 0xFFFFu));
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -985,10 +989,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 32; ++q) val[q] = first ? (u2f(v[q]) * s) * s : u2f(v[q]);
         } else {
-          // B' = b A + c A A + a I (the a X term of the update rides on B' hi)
+          // B' = b A + c A A + a I (the a X term of the update rides on B' hi);
+          // only a block that starts on the diagonal holds diagonal elements
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q)) + (j0 + q == i ? a_c : 0.0f);
+          for (int q = 0; q < 32; ++q) val[q] = fmaf(c_c, u2f(v[q]), b_c * bf_at(xa, q));
+          if (j0 == i_lo) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q == lane) val[q] += a_c;
+          }
         }
         // symmetric products
         __align__(16) __nv_bfloat16 h[32];
@@ -1002,9 +1011,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
           const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
           publish(map, j0, i_lo, map, i_lo, j0);
+        } else if (inside) {
+          // diagonal block (j0 == i_lo): the diagonal and the part below it
+          // from this thread's row, the part above from the transpose, so
+          // the block is stored exactly symmetric, whole, in one bulk store
+          staging_free();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
+          __syncwarp();
+          uint4 tr[4];  // row `lane` of the transpose: element q is (j0 + q, i)
+          read_row32(blk1, lane, tr);
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (q > lane) h[q] = __ushort_as_bfloat16(bf_bits(tr, q));
+          write_row32(blk0, lane, h);
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB), blk0_s, j0, i_lo);
+            bulk_commit();
+          }
         } else {
-          // diagonal or ragged block: element-wise with masks (a ragged
-          // block below the diagonal is written whole, with its mirror)
+          // ragged block (past the edge of the product): element-wise with
+          // masks; below the diagonal it is written whole, with its mirror
           const bool whole = (md == 1);
           __nv_bfloat16* out = (g.phase == kPhaseGram ? g.ws.A : g.ws.B) + mi.off_a;
           __nv_bfloat16* row = out + static_cast<size_t>(i) * mi.lda;
