@@ -506,22 +506,12 @@ __device__ __forceinline__ void write_row32(uint8_t* blk, int r, const __nv_bflo
   for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(blk + chunk_off(r, q)) = reinterpret_cast<const uint4*>(h)[q];
 }
 
-// Coalesced read of a 32 x 32 bf16 block src[(g_row0 + rr) * ld + g_col0 + cc]
-// into registers: lane l holds rows 8k + l/4, 16-byte chunk l % 4.
-__device__ __forceinline__ void load_block32(const __nv_bfloat16* src, int ld, int g_row0, int g_col0, int lane,
-                                             uint4 (&out)[4]) {
-  const int c16 = lane & 3;
+// This thread's row segment src[row * ld + col0 .. + 32), 64 contiguous bytes,
+// through the read-only path (the array is not written during the launch).
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int ld, int row, int col0, uint4 (&out)[4]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * ld + col0);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int rr = 8 * k + (lane >> 2);
-    out[k] = __ldcg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(g_row0 + rr) * ld + g_col0 + c16 * 8));
-  }
-}
-
-__device__ __forceinline__ void put_block32(uint8_t* blk, int lane, const uint4 (&in)[4]) {
-  const int c16 = lane & 3;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(blk + chunk_off(8 * k + (lane >> 2), c16)) = in[k];
+  for (int q = 0; q < 4; ++q) out[q] = __ldg(p + q);
 }
 
 // Asynchronous (cp.async, no registers) copy of a 32 x 32 bf16 block
@@ -567,6 +557,40 @@ __device__ __forceinline__ float bf_at(const uint4 (&p)[4], int q) {
 __device__ __forceinline__ unsigned short bf_bits(const uint4 (&p)[4], int q) {
   const uint32_t w = reinterpret_cast<const uint32_t*>(&p[q >> 3])[(q & 7) >> 1];
   return static_cast<unsigned short>((q & 1) ? (w >> 16) : (w & 0xFFFFu));
+}
+
+// bf16 pair (x in the low half, y in the high half) as one word
+__device__ __forceinline__ uint32_t pack_bf2(float x, float y) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// X-update row segment: val = alpha (a lo + acc) for the 32 columns of this
+// thread's row (alpha = s when kScaled, else 1), split into hi = bf16(val) and
+// lo = bf16(val - hi), staged in blk_hi / blk_lo
+template <bool kScaled>
+__device__ __forceinline__ void upd_stage_row(const uint32_t (&v)[32], const uint4 (&xa)[4], float a_c, float s,
+                                              uint8_t* blk_hi, uint8_t* blk_lo, int lane) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = 8 * q4 + 2 * u;
+      const uint32_t xw = reinterpret_cast<const uint32_t*>(&xa[q4])[u];  // lo of columns q, q + 1
+      float v0 = fmaf(a_c, __uint_as_float(xw << 16), __uint_as_float(v[q]));
+      float v1 = fmaf(a_c, __uint_as_float(xw & 0xFFFF0000u), __uint_as_float(v[q + 1]));
+      if (kScaled) {
+        v0 *= s;
+        v1 *= s;
+      }
+      const uint32_t hb = pack_bf2(v0, v1);
+      hw[u] = hb;
+      lw[u] = pack_bf2(v0 - __uint_as_float(hb << 16), v1 - __uint_as_float(hb & 0xFFFF0000u));
+    }
+    *reinterpret_cast<uint4*>(blk_hi + chunk_off(lane, q4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(blk_lo + chunk_off(lane, q4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -833,16 +857,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto block_inside = [&](int ch) {
         return i_lo + 31 < rows_in && c.col(ch * kEpiBoxCols) + 32 <= cols_in;
       };
-      // polynomial: coalesced prefetch of an A block into registers; pf_ch
-      // is the chunk whose block pf0 holds (a tile may skip chunks and need
-      // later ones, so the next needed chunk is looked up, not assumed)
+      // polynomial: prefetch of this thread's row of the next A block into
+      // registers; pf_ch is the chunk whose row pf0 holds (a tile may skip
+      // chunks and need later ones, so the next needed chunk is looked up,
+      // not assumed)
       uint4 pf0[4];
       int pf_ch = -1;
       auto prefetch_from = [&](int from) {
         if (!poly) return;
         for (int nx = from; nx < c.nch; nx += kEpiGroups)
           if (needed(nx) && block_inside(nx)) {
-            load_block32(in0, ld_in, i_lo, c.col(nx * kEpiBoxCols), lane, pf0);
+            load_row32(in0, ld_in, i, c.col(nx * kEpiBoxCols), pf0);
             pf_ch = nx;
             return;
           }
@@ -905,12 +930,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         } else if (poly) {
           if (inside) {
-            if (pf_ch != ch) load_block32(in0, ld_in, i_lo, j0, lane, pf0);  // fallback; prefetch_from lands here
-            staging_free();
-            put_block32(blk0, lane, pf0);
-            __syncwarp();
-            read_row32(blk0, lane, xa);
-            __syncwarp();
+            if (pf_ch != ch) load_row32(in0, ld_in, i, j0, pf0);  // fallback; prefetch_from lands here
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xa[q] = pf0[q];
           } else {
             load_row32_masked(in0, ld_in, rows_in, cols_in, i, j0, xa);
           }
@@ -948,19 +970,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float alpha = (g.iter == 0) ? s : 1.0f;
           if (inside) {
             staging_free();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              __align__(16) __nv_bfloat16 h8[8];
-              __align__(16) __nv_bfloat16 l8[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const float val = alpha * fmaf(a_c, bf_at(xa, 8 * q4 + u), u2f(v[8 * q4 + u]));
-                h8[u] = __float2bfloat16_rn(val);
-                l8[u] = __float2bfloat16_rn(val - __bfloat162float(h8[u]));
-              }
-              *reinterpret_cast<uint4*>(blk0 + chunk_off(lane, q4)) = *reinterpret_cast<const uint4*>(h8);
-              *reinterpret_cast<uint4*>(blk1 + chunk_off(lane, q4)) = *reinterpret_cast<const uint4*>(l8);
-            }
+            // two columns per step: their lo inputs share a word, and each
+            // rounding to bf16 converts the pair at once
+            if (g.iter == 0)
+              upd_stage_row<true>(v, xa, a_c, s, blk0, blk1, lane);
+            else
+              upd_stage_row<false>(v, xa, a_c, s, blk0, blk1, lane);
             // blk1 follows blk0: one 3-D store writes the hi block and the lo block
             fence_proxy_async();
             __syncwarp();
