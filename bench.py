@@ -436,6 +436,101 @@ def hybrid_mixed8(dev, steps: int = 5, warmup: int = 3):
             "ns_ms_per_step": gemm_ms, "ns_tflops": nz / (gemm_ms * 1e-3) / 1e12}
 
 
+def other_workloads(dev, peak: float, reps: int = 10, steps: int = 10, warmup: int = 3):
+    """The Newton-Schulz size sweep and the 16-layer dense stack, timed in the
+    same process after the main timed region (CUDA events; Newton-Schulz time
+    from the span profile).  Sweep: one plan per shape, a bf16 input of rank
+    64 with singular scales decaying geometrically from 1 to 1e-3 plus noise
+    (the workload recipe, drawn on the device), 5 iterations per call.  Dense
+    stack: full Muon steps over its 96 matrices on resident synthetic inputs.
+    Each case warms up for about 50 ms and times at least `reps` (`steps`)
+    calls and about 100 ms."""
+    import torch
+    from matrix_orthogonalizing_optimizer_muon_b200 import workloads as wlm
+    from matrix_orthogonalizing_optimizer_muon_b200.api import MuonPlan
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321)
+
+    cur_plan = []
+
+    def prof_on():
+        cur_plan[-1].profile(True, spans=True)
+        cur_plan[-1].profile_read()
+
+    def timed(fn, n):
+        # warm up for about 50 ms and time at least n calls and about 100 ms,
+        # so that a short call is not timed while the clock still recovers
+        # from the previous, heavier workload
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(warmup):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        est = max(e0.elapsed_time(e1) / warmup, 1e-3)
+        for _ in range(int(50.0 / est)):
+            fn()
+        n = max(n, int(100.0 / est))
+        torch.cuda.synchronize()
+        prof_on()
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, n
+
+    sweep = []
+    k = wlm.LOWRANK_RANK
+    sig = wlm.LOWRANK_SIGMA_MIN ** (torch.arange(k, device=dev, dtype=torch.float32) / (k - 1))
+    for r, c in wlm.NS_SWEEP_SHAPES:
+        P = torch.randn((r, k), device=dev, generator=gen) * sig
+        Q = torch.randn((c, k), device=dev, generator=gen)
+        x = (P @ Q.T + wlm.LOWRANK_NOISE_STD * torch.randn((r, c), device=dev, generator=gen)).to(torch.bfloat16)
+        o = torch.empty((r, c), device=dev)
+        plan = MuonPlan([(r, c)])
+        cur_plan.append(plan)
+        ms, n = timed(lambda: plan.orthogonalize([x], [o]), reps)
+        prof = plan.profile_read()
+        st = plan.status()
+        plan.close()
+        ns_ms = prof["ms"]["newton_schulz"] / max(prof["calls"], 1)
+        tf = ns_flops(r, c, 5) / (ns_ms * 1e-3) / 1e12
+        sweep.append({"shape": f"{r}x{c}", "ms_per_call": ms, "calls": n, "ns_ms": ns_ms, "ns_tflops": tf,
+                      "frac": tf / peak, "status": st})
+        del P, Q, x, o
+
+    wl = wlm.llama16()
+    shapes = [(r, c) for _, r, c in wl.shapes]
+    sizes = [r * c for r, c in shapes]
+    total = sum(sizes)
+    Wbuf = torch.empty(total, device=dev).normal_(0.0, 0.02, generator=gen)
+    Gbuf = torch.empty(total, device=dev).normal_(0.0, 1e-3, generator=gen).to(torch.bfloat16)
+    Mbuf = torch.empty(total, device=dev)
+    params, off = [], 0
+    for (r, c), e in zip(shapes, sizes):
+        params.append((Wbuf[off:off + e].view(r, c), Gbuf[off:off + e].view(r, c), Mbuf[off:off + e].view(r, c)))
+        off += e
+    plan = MuonPlan(shapes, momenta=[m for _, _, m in params])
+    cur_plan.append(plan)
+    plan.bind(params)
+    hp = dict(lr=4.2e-4, weight_decay=0.1, momentum=0.95, ns_steps=5)
+    ms, n = timed(lambda: plan.step(**hp), steps)
+    prof = plan.profile_read()
+    st = plan.status()
+    plan.close()
+    ns_ms = prof["ms"]["newton_schulz"] / max(prof["calls"], 1)
+    tf = sum(ns_flops(r, c, 5) for r, c in shapes) / (ns_ms * 1e-3) / 1e12
+    del params, Wbuf, Gbuf, Mbuf
+    torch.cuda.empty_cache()
+    return {"what": "Newton-Schulz size sweep (orthogonalize, one matrix per plan) and the 16-layer dense stack "
+                    "(Muon steps over 96 matrices), same process after the main timed region; frac of the same "
+                    "peak as the roofline",
+            "ns_sweep": sweep,
+            "llama16": {"matrices": len(shapes), "ms_per_step": ms, "ns_ms_per_step": ns_ms, "ns_tflops": tf,
+                        "frac": tf / peak, "steps": n, "status": st}}
+
+
 def run_reference(args, wl, rank: int):
     if rank != 0:
         return
@@ -499,6 +594,8 @@ def main(argv=None) -> int:
                     help="skip the hybrid Muon + AdamW step of the 1624-matrix mixed model")
     ap.add_argument("--no-ceiling", action="store_true",
                     help="skip the library batched-GEMM context point of the three product shapes")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the Newton-Schulz size sweep and the 16-layer dense stack")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -711,7 +808,8 @@ def main(argv=None) -> int:
 
     adamw = None
     hybrid = None
-    if not (args.no_adamw and args.no_hybrid):
+    others = None
+    if not (args.no_adamw and args.no_hybrid and args.no_others):
         plan.close()
         del Wbuf, Gbuf, Mbuf, Ws, Gs, Ms, params
         torch.cuda.empty_cache()
@@ -719,6 +817,8 @@ def main(argv=None) -> int:
             adamw = bench_adamw(dev)
         if not args.no_hybrid:
             hybrid = hybrid_mixed8(dev)
+        if not args.no_others:
+            others = other_workloads(dev, peak)
 
     cpu = None
     if world == 1 and args.cpu_budget > 0:
@@ -764,6 +864,7 @@ def main(argv=None) -> int:
         "context_torch_eager_ns": context,
         "context_library_batched_gemm": ceiling,
         "hybrid_step_mixed8": hybrid,
+        "other_workloads": others,
         "adamw_companion": adamw,
         "svd_entropy": entropy,
         "e2e": e2e,
