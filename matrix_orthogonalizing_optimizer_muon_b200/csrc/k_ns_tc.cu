@@ -66,9 +66,6 @@ constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;      // 32 KiB
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpEpi0 = 2;
 // Producer warps: warp 0 and the warps after the epilogue; fill f of the
 // stage ring goes to producer f mod kProducers.
-#ifndef MUON_TC_PF_DIST
-#define MUON_TC_PF_DIST 0
-#endif
 #ifndef MUON_TC_PRODUCERS
 #define MUON_TC_PRODUCERS 2
 #endif
@@ -238,12 +235,6 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* tmap, in
       "%3}], [%4];" ::"r"(dst),
       "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
-}
-
-// L2 prefetch of one box (no shared memory, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_l2(const void* tmap, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
-               : "memory");
 }
 
 // Bring a tensor map into the TMA descriptor cache ahead of its first use.
@@ -721,14 +712,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int mn0 = (is_a ? arow : brow) + h * kBoxInner;
           const uint32_t dst = (is_a ? sa : sb) + h * kBox64Bytes;
           tma_load_pair(dst, o.tmap, o.mn ? mn0 : k0, o.mn ? k0 : mn0 - h * kBoxInner, fb);
-#if MUON_TC_PF_DIST > 0
-          // bring the box MUON_TC_PF_DIST stages ahead into L2, so that its load
-          // later finds it there rather than in HBM
-          if (kb + MUON_TC_PF_DIST < c.nk) {
-            const int kp = k0 + MUON_TC_PF_DIST * kBK;
-            tma_prefetch_l2(o.tmap, o.mn ? mn0 : kp, o.mn ? kp : mn0 - h * kBoxInner);
-          }
-#endif
         }
       }
       if (!ok) break;
