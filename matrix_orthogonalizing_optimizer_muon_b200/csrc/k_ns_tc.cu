@@ -556,6 +556,22 @@ __device__ __forceinline__ uint32_t pack_bf2(float x, float y) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Staged transpose of a 32 x 32 bf16 block: row q, column t of `blk` gets
+// element q of lane t's row (hw holds the row as 16 packed pairs).  Each
+// pair of neighbouring lanes swaps a word, so that every lane stores whole
+// words: an even lane t the pair (t, t + 1) of row q = 2u, an odd lane the
+// pair (t - 1, t) of row 2u + 1; one store covers two rows, all 32 banks.
+__device__ __forceinline__ void stage_transpose(uint8_t* blk, int lane, const uint32_t (&hw)[16]) {
+  const int odd = lane & 1;
+  const uint32_t sel = odd ? 0x3276u : 0x5410u;  // odd: high halves (nb, own); even: low halves (own, nb)
+  const int le = lane & ~1;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const uint32_t nb = __shfl_xor_sync(0xffffffffu, hw[u], 1);
+    *reinterpret_cast<uint32_t*>(blk + swz64(2 * u + odd, le)) = __byte_perm(hw[u], nb, sel);
+  }
+}
+
 // X-update row segment: val = alpha (a lo + acc) for the 32 columns of this
 // thread's row (alpha = s when kScaled, else 1), split into hi = bf16(val) and
 // lo = bf16(val - hi), staged in blk_hi / blk_lo
@@ -998,15 +1014,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         // symmetric products
-        __align__(16) __nv_bfloat16 h[32];
+        __align__(16) uint32_t hw[16];  // this thread's row, packed pairs
 #pragma unroll
-        for (int q = 0; q < 32; ++q) h[q] = __float2bfloat16_rn(val[q]);
+        for (int u = 0; u < 16; ++u) hw[u] = pack_bf2(val[2 * u], val[2 * u + 1]);
+        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(hw);
         if (inside && md == 1) {
           // off-diagonal block: stage it and its transpose, store both
           staging_free();
           write_row32(blk0, lane, h);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
+          stage_transpose(blk1, lane, hw);
           const void* map = tmap_of(g, c.p, g.phase == kPhaseGram ? kMapStA : kMapStB);
           publish(map, j0, i_lo, map, i_lo, j0);
         } else if (inside) {
@@ -1014,8 +1030,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // from this thread's row, the part above from the transpose, so
           // the block is stored exactly symmetric, whole, in one bulk store
           staging_free();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) *reinterpret_cast<__nv_bfloat16*>(blk1 + swz64(q, lane)) = h[q];
+          stage_transpose(blk1, lane, hw);
           __syncwarp();
           uint4 tr[4];  // row `lane` of the transpose: element q is (j0 + q, i)
           read_row32(blk1, lane, tr);
