@@ -87,10 +87,14 @@ class MuonPlan:
     def bind(self, params):
         """Fill the descriptor array from [(W, G, M), ...].  The last few
         distinct bindings are kept, so alternating between buffer sets (double
-        buffered gradients) costs no re-validation."""
+        buffered gradients) costs no re-validation.  A binding is reused only
+        when every tensor has the same address, shape, dtype and contiguity
+        (which fix its layout), so another tensor or a view at a cached
+        address is validated afresh."""
         if len(params) != self.n:
             raise ValueError(f"expected {self.n} (W, G, M) triples, got {len(params)}")
-        key = tuple((W.data_ptr(), G.data_ptr(), M.data_ptr(), G.dtype) for W, G, M in params)
+        key = tuple((W.data_ptr(), G.data_ptr(), M.data_ptr(), W.shape, G.shape, M.shape, W.dtype, G.dtype, M.dtype,
+                     W.is_contiguous(), G.is_contiguous(), M.is_contiguous()) for W, G, M in params)
         if key == self._key:
             return
         cached = self._bound.get(key)

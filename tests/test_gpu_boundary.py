@@ -220,3 +220,23 @@ def test_zero_input_after_nonzero_gives_exact_zero_output():
     torch.cuda.synchronize()
     assert all(torch.equal(o, torch.zeros_like(o)) for o in outs)
     plan.close()
+
+
+def test_cached_binding_does_not_skip_validation_of_a_view():
+    """A binding is reused only for the same addresses, shapes, dtypes and
+    contiguity: a transposed view of a square tensor at a cached address, or
+    a gradient of another dtype there, is validated again and rejected."""
+    s = (64, 64)
+    plan = MuonPlan([s])
+    W = torch.zeros(s, device="cuda")
+    G = torch.zeros(s, device="cuda", dtype=torch.bfloat16)
+    M = torch.zeros(s, device="cuda")
+    plan.bind([(W, G, M)])
+    with pytest.raises(ValueError):
+        plan.bind([(W.t(), G, M)])  # same address and shape, not contiguous
+    with pytest.raises(TypeError):
+        plan.bind([(W, G.view(torch.float16), M)])  # same address and shape, another dtype
+    plan.bind([(W, G, M)])  # the cached binding is still good
+    plan.step(lr=LR, weight_decay=WD, momentum=MU)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
