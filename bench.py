@@ -77,7 +77,12 @@ def ncu_summary(workload: str):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock and throttle-reason samples of one GPU, kept for the
+    timed region only.  start() launches the sampler and waits for its first
+    sample (starting nvidia-smi can take longer than a short timed region);
+    mark_start() and mark_end() bracket the region, and samples whose
+    timestamps fall outside it (warm-up, tail) are dropped."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -85,18 +90,30 @@ class ClockSampler:
         self.gpu = gpu_index
         self.interval_ms = interval_ms
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self, wait_s: float = 5.0):
+        import select
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return self
+        ready, _, _ = select.select([self.proc.stdout], [], [], wait_s)
+        if ready:  # raw read: stop() collects the rest from the same descriptor
+            self.lines += os.read(self.proc.stdout.fileno(), 1 << 16).decode(errors="replace").splitlines()
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -104,7 +121,22 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.lines += out.splitlines()
+            self.proc = None
+        self.lines = [ln for ln in self.lines if ln.strip()]
+
+    def in_region(self, ts: str) -> bool:
+        """Whether a sample's timestamp lies in the marked region (with one
+        sampling interval of slack at either end); unmarked regions and
+        unparsable timestamps keep the sample."""
+        if self.t0 is None or self.t1 is None:
+            return True
+        try:
+            t = datetime.datetime.strptime(ts.strip(), "%Y/%m/%d %H:%M:%S.%f")
+        except ValueError:
+            return True
+        slack = datetime.timedelta(milliseconds=self.interval_ms)
+        return self.t0 - slack <= t <= self.t1 + slack
 
     def summary(self):
         """Median SM clock under load (samples with power above 400 W, the
@@ -114,10 +146,11 @@ class ClockSampler:
         counts = {}
         loaded = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10 or not self.in_region(f[0]):
                 continue
+            f = f[1:]  # index, clocks, power, reasons
             try:
                 sm.append(float(f[1]))
                 mx.append(float(f[2]))
@@ -658,11 +691,20 @@ def main(argv=None) -> int:
         if dist is not None:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        plan.step(**hp, update_rms=rms)
-    torch.cuda.synchronize()
+    # the clock sampler runs from before the warm-up, so that its first
+    # sample is in hand when the timed region starts; only samples inside the
+    # region are kept
+    clk = ClockSampler(local).start()
+    try:
+        for _ in range(args.warmup):
+            plan.step(**hp, update_rms=rms)
+        torch.cuda.synchronize()
+    except BaseException:
+        clk.stop()
+        raise
     st = plan.status()
     if st != 0:
+        clk.stop()
         raise RuntimeError(f"device status {st} after warm-up")
 
     # ---- timed region: inputs resident in HBM
@@ -680,7 +722,8 @@ def main(argv=None) -> int:
     # median is reported beside the mean); a boundary event sits between two
     # steps, not inside the Newton-Schulz chain
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
-    with ClockSampler(local) as clk:
+    try:
+        clk.mark_start()
         ev0.record(stream)
         for k in range(args.steps):
             plan.step(**hp, update_rms=rms)
@@ -688,6 +731,9 @@ def main(argv=None) -> int:
                 step_ev[k].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
+    finally:
+        clk.stop()
     bounds = [ev0] + step_ev + [ev1]
     step_ms = sorted(bounds[k].elapsed_time(bounds[k + 1]) for k in range(args.steps))
     half = len(step_ms) // 2

@@ -93,3 +93,30 @@ def test_entropy_trailing_byte_count():
         want = sum(8 * (m - 1 - j) ** 2 for j in range(m - 1))
         assert bench.entropy_trailing_bytes([shape]) == want
     assert bench.entropy_trailing_bytes([(3, 4), (5, 2)]) == 8 * (4 + 1) + 8 * 1
+
+
+def test_clock_sampler_keeps_the_timed_region_only():
+    """Samples of nvidia-smi's CSV (timestamp first) outside the marked region
+    (warm-up before it, the tail after it) are dropped; the median counts
+    samples under load only; without a sampler the record says unavailable."""
+    import datetime as dt
+    c = bench.ClockSampler(0, interval_ms=25)
+    t0 = dt.datetime(2026, 1, 2, 3, 4, 5, 0)
+    c.t0, c.t1 = t0, t0 + dt.timedelta(milliseconds=300)
+
+    def line(ms, mhz, watts, cap):
+        ts = (t0 + dt.timedelta(milliseconds=ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {mhz}, 1965, {watts}, 0x4, Not Active, Not Active, Not Active, {cap}"
+
+    c.lines = [line(-500, 1965, 700.0, "Not Active"),       # warm-up: dropped
+               line(-10, 1900, 650.0, "Not Active"),        # within one interval of the start: kept
+               line(100, 1400, 990.0, "Active"),
+               line(200, 1420, 995.0, "Active"),
+               line(250, 1500, 300.0, "Not Active"),        # not under load: not in the median
+               line(900, 1965, 250.0, "Not Active")]        # after the region: dropped
+    s = c.summary()
+    assert s["samples"] == 4 and s["samples_under_load"] == 3
+    assert s["sm_mhz"] == 1420.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["reason_samples"] == {"sw_power_cap": 2}
+    empty = bench.ClockSampler(0)
+    assert empty.summary()["reasons"] == ["unavailable"]
